@@ -1,0 +1,31 @@
+"""B200-native Monarch attention forward (MonarchRT).
+
+    out = P^T B2 P B1 V
+
+over a video token grid N = T*H*W: stage 1 is softmax attention inside each
+frame (or spatial tile of a frame), stage 2 is softmax attention across frames
+at each spatial position, applied to stage 1's output.  Every step runs in
+hand-written sm_100a CUDA kernels behind a C ABI (``include/monarch_attn.h``);
+this package is the thin ctypes binding over it.
+
+The binding is imported lazily so that ``workloads`` (seeded inputs) can be
+used without loading the CUDA library.
+"""
+
+__all__ = [
+    "monarch_attn_fwd", "monarch_attn_fwd_host", "MonarchError", "lib_path",
+    "FACT_FRAME", "FACT_TILED", "DTYPE_F32", "DTYPE_BF16",
+]
+
+FACT_FRAME = 0
+FACT_TILED = 1
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
+
+def __getattr__(name):
+    if name in ("monarch_attn_fwd", "monarch_attn_fwd_host", "MonarchError", "lib_path",
+                "load_library", "strerror", "last_device_error"):
+        from . import binding
+        return getattr(binding, name)
+    raise AttributeError(name)

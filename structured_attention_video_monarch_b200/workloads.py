@@ -1,0 +1,151 @@
+"""Seeded synthetic workloads for the Monarch attention forward.
+
+This module holds the five workload shapes and the seeded input recipes.  It
+contains none of the operator's arithmetic: it only draws random tensors, so
+both the CUDA path (tests, bench) and the fp64 oracle's tests can use it.
+
+The pages (MonarchRT: Efficient Attention for Real-Time Video Generation,
+gist.science/zh/paper/2602.12271, section 4 "Results") measure kernel latency
+at 720p and end-to-end generation with Self-Forcing at 480p but print no
+tensor shapes; these synthetic shapes stand in for those workloads:
+a Wan-style latent grid of 30x52 (480p) or 45x80 (720p) tokens per frame,
+21 latent frames per clip, 12 heads of width 128.
+
+Recipe (every draw on a CPU ``torch.Generator`` seeded with the workload's
+index, fp32 draws in the order Q, K, V, then extras, then cast):
+  0 tiny_fp32     Q, K, V iid N(0,1) * d^-1/2, kept fp32.
+  1 chunk_bf16    Q, K, V iid N(0,1).
+  2 fullclip_bf16 Q, K, V iid N(0,1); then R (8 x d) iid N(0,1) and the
+                  shared positional term 0.5 * u(n) R added to Q and K, where
+                  u(n) = [cos 2pi t/T, sin 2pi t/T, cos 2pi h/H, sin 2pi h/H,
+                  cos 2pi w/W, sin 2pi w/W, cos 2pi(h/H+w/W), sin 2pi(h/H+w/W)]
+                  (periodic and separable, like the positional part of the
+                  attention map the pages describe; unit variance per entry).
+  3 tiled_bf16    Q, K, V iid N(0,1).
+  4 large_bf16    Q, K, V iid N(0,1); then randperm(N)[:5% of N] picks key
+                  rows that are multiplied by 4 in every batch and head
+                  (a stand-in for the sparse semantic outliers).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+FACT_FRAME = 0
+FACT_TILED = 1
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    index: int
+    name: str
+    B: int
+    heads: int
+    d: int
+    T: int
+    H: int
+    W: int
+    dtype: str  # "f32" or "bf16"
+    fact: int = FACT_FRAME
+    tile_h: int = 0
+    tile_w: int = 0
+    extra: str = ""  # "scaled", "positional", "outliers" or ""
+
+    @property
+    def N(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def m(self) -> int:
+        """Tokens per stage-1 block."""
+        if self.fact == FACT_TILED:
+            return self.tile_h * self.tile_w
+        return self.H * self.W
+
+    @property
+    def b(self) -> int:
+        """Tokens per stage-2 group (one spatial position across frames)."""
+        return self.T
+
+    @property
+    def flops(self) -> float:
+        """Algorithmic FLOPs: 4*N*(m+b)*d per (batch, head); no padding."""
+        return 4.0 * self.N * (self.m + self.b) * self.d * self.B * self.heads
+
+    @property
+    def io_bytes(self) -> int:
+        """Minimum HBM bytes: read Q, K, V once, write O once."""
+        es = 4 if self.dtype == "f32" else 2
+        return 4 * self.B * self.heads * self.N * self.d * es
+
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+WORKLOADS = [
+    Workload(0, "tiny_fp32", 1, 2, 64, 4, 8, 8, "f32", extra="scaled"),
+    Workload(1, "chunk_bf16", 1, 12, 128, 3, 30, 52, "bf16"),
+    Workload(2, "fullclip_bf16", 1, 12, 128, 21, 30, 52, "bf16", extra="positional"),
+    Workload(3, "tiled_bf16", 1, 12, 128, 21, 30, 52, "bf16", FACT_TILED, 10, 13),
+    Workload(4, "large_bf16", 2, 12, 128, 21, 45, 80, "bf16", extra="outliers"),
+]
+BY_NAME = {w.name: w for w in WORKLOADS}
+
+
+def positional_features(T: int, H: int, W: int) -> torch.Tensor:
+    """u(n) for every token n = (t*H + h)*W + w, shape [N, 8] (float64)."""
+    t = torch.arange(T, dtype=torch.float64).view(T, 1, 1).expand(T, H, W)
+    h = torch.arange(H, dtype=torch.float64).view(1, H, 1).expand(T, H, W)
+    w = torch.arange(W, dtype=torch.float64).view(1, 1, W).expand(T, H, W)
+    tp = 2 * math.pi
+    feats = [torch.cos(tp * t / T), torch.sin(tp * t / T),
+             torch.cos(tp * h / H), torch.sin(tp * h / H),
+             torch.cos(tp * w / W), torch.sin(tp * w / W),
+             torch.cos(tp * (h / H + w / W)), torch.sin(tp * (h / H + w / W))]
+    return torch.stack([f.reshape(-1) for f in feats], dim=1)
+
+
+def generate(wl: Workload, seed: int | None = None, B: int | None = None,
+             heads: int | None = None):
+    """Seeded (Q, K, V) on the CPU, shape [B, heads, N, d], workload dtype.
+
+    ``B``/``heads`` may be lowered for a bounded sample; the first draws are
+    then those of the smaller tensor, so a sample is not a slice of the full
+    workload -- both sides of any comparison must use the same call.
+    """
+    seed = wl.index if seed is None else seed
+    B = wl.B if B is None else B
+    heads = wl.heads if heads is None else heads
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (B, heads, wl.N, wl.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    if wl.extra == "scaled":
+        s = wl.d ** -0.5
+        q.mul_(s); k.mul_(s); v.mul_(s)
+    elif wl.extra == "positional":
+        R = torch.randn((8, wl.d), generator=g, dtype=torch.float32)
+        pos = (0.5 * positional_features(wl.T, wl.H, wl.W).float() @ R)  # [N, d]
+        q.add_(pos); k.add_(pos)
+    elif wl.extra == "outliers":
+        n_out = (wl.N * 5) // 100
+        rows = torch.randperm(wl.N, generator=g)[:n_out]
+        k[:, :, rows, :] *= 4.0
+    dt = wl.torch_dtype()
+    return q.to(dt), k.to(dt), v.to(dt)
+
+
+def random_inputs(B, heads, T, H, W, d, dtype=torch.bfloat16, seed=0, scale=1.0):
+    """Seeded iid N(0, scale^2) inputs for ad-hoc shapes (edge-case tests)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (B, heads, T * H * W, d)
+    out = []
+    for _ in range(3):
+        x = torch.randn(shape, generator=g, dtype=torch.float32) * scale
+        out.append(x.to(dtype))
+    return tuple(out)

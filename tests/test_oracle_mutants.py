@@ -1,0 +1,89 @@
+"""Mutation check of the oracle's pins: each test compiles a copy of the
+oracle's C source with one plausible mistake planted in it (on the CPU, in a
+temporary directory) and requires that at least one pin from
+``test_oracle_pins`` rejects the broken copy.  A mutant that no pin catches
+would mean the pins leave that part of the oracle unchecked.
+"""
+import json
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "monarch_oracle.c")
+
+# (name, original text, replacement) -- every occurrence is replaced.
+MUTANTS = [
+    ("scale_1_over_d", "1.0 / sqrt((double)d)", "1.0 / (double)d"),
+    ("no_scale", "1.0 / sqrt((double)d)", "1.0"),
+    ("wrong_sign", "logit[j] = scale * acc;", "logit[j] = -scale * acc;"),
+    ("unnormalised", "double p = logit[j] / z;", "double p = logit[j];"),
+    ("dropped_feature", "for (int c = 0; c < d; ++c) acc += q[c] * krows[j][c];",
+     "for (int c = 1; c < d; ++c) acc += q[c] * krows[j][c];"),
+    ("shifted_value_column", "y[c] += p * vrows[j][c];", "y[c] += p * vrows[j][(c + 1) % d];"),
+    ("stage2_values_are_v", "st = oracle_monarch_stage2(q, k, y1, out,",
+     "st = oracle_monarch_stage2(q, k, v, out,"),
+    ("stage1_blocks_position_major", "return b * (long)H * W + i;", "return i * (long)T + b;"),
+    ("stage2_keys_contiguous", "kr[t] = kb + (t * HW + pos) * d;", "kr[t] = kb + (pos * T + t) * d;"),
+    ("stage2_query_is_key", "attend_one(qb + (t * HW + pos) * d, kr, vr, T,",
+     "attend_one(kb + (t * HW + pos) * d, kr, vr, T,"),
+    ("tile_rows_interleaved", "long h = ti * tile_h + hl, w = tj * tile_w + wl;",
+     "long h = ti + hl * (H / tile_h), w = tj * tile_w + wl;"),
+    ("tile_cols_interleaved", "long h = ti * tile_h + hl, w = tj * tile_w + wl;",
+     "long h = ti * tile_h + hl, w = tj + wl * (W / tile_w);"),
+    ("stage_order_swapped",
+     "st = oracle_monarch_stage1(q, k, v, y1, B, heads, T, H, W, d, fact, tile_h, tile_w);\n"
+     "    if (!st) st = oracle_monarch_stage2(q, k, y1, out, B, heads, T, H, W, d);",
+     "st = oracle_monarch_stage2(q, k, v, y1, B, heads, T, H, W, d);\n"
+     "    if (!st) st = oracle_monarch_stage1(q, k, y1, out, B, heads, T, H, W, d, fact, tile_h, tile_w);"),
+]
+
+GOLDEN = json.load(open(pins.GOLDEN))["cases"]
+
+# The pins, as (label, callable) with fixed parameters.
+PROBES = [(f"golden:{c['name']}", (lambda c=c: pins.test_hand_derived_golden(c))) for c in GOLDEN] + [
+    ("single_frame", lambda: pins.test_single_frame_is_dense_attention(4, 5, 8)),
+    ("single_position", lambda: pins.test_single_position_is_dense_attention_across_frames(5, 8)),
+    ("brute_frame", lambda: pins.test_brute_force_effective_matrix(*pins.BRUTE_SHAPES[0])),
+    ("brute_tiled", lambda: pins.test_brute_force_effective_matrix(*pins.BRUTE_SHAPES[2])),
+    ("zero_qk", pins.test_zero_qk_gives_global_mean),
+    ("zero_qk_tiled", pins.test_zero_qk_tiled_gives_tile_mean),
+    ("transpose", lambda: pins.test_transpose_h_w(1, 2, 3)),
+    ("numpy", lambda: pins.test_numpy_restatement_small((1, 2, 6, 4, 6, 1, 2, 3))),
+]
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert old in src, f"mutant {name}: pattern not found in the oracle source"
+    mut = src.replace(old, new)
+    c = tmp_path / f"{name}.c"
+    so = tmp_path / f"lib{name}.so"
+    c.write_text(mut)
+    subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-std=c11", "-o", str(so), str(c), "-lm"],
+                   check=True)
+    return str(so)
+
+
+def test_unmutated_passes_every_probe():
+    for label, fn in PROBES:
+        fn()
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    so = _build_mutant(tmp_path, name, old, new)
+    prev = oracle.use_library(so)
+    caught = []
+    try:
+        for label, fn in PROBES:
+            try:
+                fn()
+            except (AssertionError, ValueError, FloatingPointError):
+                caught.append(label)
+    finally:
+        oracle.restore_library(prev)
+    assert caught, f"no pin rejects the planted mistake '{name}'"
