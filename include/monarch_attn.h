@@ -1,0 +1,139 @@
+/*
+ * monarch_attn.h -- C ABI of the B200 (sm_100a) Monarch attention forward.
+ *
+ * The operator (MonarchRT: Efficient Attention for Real-Time Video
+ * Generation; gist.science/nl/paper/2602.12271, section "Methodologie": the
+ * attention matrix is a product of permutation and block-diagonal matrices;
+ * gist.science/zh/paper/2602.12271, section 2.2: blocks aligned with the
+ * frame/height/width axes, and tiled Monarch):
+ *
+ *     out = M V,   M = P^T B2 P B1,
+ *
+ * per (batch, head) over the N = T*H*W tokens of a video latent, token index
+ * n = (t*H + h)*W + w.  B1 is block diagonal over stage-1 blocks (one frame of
+ * H*W tokens, or one tile_h x tile_w spatial tile of one frame); P swaps the
+ * block index and the in-block index; B2 is block diagonal over the groups of
+ * T tokens sharing a spatial position (h, w).  Every diagonal block is a dense
+ * softmax attention with scale 1/sqrt(d): stage 1 attends Q to K with values
+ * V inside its block, stage 2 attends the same Q and K rows inside a group
+ * with the stage-1 outputs as values.
+ *
+ * Every entry point is plain C: raw pointers, ints, and a cudaStream_t passed
+ * as void*.  No entry point allocates device memory.
+ */
+#ifndef MONARCH_ATTN_H
+#define MONARCH_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    MONARCH_OK = 0,
+    MONARCH_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment, aliasing or enum; nothing launched */
+    MONARCH_ERR_UNSUPPORTED = 2, /* valid but outside this build's limits (see below); nothing launched */
+    MONARCH_ERR_LAUNCH = 3,      /* a kernel launch failed (cudaGetLastError after launch) */
+    MONARCH_ERR_TIMEOUT = 4,     /* a device-side wait gave up (reported by monarch_attn_device_status) */
+    MONARCH_ERR_CUDA = 5         /* a CUDA runtime/driver call other than a launch failed */
+} monarch_status_t;
+
+/* Element type of q, k, v and out. */
+typedef enum {
+    MONARCH_DTYPE_F32 = 0,  /* fp32 in and out; exact path on CUDA cores, fp32 accumulation */
+    MONARCH_DTYPE_BF16 = 1  /* bf16 in and out; tcgen05 tensor cores, fp32 accumulation and softmax */
+} monarch_dtype_t;
+
+/* Choice of stage-1 blocks (block alignment: every video axis lies inside one
+ * block dimension). */
+typedef enum {
+    MONARCH_FACT_FRAME = 0, /* block = one frame, m = H*W tokens, b = T blocks */
+    MONARCH_FACT_TILED = 1  /* block = one tile_h x tile_w spatial tile of one frame */
+} monarch_fact_t;
+
+/*
+ * monarch_attn_fwd -- out = P^T B2 P B1 V (see the top of this file).
+ *
+ * Arguments
+ *   q, k, v   device pointers, inputs, layout [B][heads][N][d] contiguous
+ *             (N = T*H*W, token order n = (t*H + h)*W + w), element type
+ *             `dtype`.  Read only.
+ *   out       device pointer, output, same layout and type.  Must not overlap
+ *             q, k or v.  The stage-1 result is kept in `out` between the two
+ *             stages (stage 2 reads and overwrites it group by group), so no
+ *             scratch buffer is needed; out's prior contents are ignored.
+ *   B, heads  batch size and head count, >= 1.
+ *   T, H, W   frames, height and width of the token grid, >= 1.
+ *   d         head width: 64 or 128.
+ *   factorisation  MONARCH_FACT_FRAME or MONARCH_FACT_TILED.
+ *   tile_h, tile_w tile size for MONARCH_FACT_TILED; must divide H and W
+ *             respectively.  Ignored for MONARCH_FACT_FRAME.
+ *   dtype     MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32.
+ *   stream    cudaStream_t (NULL = legacy default stream) the work is queued on.
+ *
+ * Limits of this build (MONARCH_ERR_UNSUPPORTED otherwise): T <= 128;
+ * tile_w <= 128 for MONARCH_FACT_TILED; N <= 2^31; a device of compute
+ * capability 10.0 (B200).  Pointers must be 16-byte aligned
+ * (MONARCH_ERR_INVALID_ARG otherwise).
+ *
+ * Errors and ownership
+ *   The caller owns all four buffers.  Argument errors are reported before
+ *   anything is queued.  The call is asynchronous: it returns after queueing
+ *   the kernels on `stream`; device faults surface at the caller's next
+ *   synchronisation, following CUDA convention.  Device-side waits are
+ *   bounded: a wait that gives up records MONARCH_ERR_TIMEOUT in a device
+ *   status word that monarch_attn_device_status() returns.  With the
+ *   environment variable MONARCH_ATTN_DEBUG=1 the call synchronises `stream`
+ *   and returns that status directly.
+ */
+int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                     int B, int heads, int T, int H, int W, int d,
+                     int factorisation, int tile_h, int tile_w, int dtype,
+                     void *stream);
+
+/*
+ * monarch_attn_fwd_host -- the same operator for inputs and output in host
+ * memory.  Queues on `stream`: copies of h_q, h_k, h_v into the caller's
+ * device buffers d_q, d_k, d_v (one cudaMemcpyAsync each), monarch_attn_fwd
+ * on the device buffers, and a copy of d_out back into h_out; then waits for
+ * the stream.  Host buffers should be pinned for asynchronous copies.  All
+ * eight buffers are owned by the caller and hold B*heads*N*d elements of
+ * `dtype`; the device buffers follow monarch_attn_fwd's rules.
+ * Returns after h_out is written, or with the first error.
+ */
+int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, void *h_out,
+                          void *d_q, void *d_k, void *d_v, void *d_out,
+                          int B, int heads, int T, int H, int W, int d,
+                          int factorisation, int tile_h, int tile_w, int dtype,
+                          void *stream);
+
+/* Human-readable text of a status code; never NULL, owned by the library. */
+const char *monarch_attn_strerror(int status);
+
+/*
+ * monarch_attn_device_status -- synchronises `stream`, then returns
+ * MONARCH_ERR_TIMEOUT if any kernel of this library on the current device
+ * recorded a timed-out wait since the last reset, MONARCH_ERR_CUDA if the
+ * synchronisation itself failed, else MONARCH_OK.  With reset != 0 the
+ * device status word is cleared afterwards.
+ */
+int monarch_attn_device_status(void *stream, int reset);
+
+/*
+ * monarch_attn_selftest_timeout -- exercises the bounded-wait machinery:
+ * launches one block whose thread waits on a barrier that nothing completes,
+ * for at most `limit_cycles` SM clock cycles, then records a timeout in the
+ * device status word and returns.  Returns the value monarch_attn_device_status
+ * would (MONARCH_ERR_TIMEOUT when the machinery works) and clears the word.
+ * No counterpart in the pages: this is error-path test support.
+ */
+int monarch_attn_selftest_timeout(long long limit_cycles, void *stream);
+
+/* Version of this library as MAJOR*10000 + MINOR*100 + PATCH. */
+int monarch_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MONARCH_ATTN_H */

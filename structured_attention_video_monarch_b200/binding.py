@@ -1,0 +1,134 @@
+"""ctypes binding over the C ABI in ``include/monarch_attn.h``.
+
+Argument marshalling only: every step of the operator runs in the CUDA
+library.  Tensors are PyTorch tensors purely as device memory; the stream is
+PyTorch's current stream unless one is given.  There is no fallback: if the
+library is missing or the call fails, this raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+FACT_FRAME = 0
+FACT_TILED = 1
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
+STATUS_NAMES = {0: "MONARCH_OK", 1: "MONARCH_ERR_INVALID_ARG", 2: "MONARCH_ERR_UNSUPPORTED",
+                3: "MONARCH_ERR_LAUNCH", 4: "MONARCH_ERR_TIMEOUT", 5: "MONARCH_ERR_CUDA"}
+
+_lib = None
+
+
+class MonarchError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({strerror(status)})")
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def load_library(path: str | None = None):
+    """Load libmonarch_attn.so (built in-tree by ``build.build()``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    path = path or _build.LIB
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library not built: {path} (run __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.monarch_attn_fwd.argtypes = [vp, vp, vp, vp] + [i] * 10 + [vp]
+    lib.monarch_attn_fwd.restype = i
+    lib.monarch_attn_fwd_host.argtypes = [vp] * 8 + [i] * 10 + [vp]
+    lib.monarch_attn_fwd_host.restype = i
+    lib.monarch_attn_strerror.argtypes = [i]
+    lib.monarch_attn_strerror.restype = ctypes.c_char_p
+    lib.monarch_attn_device_status.argtypes = [vp, i]
+    lib.monarch_attn_device_status.restype = i
+    lib.monarch_attn_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
+    lib.monarch_attn_selftest_timeout.restype = i
+    lib.monarch_attn_version.argtypes = []
+    lib.monarch_attn_version.restype = i
+    if path == _build.LIB:
+        _lib = lib
+    return lib
+
+
+def strerror(status: int) -> str:
+    return load_library().monarch_attn_strerror(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float32")
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def monarch_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, T: int, H: int, W: int,
+                     factorisation: int = FACT_FRAME, tile_h: int = 0, tile_w: int = 0,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out = P^T B2 P B1 V for q, k, v of shape [B, heads, T*H*W, d] on a CUDA device.
+
+    Queued on ``stream`` (default: PyTorch's current stream); returns ``out``.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, heads, N, d]")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, heads, N, d] shape")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share one dtype")
+    B, heads, N, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor shaped and typed like q")
+    if N != T * H * W:
+        raise ValueError(f"N={N} does not equal T*H*W={T * H * W}")
+    st = load_library().monarch_attn_fwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, heads, T, H, W, d,
+        int(factorisation), int(tile_h), int(tile_w), _dtype_code(q), _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd")
+    return out
+
+
+def monarch_attn_fwd_host(h_q, h_k, h_v, h_out, d_q, d_k, d_v, d_out, T, H, W,
+                          factorisation=FACT_FRAME, tile_h=0, tile_w=0, stream=None):
+    """Host-buffer variant: copies in, computes on the device buffers, copies out, syncs."""
+    B, heads, N, d = h_q.shape
+    st = load_library().monarch_attn_fwd_host(
+        h_q.data_ptr(), h_k.data_ptr(), h_v.data_ptr(), h_out.data_ptr(),
+        d_q.data_ptr(), d_k.data_ptr(), d_v.data_ptr(), d_out.data_ptr(),
+        B, heads, T, H, W, d, int(factorisation), int(tile_h), int(tile_w),
+        _dtype_code(h_q), _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_host")
+    return h_out
+
+
+def last_device_error(reset: bool = True, stream=None) -> int:
+    """Status word of the library's device-side waits (0 = none timed out)."""
+    return int(load_library().monarch_attn_device_status(_stream_ptr(stream), 1 if reset else 0))
+
+
+def selftest_timeout(limit_cycles: int, stream=None) -> int:
+    return int(load_library().monarch_attn_selftest_timeout(int(limit_cycles), _stream_ptr(stream)))

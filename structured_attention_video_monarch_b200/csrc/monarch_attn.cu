@@ -1,0 +1,382 @@
+// monarch_attn.cu -- C ABI of the Monarch attention forward (include/monarch_attn.h):
+// argument validation, TMA tensor-map construction (the (T,H,W) reshape and
+// the stage permutation P are expressed as tensor-map boxes), and kernel
+// launches on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/monarch_attn.h"
+#include "attn_f32.cuh"
+#include "attn_tc.cuh"
+
+namespace monarch {
+
+__device__ unsigned g_device_status = 0u;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    int sms = 0;
+    bool tc_attr[2] = {false, false};
+    bool f32_attr[2] = {false, false};
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return MONARCH_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return MONARCH_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return MONARCH_OK;
+}
+
+int device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &di = g_dev[dev];
+    if (!di.init) {
+        int sms = 0, major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return MONARCH_ERR_CUDA;
+        if (major != 10 || minor != 0) return MONARCH_ERR_UNSUPPORTED;  // built for sm_100a only
+        di.sms = sms;
+        di.init = true;
+    }
+    *out = &di;
+    return MONARCH_OK;
+}
+
+bool env_debug() {
+    const char *e = std::getenv("MONARCH_ATTN_DEBUG");
+    return e && e[0] == '1';
+}
+
+long long env_timeout_cycles() {
+    const char *e = std::getenv("MONARCH_ATTN_TIMEOUT_CYCLES");
+    if (e && *e) {
+        long long v = std::atoll(e);
+        if (v > 0) return v;
+    }
+    return 4000000000ll;  // about 2 s at the B200 boost clock
+}
+
+bool overlaps(const void *a, const void *b, size_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+struct Shape {
+    int B, heads, T, H, W, d, fact, tile_h, tile_w, dtype;
+    long long N, elems;
+};
+
+int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
+    if (!q || !k || !v || !out) return MONARCH_ERR_INVALID_ARG;
+    if (s.B < 1 || s.heads < 1 || s.T < 1 || s.H < 1 || s.W < 1) return MONARCH_ERR_INVALID_ARG;
+    if (s.d != 64 && s.d != 128) return MONARCH_ERR_INVALID_ARG;
+    if (s.dtype != MONARCH_DTYPE_F32 && s.dtype != MONARCH_DTYPE_BF16) return MONARCH_ERR_INVALID_ARG;
+    if (s.fact != MONARCH_FACT_FRAME && s.fact != MONARCH_FACT_TILED) return MONARCH_ERR_INVALID_ARG;
+    if (s.fact == MONARCH_FACT_TILED) {
+        if (s.tile_h < 1 || s.tile_w < 1 || s.H % s.tile_h != 0 || s.W % s.tile_w != 0)
+            return MONARCH_ERR_INVALID_ARG;
+    }
+    for (const void *p : {q, k, v, static_cast<const void *>(out)})
+        if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return MONARCH_ERR_INVALID_ARG;
+    s.N = static_cast<long long>(s.T) * s.H * s.W;
+    if (s.N > (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+    s.elems = static_cast<long long>(s.B) * s.heads * s.N * s.d;
+    const size_t bytes = static_cast<size_t>(s.elems) * (s.dtype == MONARCH_DTYPE_F32 ? 4 : 2);
+    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
+        return MONARCH_ERR_INVALID_ARG;
+    if (s.T > 128) return MONARCH_ERR_UNSUPPORTED;
+    if (s.fact == MONARCH_FACT_TILED && s.tile_w > 128) return MONARCH_ERR_UNSUPPORTED;
+    if (static_cast<long long>(s.B) * s.heads > (1ll << 30)) return MONARCH_ERR_UNSUPPORTED;
+    return MONARCH_OK;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides
+// in bytes for dims 1..rank-1.
+int make_map(CUtensorMap *map, const void *ptr, int rank, const cuuint64_t *dims,
+             const cuuint64_t *strides, const cuuint32_t *box) {
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MONARCH_OK : MONARCH_ERR_CUDA;
+}
+
+// Stage-1 view of a [B*heads][N][d] bf16 tensor.
+//   frame: (d, m, B*heads*T), box (64, 128, 1): one 128-token slab of a frame
+//   tiled: (d, tile_w, tiles_w, tile_h, tiles_h*B*heads*T),
+//          box (64, tile_w, 1, rows, 1): `rows` tile rows of one tile
+int stage1_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams &p) {
+    const cuuint64_t es = 2, d = s.d;
+    if (s.fact == MONARCH_FACT_FRAME) {
+        cuuint64_t dims[3] = {d, static_cast<cuuint64_t>(p.m),
+                              static_cast<cuuint64_t>(s.B) * s.heads * s.T};
+        cuuint64_t strides[2] = {d * es, static_cast<cuuint64_t>(p.m) * d * es};
+        cuuint32_t box[3] = {64, 128, 1};
+        return make_map(map, ptr, 3, dims, strides, box);
+    }
+    cuuint64_t dims[5] = {d, static_cast<cuuint64_t>(s.tile_w), static_cast<cuuint64_t>(p.tiles_w),
+                          static_cast<cuuint64_t>(s.tile_h),
+                          static_cast<cuuint64_t>(p.tiles_h) * s.B * s.heads * s.T};
+    cuuint64_t strides[4] = {d * es, static_cast<cuuint64_t>(s.tile_w) * d * es,
+                             static_cast<cuuint64_t>(s.W) * d * es,
+                             static_cast<cuuint64_t>(s.tile_h) * s.W * d * es};
+    cuuint32_t box[5] = {64, static_cast<cuuint32_t>(s.tile_w), 1,
+                         static_cast<cuuint32_t>(p.rows_per_tile), 1};
+    return make_map(map, ptr, 5, dims, strides, box);
+}
+
+// Stage-2 view: (d, H*W, T, B*heads), box (64, npos, T, 1): npos consecutive
+// positions across all T frames, landing in shared memory as rows t*npos + pos.
+int stage2_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams &p) {
+    const cuuint64_t es = 2, d = s.d;
+    cuuint64_t dims[4] = {d, static_cast<cuuint64_t>(p.HW), static_cast<cuuint64_t>(s.T),
+                          static_cast<cuuint64_t>(s.B) * s.heads};
+    cuuint64_t strides[3] = {d * es, static_cast<cuuint64_t>(p.HW) * d * es,
+                             static_cast<cuuint64_t>(s.N) * d * es};
+    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(p.npos), static_cast<cuuint32_t>(s.T), 1};
+    return make_map(map, ptr, 4, dims, strides, box);
+}
+
+template <int D>
+int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
+              cudaStream_t stream) {
+    DeviceInfo *di = nullptr;
+    int st = device_info(&di);
+    if (st) return st;
+    if ((st = get_encode())) return st;
+    using L = TcLayout<D>;
+    const int di_idx = D == 128 ? 1 : 0;
+    if (!di->tc_attr[di_idx]) {
+        if (cudaFuncSetAttribute(monarch_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::ALLOC) != cudaSuccess)
+            return MONARCH_ERR_CUDA;
+        di->tc_attr[di_idx] = true;
+    }
+    TcParams p{};
+    p.B = s.B; p.heads = s.heads; p.T = s.T; p.H = s.H; p.W = s.W; p.HW = s.H * s.W;
+    p.fact = s.fact;
+    if (s.fact == MONARCH_FACT_TILED) {
+        p.tile_h = s.tile_h; p.tile_w = s.tile_w;
+        p.tiles_h = s.H / s.tile_h; p.tiles_w = s.W / s.tile_w;
+        const int r = 128 / s.tile_w;
+        p.rows_per_tile = r < s.tile_h ? r : s.tile_h;
+        p.m = s.tile_h * s.tile_w;
+        p.nblk_bh = s.T * p.tiles_h * p.tiles_w;
+        p.nqt = (s.tile_h + p.rows_per_tile - 1) / p.rows_per_tile;
+    } else {
+        p.tile_h = p.tile_w = p.tiles_h = p.tiles_w = 0;
+        p.rows_per_tile = 0;
+        p.m = p.HW;
+        p.nblk_bh = s.T;
+        p.nqt = (p.m + 127) / 128;
+    }
+    p.s1_pairs = (p.nqt + 1) / 2;
+    p.npos = 128 / s.T;
+    p.s2_chunks = (p.HW + p.npos - 1) / p.npos;
+    p.s2_pairs = (p.s2_chunks + 1) / 2;
+    const long long bh = static_cast<long long>(s.B) * s.heads;
+    p.s1_units = bh * p.nblk_bh * p.s1_pairs;
+    p.s2_units = bh * p.s2_pairs;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.d)));
+    p.timeout_cycles = env_timeout_cycles();
+    unsigned *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_device_status) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    p.status = status;
+
+    CUtensorMap mq1, mk1, mv1, mo1, mq2, mk2, my2, mo2;
+    if ((st = stage1_map(&mq1, q, s, p)) || (st = stage1_map(&mk1, k, s, p)) ||
+        (st = stage1_map(&mv1, v, s, p)) || (st = stage1_map(&mo1, out, s, p)) ||
+        (st = stage2_map(&mq2, q, s, p)) || (st = stage2_map(&mk2, k, s, p)) ||
+        (st = stage2_map(&my2, out, s, p)) || (st = stage2_map(&mo2, out, s, p)))
+        return st;
+
+    // stage 1: Y1 = B1 V into out; stage 2: out = P^T B2 P Y1 in place.
+    const long long ranges[2][2] = {{0, p.s1_units}, {p.s1_units, p.s1_units + p.s2_units}};
+    for (int r = 0; r < 2; ++r) {
+        p.unit_begin = ranges[r][0];
+        p.unit_end = ranges[r][1];
+        const long long units = p.unit_end - p.unit_begin;
+        if (units <= 0) continue;
+        const int grid = static_cast<int>(units < di->sms ? units : di->sms);
+        monarch_tc_kernel<D><<<grid, 512, L::ALLOC, stream>>>(mq1, mk1, mv1, mo1, mq2, mk2, my2, mo2, p);
+        if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    }
+    return MONARCH_OK;
+}
+
+template <int D>
+int launch_f32(const void *q, const void *k, const void *v, void *out, const Shape &s,
+               cudaStream_t stream) {
+    DeviceInfo *di = nullptr;
+    int st = device_info(&di);
+    if (st) return st;
+    F32Params p{};
+    p.T = s.T; p.H = s.H; p.W = s.W; p.HW = s.H * s.W; p.N = s.N;
+    p.fact = s.fact;
+    if (s.fact == MONARCH_FACT_TILED) {
+        p.tile_h = s.tile_h; p.tile_w = s.tile_w;
+        p.tiles_h = s.H / s.tile_h; p.tiles_w = s.W / s.tile_w;
+        p.m = s.tile_h * s.tile_w;
+        p.nblk_bh = s.T * p.tiles_h * p.tiles_w;
+    } else {
+        p.m = p.HW;
+        p.nblk_bh = s.T;
+    }
+    p.qchunks = (p.m + 63) / 64;
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.d)));
+    const long long bh = static_cast<long long>(s.B) * s.heads;
+    const long long g1 = bh * p.nblk_bh * p.qchunks;
+    const long long g2 = bh * p.HW;
+    if (g1 >= (1ll << 31) || g2 >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+    const int smem2 = 2 * s.T * D * 4;
+    const int di_idx = D == 128 ? 1 : 0;
+    if (!di->f32_attr[di_idx]) {
+        if (cudaFuncSetAttribute(monarch_f32_stage2<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 2 * 128 * D * 4) != cudaSuccess)
+            return MONARCH_ERR_CUDA;
+        di->f32_attr[di_idx] = true;
+    }
+    const float *fq = static_cast<const float *>(q);
+    const float *fk = static_cast<const float *>(k);
+    const float *fv = static_cast<const float *>(v);
+    float *fo = static_cast<float *>(out);
+    monarch_f32_stage1<D><<<static_cast<unsigned>(g1), 128, 0, stream>>>(fq, fk, fv, fo, p);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    const int threads2 = ((2 * s.T + 31) / 32) * 32;
+    monarch_f32_stage2<D><<<static_cast<unsigned>(g2), threads2, smem2, stream>>>(fq, fk, fo, p);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    return MONARCH_OK;
+}
+
+__global__ void selftest_timeout_kernel(long long limit, unsigned *status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        mbar_init(smem_addr(&bar), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        WaitCtl ctl{&abort_flag, status, limit};
+        // nothing ever arrives on this barrier: the wait must give up
+        (void)mbar_wait(smem_addr(&bar), 0u, ctl);
+    }
+}
+
+int read_status(cudaStream_t stream, int reset) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MONARCH_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return MONARCH_ERR_CUDA;
+    if (reset && v) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+            return MONARCH_ERR_CUDA;
+    }
+    return (v & DEVERR_TIMEOUT) ? MONARCH_ERR_TIMEOUT : MONARCH_OK;
+}
+
+}  // namespace
+}  // namespace monarch
+
+using namespace monarch;
+
+extern "C" {
+
+int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out, int B, int heads, int T,
+                     int H, int W, int d, int factorisation, int tile_h, int tile_w, int dtype,
+                     void *stream) {
+    Shape s{B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
+    int st = validate(q, k, v, out, s);
+    if (st) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (dtype == MONARCH_DTYPE_BF16)
+        st = d == 128 ? launch_tc<128>(q, k, v, out, s, cs) : launch_tc<64>(q, k, v, out, s, cs);
+    else
+        st = d == 128 ? launch_f32<128>(q, k, v, out, s, cs) : launch_f32<64>(q, k, v, out, s, cs);
+    if (st) return st;
+    if (env_debug()) return read_status(cs, 0);
+    return MONARCH_OK;
+}
+
+int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, void *h_out, void *d_q,
+                          void *d_k, void *d_v, void *d_out, int B, int heads, int T, int H, int W,
+                          int d, int factorisation, int tile_h, int tile_w, int dtype,
+                          void *stream) {
+    if (!h_q || !h_k || !h_v || !h_out) return MONARCH_ERR_INVALID_ARG;
+    Shape s{B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
+    int st = validate(d_q, d_k, d_v, d_out, s);
+    if (st) return st;
+    const size_t bytes = static_cast<size_t>(s.elems) * (dtype == MONARCH_DTYPE_F32 ? 4 : 2);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(d_q, h_q, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(d_k, h_k, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaMemcpyAsync(d_v, h_v, bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    st = monarch_attn_fwd(d_q, d_k, d_v, d_out, B, heads, T, H, W, d, factorisation, tile_h, tile_w,
+                          dtype, stream);
+    if (st) return st;
+    if (cudaMemcpyAsync(h_out, d_out, bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return MONARCH_ERR_CUDA;
+    return MONARCH_OK;
+}
+
+const char *monarch_attn_strerror(int status) {
+    switch (status) {
+        case MONARCH_OK: return "success";
+        case MONARCH_ERR_INVALID_ARG: return "invalid argument (pointer, size, alignment, aliasing or enum)";
+        case MONARCH_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case MONARCH_ERR_LAUNCH: return "kernel launch failed";
+        case MONARCH_ERR_TIMEOUT: return "a device-side wait timed out";
+        case MONARCH_ERR_CUDA: return "CUDA runtime or driver call failed";
+        default: return "unknown status";
+    }
+}
+
+int monarch_attn_device_status(void *stream, int reset) {
+    return read_status(static_cast<cudaStream_t>(stream), reset);
+}
+
+int monarch_attn_selftest_timeout(long long limit_cycles, void *stream) {
+    if (limit_cycles <= 0) return MONARCH_ERR_INVALID_ARG;
+    DeviceInfo *di = nullptr;
+    int st = device_info(&di);
+    if (st) return st;
+    unsigned *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_device_status) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    selftest_timeout_kernel<<<1, 32, 0, cs>>>(limit_cycles, status);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    return read_status(cs, 1);
+}
+
+int monarch_attn_version(void) { return 100; }
+
+}  // extern "C"

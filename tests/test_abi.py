@@ -1,0 +1,101 @@
+"""C ABI checks that need no GPU: the library builds for sm_100a and loads,
+every entry point declared in include/monarch_attn.h is exported, status
+strings exist, and argument validation rejects bad calls before touching
+CUDA (so these calls are safe on a machine without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from structured_attention_video_monarch_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "monarch_attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(monarch_attn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    assert "monarch_attn_fwd" in names and "monarch_attn_strerror" in names
+    assert len(names) >= 5
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in declared_functions():
+        assert name in exported, f"{name} declared but not exported"
+        assert hasattr(lib, name)
+
+
+def test_strerror_and_version(lib):
+    for code in range(6):
+        s = binding.strerror(code)
+        assert isinstance(s, str) and s
+    assert binding.strerror(99) == "unknown status"
+    assert lib.monarch_attn_version() >= 100
+
+
+def _call(lib, q=16, k=32, v=48, out=4096, B=1, heads=1, T=2, H=4, W=4, d=128, fact=0, th=0, tw=0,
+          dtype=1):
+    return lib.monarch_attn_fwd(q, k, v, out, B, heads, T, H, W, d, fact, th, tw, dtype, None)
+
+
+@pytest.mark.parametrize("kwargs", [
+    dict(q=0),                      # null pointer
+    dict(out=0),
+    dict(B=0), dict(heads=0), dict(T=0), dict(H=0), dict(W=-1),
+    dict(d=96), dict(d=256),        # unsupported head width
+    dict(dtype=2),                  # unknown dtype
+    dict(fact=2),                   # unknown factorisation
+    dict(fact=1, th=3, tw=2),       # tile does not divide H
+    dict(fact=1, th=2, tw=0),
+    dict(q=18),                     # misaligned (not 16-byte aligned)
+    dict(out=16),                   # out aliases q
+])
+def test_validation_rejects_without_cuda(lib, kwargs):
+    assert _call(lib, **kwargs) == 1  # MONARCH_ERR_INVALID_ARG
+
+
+def test_unsupported_sizes(lib):
+    # disjoint fake addresses far apart; rejected before any CUDA call
+    big = 1 << 40
+    assert lib.monarch_attn_fwd(16, big, 2 * big, 3 * big, 1, 1, 129, 1, 1, 128, 0, 0, 0, 1, None) == 2
+    assert lib.monarch_attn_fwd(16, big, 2 * big, 3 * big, 1, 1, 2, 2, 256, 128, 1, 1, 256, 1,
+                                None) == 2
+
+
+def test_host_entry_rejects_null_host_buffers(lib):
+    assert lib.monarch_attn_fwd_host(0, 16, 32, 48, 64, 80, 96, 4096, 1, 1, 2, 4, 4, 128, 0, 0, 0,
+                                     1, None) == 1
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.monarch_attn_fwd(x, x, x, 2, 2, 2)
+
+
+def test_product_package_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "structured_attention_video_monarch_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "monarch_oracle" not in text, f

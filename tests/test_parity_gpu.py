@@ -1,0 +1,220 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances: fp32 inputs max-abs <= 1e-5; bf16 inputs max-abs <= 2e-2 and
+relative L2 <= 1e-2.  Outputs are poisoned with NaN before each call so an
+unwritten element fails.  Full-size workloads are checked on oracle rows of
+sampled stage-2 groups (exact for those rows) plus properties that hold at
+any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from structured_attention_video_monarch_b200 import binding, workloads
+
+pytestmark = pytest.mark.gpu
+
+F32_ATOL = 1e-5
+BF16_ATOL = 2e-2
+BF16_RL2 = 1e-2
+
+
+def _dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return torch.device("cuda:0")
+
+
+def _run(q, k, v, T, H, W, fact=0, th=0, tw=0):
+    dev = _dev()
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    out = torch.full_like(qd, float("nan"))
+    binding.monarch_attn_fwd(qd, kd, vd, T, H, W, fact, th, tw, out=out)
+    torch.cuda.synchronize()
+    assert binding.last_device_error() == 0
+    return out.cpu()
+
+
+def _check(got: torch.Tensor, ref: np.ndarray, dtype):
+    g = got.double().numpy()
+    assert np.isfinite(g).all(), "non-finite output (unwritten or overflowed element)"
+    err = np.abs(g - ref)
+    if dtype == torch.float32:
+        assert err.max() <= F32_ATOL, f"max-abs {err.max():.3e}"
+    else:
+        rl2 = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)
+        assert err.max() <= BF16_ATOL, f"max-abs {err.max():.3e} (rel-L2 {rl2:.3e})"
+        assert rl2 <= BF16_RL2, f"rel-L2 {rl2:.3e}"
+
+
+def _groups(B, heads, HW, n, seed, must=()):
+    rng = np.random.default_rng(seed)
+    g = [(int(rng.integers(B * heads)), int(rng.integers(HW))) for _ in range(n)]
+    return list(must) + g
+
+
+# ------------------------------------------------------------------ workloads
+
+def test_tiny_fp32_full():
+    wl = workloads.BY_NAME["tiny_fp32"]
+    q, k, v = workloads.generate(wl)
+    got = _run(q, k, v, wl.T, wl.H, wl.W)
+    _check(got, oracle.monarch_fwd(q, k, v, wl.T, wl.H, wl.W), torch.float32)
+
+
+def test_chunk_bf16_full_heads():
+    wl = workloads.BY_NAME["chunk_bf16"]
+    q, k, v = workloads.generate(wl)
+    got = _run(q, k, v, wl.T, wl.H, wl.W)
+    hs = slice(0, 3)  # heads are independent: the oracle on a head slice is exact for it
+    ref = oracle.monarch_fwd(q[:, hs], k[:, hs], v[:, hs], wl.T, wl.H, wl.W)
+    _check(got[:, hs], ref, torch.bfloat16)
+    assert torch.isfinite(got.float()).all()
+
+
+@pytest.mark.parametrize("name", ["fullclip_bf16", "tiled_bf16", "large_bf16"])
+def test_full_size_sampled_groups(name):
+    wl = workloads.BY_NAME[name]
+    q, k, v = workloads.generate(wl)
+    got = _run(q, k, v, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w)
+    g = got.float()
+    assert torch.isfinite(g).all(), "non-finite output at full size"
+    HW = wl.H * wl.W
+    # include the first/last positions (ragged last query tile, last stage-2 chunk)
+    must = [(0, 0), (wl.B * wl.heads - 1, HW - 1), (1, HW - 2), (2, 1535 % HW), (3, 1559 % HW)]
+    groups = _groups(wl.B, wl.heads, HW, 40, seed=wl.index, must=must)
+    ref = oracle.monarch_fwd_groups(q, k, v, wl.T, wl.H, wl.W, groups, wl.fact, wl.tile_h, wl.tile_w)
+    gr = got.reshape(wl.B * wl.heads, wl.T, HW, wl.d)
+    rows = torch.stack([gr[bh, :, pos] for bh, pos in groups])
+    _check(rows, ref, torch.bfloat16)
+    # any-size property: every output row is a convex combination of value rows,
+    # so it lies inside the per-(batch, head) range of V (up to bf16 rounding)
+    vf = v.float().reshape(wl.B * wl.heads, -1, wl.d)
+    lo = vf.min(dim=1).values[:, None, None, :]
+    hi = vf.max(dim=1).values[:, None, None, :]
+    assert (gr >= lo - 0.02).all() and (gr <= hi + 0.02).all()
+
+
+# ------------------------------------------------------------------ edge cases (full oracle)
+
+FRAME_CASES = [
+    # B, heads, T, H, W, d
+    (1, 2, 3, 5, 7, 128),     # m = 35 < one tile
+    (1, 1, 2, 8, 16, 128),    # m = 128 exactly
+    (2, 1, 2, 16, 16, 128),   # m = 256 (two full tiles, one pair)
+    (1, 2, 2, 3, 43, 128),    # m = 129 (ragged by one)
+    (1, 1, 3, 20, 20, 128),   # m = 400: 4 tiles, 2 pairs, ragged tail
+    (1, 1, 5, 13, 37, 128),   # m = 481: 4 tiles (odd pair count), stage-2 npos = 25
+    (1, 1, 1, 17, 19, 128),   # T = 1: stage 2 is the identity
+    (1, 2, 21, 1, 1, 128),    # m = 1: stage 1 is the identity
+    (1, 1, 128, 2, 3, 128),   # T = 128: one position per stage-2 chunk
+    (1, 1, 65, 3, 3, 128),    # T = 65: npos = 1
+    (2, 3, 4, 9, 11, 64),     # d = 64
+    (1, 1, 7, 30, 52, 64),    # d = 64, m = 1560
+]
+
+
+@pytest.mark.parametrize("B,heads,T,H,W,d", FRAME_CASES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_frame_edge_cases(B, heads, T, H, W, d, dtype):
+    q, k, v = workloads.random_inputs(B, heads, T, H, W, d, dtype=dtype, seed=T * 1000 + H * 10 + W,
+                                      scale=1.0 if dtype == torch.bfloat16 else d ** -0.25)
+    got = _run(q, k, v, T, H, W)
+    _check(got, oracle.monarch_fwd(q, k, v, T, H, W), dtype)
+
+
+TILED_CASES = [
+    # B, heads, T, H, W, d, tile_h, tile_w
+    (1, 2, 3, 20, 26, 128, 10, 13),  # the workload's 10 x 13 tiles on a small grid
+    (1, 1, 2, 16, 32, 128, 8, 16),   # tile of exactly 128 tokens
+    (1, 1, 2, 6, 100, 128, 3, 50),   # tile_w = 50: 2 rows per 128-row tile
+    (1, 1, 2, 4, 256, 128, 2, 128),  # tile_w = 128: one row per tile
+    (2, 2, 4, 12, 12, 64, 4, 3),     # small tiles, d = 64
+    (1, 1, 5, 9, 10, 128, 9, 5),     # tall narrow tiles
+]
+
+
+@pytest.mark.parametrize("B,heads,T,H,W,d,th,tw", TILED_CASES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "f32"])
+def test_tiled_edge_cases(B, heads, T, H, W, d, th, tw, dtype):
+    q, k, v = workloads.random_inputs(B, heads, T, H, W, d, dtype=dtype, seed=th * 100 + tw,
+                                      scale=1.0 if dtype == torch.bfloat16 else d ** -0.25)
+    got = _run(q, k, v, T, H, W, 1, th, tw)
+    _check(got, oracle.monarch_fwd(q, k, v, T, H, W, 1, th, tw), dtype)
+
+
+def test_large_logits_rescale_path():
+    """Peaked softmax rows (large |q.k|) exercise the running-max rescale."""
+    B, heads, T, H, W, d = 1, 2, 3, 30, 52, 128
+    q, k, v = workloads.random_inputs(B, heads, T, H, W, d, seed=77)
+    # make later key tiles of each frame dominate so the running max grows
+    k = k.float()
+    k.view(B, heads, T, H * W, d)[:, :, :, 1000:] *= 3.0
+    k = k.to(torch.bfloat16)
+    q = (q.float() * 2.0).to(torch.bfloat16)
+    got = _run(q, k, v, T, H, W)
+    _check(got, oracle.monarch_fwd(q, k, v, T, H, W), torch.bfloat16)
+
+
+def test_constant_values_and_zero_qk():
+    T, H, W, d = 4, 10, 14, 128
+    z = torch.zeros(1, 2, T * H * W, d, dtype=torch.bfloat16)
+    v = workloads.random_inputs(1, 2, T, H, W, d, seed=5)[2]
+    got = _run(z, z, v, T, H, W).double()
+    mean = v.double().mean(dim=2, keepdim=True).expand_as(got)
+    assert (got - mean).abs().max() <= BF16_ATOL
+
+
+# ------------------------------------------------------------------ API behaviour
+
+def test_repeat_calls_bitwise_identical_and_streams():
+    wl = workloads.BY_NAME["chunk_bf16"]
+    q, k, v = (x.to(_dev()) for x in workloads.generate(wl))
+    a = binding.monarch_attn_fwd(q, k, v, wl.T, wl.H, wl.W)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = binding.monarch_attn_fwd(q, k, v, wl.T, wl.H, wl.W, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_host_entry_point_matches_device_call():
+    wl = workloads.BY_NAME["chunk_bf16"]
+    q, k, v = workloads.generate(wl)
+    hq, hk, hv = (x.pin_memory() for x in (q, k, v))
+    hout = torch.empty_like(hq).pin_memory()
+    dq, dk, dv, dout = (torch.empty_like(x, device=_dev()) for x in (q, k, v, q))
+    binding.monarch_attn_fwd_host(hq, hk, hv, hout, dq, dk, dv, dout, wl.T, wl.H, wl.W)
+    ref = binding.monarch_attn_fwd(q.to(_dev()), k.to(_dev()), v.to(_dev()), wl.T, wl.H, wl.W).cpu()
+    assert torch.equal(hout, ref)
+
+
+def test_invalid_arguments_are_rejected_without_launch():
+    dev = _dev()
+    x = torch.zeros(1, 1, 2 * 4 * 4, 128, dtype=torch.bfloat16, device=dev)
+    lib = binding.load_library()
+    s = torch.cuda.current_stream().cuda_stream
+    p = x.data_ptr()
+    # out aliasing q
+    assert lib.monarch_attn_fwd(p, p + 0, p, p, 1, 1, 2, 4, 4, 128, 0, 0, 0, 1, s) == 1
+    y = torch.zeros_like(x)
+    # misaligned pointer
+    assert lib.monarch_attn_fwd(p + 2, p, p, y.data_ptr(), 1, 1, 2, 4, 4, 128, 0, 0, 0, 1, s) == 1
+    # bad head width, bad dtype, bad tile
+    assert lib.monarch_attn_fwd(p, p, p, y.data_ptr(), 1, 1, 2, 4, 4, 96, 0, 0, 0, 1, s) == 1
+    assert lib.monarch_attn_fwd(p, p, p, y.data_ptr(), 1, 1, 2, 4, 4, 128, 0, 0, 0, 7, s) == 1
+    assert lib.monarch_attn_fwd(p, p, p, y.data_ptr(), 1, 1, 2, 4, 4, 128, 1, 3, 4, 1, s) == 1
+    # T beyond the supported limit
+    big = torch.zeros(1, 1, 129, 128, dtype=torch.bfloat16, device=dev)
+    big2 = torch.zeros_like(big)
+    assert lib.monarch_attn_fwd(big.data_ptr(), big.data_ptr(), big.data_ptr(), big2.data_ptr(),
+                                1, 1, 129, 1, 1, 128, 0, 0, 0, 1, s) == 2
+    with pytest.raises(binding.MonarchError):
+        binding.monarch_attn_fwd(x, x, x, 2, 4, 4, factorisation=1, tile_h=3, tile_w=4)
+
+
+def test_timeout_machinery_reports_and_context_survives():
+    assert binding.selftest_timeout(2_000_000) == 4  # MONARCH_ERR_TIMEOUT
+    assert binding.last_device_error() == 0          # the self-test cleared the word
+    test_tiny_fp32_full()                             # the context is still usable
