@@ -1,0 +1,399 @@
+"""Benchmark of the Monarch attention forward (one call = one step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the full-clip video latent, B=1, 12 heads, d=128, T=21 frames of
+30x52 tokens (N=32760), frame-aligned factorisation (m=1560, b=21), bf16,
+seeded synthetic inputs (see structured_attention_video_monarch_b200/workloads.py).
+Metric: effective TFLOP/s counting 4*N*(m+b)*d FLOPs per (batch, head), plus
+ms per call and the fraction of the measured B200 bf16 dense peak.
+
+Our arm times K calls with CUDA events on the launching stream, bracketed by a
+barrier and a device synchronisation, and reports the max over ranks.  Each
+rank runs its own full workload (the operator shards over independent
+(batch, head) problems with no collective, so N GPUs run N replicas: weak
+scaling).  Between timed calls the inputs rotate over three buffer sets
+(1.2 GB in all), so every call reads inputs that are not resident in the
+126 MB L2.  The reference arm (--impl reference) times the fp64 CPU oracle on
+a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Monarch attn fwd ms & effective TFLOP/s at N=32760; % of B200 bf16 peak"
+WORKLOAD = "fullclip_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(wl, extra=None):
+    cfg = {
+        "workload": (f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} T={wl.T} H={wl.H} W={wl.W} "
+                     f"(N={wl.N}), {'tiled ' + str(wl.tile_h) + 'x' + str(wl.tile_w) if wl.fact else 'frame'}"
+                     f" split m={wl.m} b={wl.b}"),
+        "global_batch": wl.B,
+        "seq_len": wl.N,
+        "heads": wl.heads,
+        "head_dim": wl.d,
+        "flops_per_call": wl.flops,
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+# ------------------------------------------------------------------ distributed helpers
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(world: int, flops_per_call: float, steps: int, max_seconds: float):
+    """Whole-job throughput: all ranks' FLOPs over the slowest rank's time."""
+    total = world * flops_per_call * steps
+    return total / max_seconds / 1e12, max_seconds * 1e3 / steps
+
+
+# ------------------------------------------------------------------ clock sampling
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r[2] > 300.0] or rows  # samples under load (power draw)
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in load:
+            for name, flag in zip(names, r[3][1:]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+
+def oracle_sample(wl, seconds: float, seed: int = 1234):
+    """Time the fp64 oracle on a bounded sample: G whole stage-2 groups (each =
+    T output rows with their exact stage-1 rows), sized to about `seconds`."""
+    import numpy as np
+    import oracle
+    from structured_attention_video_monarch_b200 import workloads
+    q, k, v = workloads.generate(wl, heads=1)  # one head's problem, same shape per head
+    HW = wl.H * wl.W
+    flops_per_group = 4.0 * wl.T * (wl.m + wl.b) * wl.d
+    rng = np.random.default_rng(seed)
+    g = 8
+    t0 = time.perf_counter()
+    oracle.monarch_fwd_groups(q, k, v, wl.T, wl.H, wl.W,
+                              [(0, int(p)) for p in rng.integers(0, HW, g)], wl.fact, wl.tile_h, wl.tile_w)
+    dt = time.perf_counter() - t0
+    g = max(8, min(HW, int(g * seconds / max(dt, 1e-6))))
+    groups = [(0, int(p)) for p in rng.integers(0, HW, g)]
+    return q, k, v, groups, flops_per_group
+
+
+def time_oracle(wl, q, k, v, groups, flops_per_group):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.monarch_fwd_groups(q, k, v, wl.T, wl.H, wl.W, groups, wl.fact, wl.tile_h, wl.tile_w)
+    dt = time.perf_counter() - t0
+    return len(groups) * flops_per_group / dt / 1e12, dt
+
+
+def run_reference(args):
+    import oracle
+    from structured_attention_video_monarch_b200 import workloads
+    rank, _, world = dist_env()
+    wl = workloads.BY_NAME[args.workload]
+    if rank != 0:
+        return 0
+    oracle.build()
+    budget = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    q, k, v, groups, fpg = oracle_sample(wl, budget)
+    for _ in range(args.warmup):
+        time_oracle(wl, q, k, v, groups, fpg)
+    total = 0.0
+    for _ in range(args.steps):
+        _, dt = time_oracle(wl, q, k, v, groups, fpg)
+        total += dt
+    value = args.steps * len(groups) * fpg / total / 1e12
+    sample = (f"{len(groups)} stage-2 groups x {wl.T} rows of one head per step "
+              f"(exact stage-1 + stage-2 rows, {len(groups) * fpg / 1e9:.2f} GFLOP)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, {"parallelism": "host cores (OpenMP)"}),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from structured_attention_video_monarch_b200 import binding, workloads
+
+    rank, local_rank, world = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    binding.load_library()
+    wl = workloads.BY_NAME[args.workload]
+    peaks, peak_src = load_peaks()
+
+    q0, k0, v0 = workloads.generate(wl)
+    nsets = 3
+    sets = []
+    for sidx in range(nsets):
+        if sidx == 0:
+            q, k, v = q0, k0, v0
+        else:  # same distribution, different seed: distinct buffers so L2 holds none of them
+            q, k, v = workloads.generate(wl, seed=wl.index + 100 * sidx)
+        sets.append(tuple(x.to(device) for x in (q, k, v)) + (torch.empty_like(q0, device=device),))
+    stream = torch.cuda.current_stream(device)
+
+    def call(i, events=None):
+        q, k, v, o = sets[i % nsets]
+        if events is None:
+            binding.monarch_attn_fwd(q, k, v, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w, out=o)
+            return 2
+        return binding.monarch_attn_fwd_profiled(q, k, v, o, wl.T, wl.H, wl.W, events, wl.fact,
+                                                 wl.tile_h, wl.tile_w)
+
+    for i in range(max(3, args.warmup)):
+        call(i)
+    torch.cuda.synchronize(device)
+
+    # clocks under load: sample during a short soak of the same calls, then the timed region
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    t_soak = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_soak < args.soak_seconds:
+        call(i)
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize(device)
+    torch.cuda.synchronize(device)
+
+    # timed region: K calls, events around each kernel launch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for e in (x for row in ev for x in row):
+        e.record(stream)  # torch creates the CUDA event on first record; the library needs the handle
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    launches = 0
+    start.record(stream)
+    for s in range(args.steps):
+        launches += call(s, ev[s])
+    stop.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    elapsed_s = start.elapsed_time(stop) / 1e3
+    stage1_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    stage2_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    max_s = max_over_ranks(elapsed_s, device)
+    value, ms = aggregate(world, wl.flops, args.steps, max_s)
+
+    # roofline of the dominant kernel (stage-1 launch): algorithmic FLOPs / launch time
+    s1_flops = 4.0 * wl.N * wl.m * wl.d * wl.B * wl.heads
+    s1_avg = statistics.mean(stage1_ms) / 1e3
+    s2_avg = statistics.mean(stage2_ms) / 1e3
+    s1_tflops = s1_flops / s1_avg / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    s2_bytes = 4 * wl.B * wl.heads * wl.N * wl.d * 2  # read Q, K, Y1; write O
+    roofline = {
+        "bound": "tensor", "achieved": s1_tflops, "peak": peak, "unit": "TFLOP/s",
+        "frac": s1_tflops / peak, "traffic": args.traffic,
+        "kernel": "monarch_tc_kernel<128> stage-1 launch (block attention, B1 V)",
+        "peak_source": f"{peak_src} bf16_tflops (burst)",
+        "frac_of_sustained": s1_tflops / peak_sus,
+        "algorithmic_flops_per_launch": s1_flops,
+        "launch_ms": s1_avg * 1e3,
+        "stage2_launch": {"bound": "hbm", "ms": s2_avg * 1e3, "algorithmic_bytes": s2_bytes,
+                          "achieved_gbs": s2_bytes / s2_avg / 1e9, "peak_gbs": hbm_peak,
+                          "frac": s2_bytes / s2_avg / 1e9 / hbm_peak},
+    }
+
+    # end to end through the host-buffer entry point: H2D of Q, K, V, the call, D2H of out
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.pin_memory() for x in (q0, k0, v0))
+        hout = torch.empty_like(q0).pin_memory()
+        dq, dk, dv, dout = sets[0]
+        for _ in range(2):
+            binding.monarch_attn_fwd_host(hq, hk, hv, hout, dq, dk, dv, dout, wl.T, wl.H, wl.W,
+                                          wl.fact, wl.tile_h, wl.tile_w)
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            binding.monarch_attn_fwd_host(hq, hk, hv, hout, dq, dk, dv, dout, wl.T, wl.H, wl.W,
+                                          wl.fact, wl.tile_h, wl.tile_w)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
+        e2e_val, e2e_ms = aggregate(world, wl.flops, e2e_steps, e2e_s)
+        nbytes = q0.numel() * q0.element_size()
+        e2e = {"value": e2e_val, "unit": "TFLOP/s", "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            import oracle
+            oracle.build()
+            qs, ks, vs, groups, fpg = oracle_sample(wl, args.cpu_seconds)
+            val, dt = time_oracle(wl, qs, ks, vs, groups, fpg)
+            cpu = {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                   "sample": (f"{len(groups)} stage-2 groups x {wl.T} rows of one head "
+                              f"({len(groups) * fpg / 1e9:.2f} GFLOP, {dt:.1f} s)")}
+        except Exception as exc:  # the CPU baseline is a report, not the product
+            cpu = {"value": None, "unit": "TFLOP/s", "cores": None, "kind": "oracle",
+                   "sample": f"failed: {exc}"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wl, {
+                "parallelism": f"replicas x{world} (independent (batch, head) problems; no collective)",
+                "l2": "inputs larger than L2: 3 rotating buffer sets of Q, K, V, out (1.2 GB)"}),
+            "pct_of_bf16_peak": {"measured_burst": value / world / peak,
+                                 "measured_sustained": value / world / peak_sus,
+                                 "datasheet_2250": value / world / 2250.0},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "stage_ms": {"stage1": s1_avg * 1e3, "stage2": s2_avg * 1e3},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--soak-seconds", type=float, default=2.0)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -107,6 +107,21 @@ int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, voi
                           int factorisation, int tile_h, int tile_w, int dtype,
                           void *stream);
 
+/*
+ * monarch_attn_fwd_profiled -- monarch_attn_fwd that also records CUDA events
+ * on `stream` so a caller can time each kernel launch of the call:
+ * events[0] before the first launch and events[i + 1] after launch i.
+ * `events` holds `nevents` cudaEvent_t handles created by the caller
+ * (entries beyond what the call needs are left untouched; NULL entries are
+ * skipped).  *nlaunch (if not NULL) receives the number of kernel launches
+ * the call queued: 2 (stage 1, then stage 2).  Same arguments, rules and
+ * status codes as monarch_attn_fwd otherwise.
+ */
+int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void *out,
+                              int B, int heads, int T, int H, int W, int d,
+                              int factorisation, int tile_h, int tile_w, int dtype,
+                              void *stream, void **events, int nevents, int *nlaunch);
+
 /* Human-readable text of a status code; never NULL, owned by the library. */
 const char *monarch_attn_strerror(int status);
 

@@ -47,6 +47,9 @@ def load_library(path: str | None = None):
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.monarch_attn_fwd.argtypes = [vp, vp, vp, vp] + [i] * 10 + [vp]
     lib.monarch_attn_fwd.restype = i
+    lib.monarch_attn_fwd_profiled.argtypes = ([vp, vp, vp, vp] + [i] * 10 +
+                                              [vp, ctypes.POINTER(vp), i, ctypes.POINTER(i)])
+    lib.monarch_attn_fwd_profiled.restype = i
     lib.monarch_attn_fwd_host.argtypes = [vp] * 8 + [i] * 10 + [vp]
     lib.monarch_attn_fwd_host.restype = i
     lib.monarch_attn_strerror.argtypes = [i]
@@ -109,6 +112,23 @@ def monarch_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, T: int, 
     if st != 0:
         raise MonarchError(st, "monarch_attn_fwd")
     return out
+
+
+def monarch_attn_fwd_profiled(q, k, v, out, T, H, W, events, factorisation=FACT_FRAME, tile_h=0,
+                              tile_w=0, stream=None) -> int:
+    """monarch_attn_fwd recording ``events`` (torch.cuda.Event list) around each
+    kernel launch: events[0] before the first, events[i+1] after launch i.
+    Returns the number of kernel launches queued."""
+    B, heads, N, d = q.shape
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    n = ctypes.c_int(0)
+    st = load_library().monarch_attn_fwd_profiled(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, heads, T, H, W, d,
+        int(factorisation), int(tile_h), int(tile_w), _dtype_code(q), _stream_ptr(stream),
+        arr, len(events), ctypes.byref(n))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_profiled")
+    return n.value
 
 
 def monarch_attn_fwd_host(h_q, h_k, h_v, h_out, d_q, d_k, d_v, d_out, T, H, W,

@@ -601,8 +601,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         const float x0 = s[32 * c + 2 * e], x1 = s[32 * c + 2 * e + 1];
                         const float a = (x0 == -INFINITY) ? 0.f : fast_exp2(fmaf(x0, sl2, -moff));
                         const float b = (x1 == -INFINITY) ? 0.f : fast_exp2(fmaf(x1, sl2, -moff));
-                        lsum += a + b;
                         pk[e] = pack_bf16x2(a, b);
+                        // the denominator sums the bf16-rounded weights the PV
+                        // MMA actually uses, so a dominant weight cancels exactly
+                        lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
                     }
                     tmem_st16(lane_base + col_s + 16 * c, pk);
                 }

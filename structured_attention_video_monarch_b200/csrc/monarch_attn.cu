@@ -161,9 +161,19 @@ int stage2_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams
     return make_map(map, ptr, 4, dims, strides, box);
 }
 
+// Optional per-launch events: ev[0] before the first launch, ev[i+1] after launch i.
+struct LaunchEvents {
+    void **ev = nullptr;
+    int n = 0;
+    int launches = 0;
+    void record(int idx, cudaStream_t s) const {
+        if (ev && idx < n && ev[idx]) cudaEventRecord(static_cast<cudaEvent_t>(ev[idx]), s);
+    }
+};
+
 template <int D>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
-              cudaStream_t stream) {
+              cudaStream_t stream, LaunchEvents &lev) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
@@ -217,6 +227,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
 
     // stage 1: Y1 = B1 V into out; stage 2: out = P^T B2 P Y1 in place.
     const long long ranges[2][2] = {{0, p.s1_units}, {p.s1_units, p.s1_units + p.s2_units}};
+    lev.record(0, stream);
     for (int r = 0; r < 2; ++r) {
         p.unit_begin = ranges[r][0];
         p.unit_end = ranges[r][1];
@@ -225,13 +236,14 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         const int grid = static_cast<int>(units < di->sms ? units : di->sms);
         monarch_tc_kernel<D><<<grid, 512, L::ALLOC, stream>>>(mq1, mk1, mv1, mo1, mq2, mk2, my2, mo2, p);
         if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+        lev.record(++lev.launches, stream);
     }
     return MONARCH_OK;
 }
 
 template <int D>
 int launch_f32(const void *q, const void *k, const void *v, void *out, const Shape &s,
-               cudaStream_t stream) {
+               cudaStream_t stream, LaunchEvents &lev) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
@@ -265,11 +277,14 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
     const float *fk = static_cast<const float *>(k);
     const float *fv = static_cast<const float *>(v);
     float *fo = static_cast<float *>(out);
+    lev.record(0, stream);
     monarch_f32_stage1<D><<<static_cast<unsigned>(g1), 128, 0, stream>>>(fq, fk, fv, fo, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    lev.record(++lev.launches, stream);
     const int threads2 = ((2 * s.T + 31) / 32) * 32;
     monarch_f32_stage2<D><<<static_cast<unsigned>(g2), threads2, smem2, stream>>>(fq, fk, fo, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    lev.record(++lev.launches, stream);
     return MONARCH_OK;
 }
 
@@ -308,20 +323,40 @@ using namespace monarch;
 
 extern "C" {
 
-int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out, int B, int heads, int T,
-                     int H, int W, int d, int factorisation, int tile_h, int tile_w, int dtype,
-                     void *stream) {
+static int fwd_impl(const void *q, const void *k, const void *v, void *out, int B, int heads, int T,
+                    int H, int W, int d, int factorisation, int tile_h, int tile_w, int dtype,
+                    void *stream, LaunchEvents &lev) {
     Shape s{B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
     int st = validate(q, k, v, out, s);
     if (st) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (dtype == MONARCH_DTYPE_BF16)
-        st = d == 128 ? launch_tc<128>(q, k, v, out, s, cs) : launch_tc<64>(q, k, v, out, s, cs);
+        st = d == 128 ? launch_tc<128>(q, k, v, out, s, cs, lev) : launch_tc<64>(q, k, v, out, s, cs, lev);
     else
-        st = d == 128 ? launch_f32<128>(q, k, v, out, s, cs) : launch_f32<64>(q, k, v, out, s, cs);
+        st = d == 128 ? launch_f32<128>(q, k, v, out, s, cs, lev) : launch_f32<64>(q, k, v, out, s, cs, lev);
     if (st) return st;
     if (env_debug()) return read_status(cs, 0);
     return MONARCH_OK;
+}
+
+int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out, int B, int heads, int T,
+                     int H, int W, int d, int factorisation, int tile_h, int tile_w, int dtype,
+                     void *stream) {
+    LaunchEvents lev;
+    return fwd_impl(q, k, v, out, B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, stream,
+                    lev);
+}
+
+int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void *out, int B, int heads,
+                              int T, int H, int W, int d, int factorisation, int tile_h, int tile_w,
+                              int dtype, void *stream, void **events, int nevents, int *nlaunch) {
+    LaunchEvents lev;
+    lev.ev = events;
+    lev.n = events ? nevents : 0;
+    const int st = fwd_impl(q, k, v, out, B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype,
+                            stream, lev);
+    if (nlaunch) *nlaunch = lev.launches;
+    return st;
 }
 
 int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, void *h_out, void *d_q,
