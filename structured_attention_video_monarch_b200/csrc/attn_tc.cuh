@@ -1,36 +1,40 @@
 // attn_tc.cuh -- bf16 Monarch attention stages on tcgen05 tensor cores.
 //
-// One persistent kernel runs "units" of block-diagonal softmax attention.
-// A unit is a pair of 128-row query tiles that share their keys:
-//   stage-1 unit: two query tiles of one stage-1 block (a frame, or a spatial
-//     tile of a frame), iterating over that block's key/value tiles with an
-//     online softmax; values are V, results (Y1) go to `out`;
-//   stage-2 unit: two "group chunks"; each chunk stacks npos spatial positions
-//     x T frames (npos*T <= 128 rows) fetched with one TMA box, so the
-//     permutation P of the Monarch factorisation is pure tensor-map
-//     addressing.  Keys are the same stacked rows; a block-diagonal mask keeps
-//     each row inside its own position's group; values are Y1 read back from
-//     `out`, results overwrite `out`.
+// One persistent kernel runs "units" of block-diagonal softmax attention
 // (MonarchRT: Efficient Attention for Real-Time Video Generation,
-// gist.science/nl/paper/2602.12271 "Methodologie"; gist.science/zh/paper/
-// 2602.12271 section 2.2 on block alignment and tiled Monarch; the pages'
-// kernels tile attention FlashAttention-style in on-chip memory without
-// materialising the dense map, section 2.2 "Finetuning & Efficient
-// Implementation".)
+// gist.science/nl/paper/2602.12271 "Methodologie": permutation and
+// block-diagonal factors; gist.science/zh/paper/2602.12271 section 2.2: blocks
+// aligned with the video axes, tiled Monarch, and FlashAttention-style tiling
+// in on-chip memory without materialising the dense map).
+//
+// A unit has two "lanes"; each lane is one 128-row query tile:
+//   stage-1 lane: a query tile of one stage-1 block (a frame, or a spatial
+//     tile of a frame); it iterates over that block's key/value tiles with an
+//     online softmax; values are V; results (Y1) go to `out`.
+//   stage-2 lane: a "group chunk" stacking npos spatial positions x T frames
+//     (npos*T <= 128 rows) fetched with one TMA box, so the permutation P of
+//     the factorisation is pure tensor-map addressing.  Keys are the same
+//     stacked rows, a block-diagonal mask keeps each row inside its own
+//     position's group, values are Y1 read back from `out`, results
+//     overwrite `out`.
+// The two lanes of a unit share their key/value tiles when they are two query
+// tiles of the same block ("shared" units); otherwise each lane streams its
+// own keys ("separate" units: the odd last query tile of two blocks, and
+// every stage-2 unit).
 //
 // Warp roles (512 threads, registers rebalanced with setmaxnreg):
-//   warps 0-3   softmax for query tile 0 (thread = row)        192 regs
-//   warps 4-7   softmax for query tile 1                        192 regs
-//   warps 8-11  epilogue: O / l -> bf16 -> shared -> TMA store   72 regs
-//   warp  12    TMA producer (Q tiles, K/V ring)                 56 regs
+//   warps 0-3   softmax for lane 0 (thread = row)                  192 regs
+//   warps 4-7   softmax for lane 1                                  192 regs
+//   warps 8-11  epilogue: O / l -> bf16 -> global stores             64 regs
+//   warp  12    TMA producer (Q tiles, K/V ring)                     64 regs
 //   warp  13    TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 14-15 idle
-// (2*128*192 + 128*72 + 128*56 = 65536, the registers the block launches with.)
+// (2*128*192 + 128*64 + 128*64 = 65536, the registers the block launches with.)
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0, O1 after them.
 // P (bf16) overwrites the first 64 columns of its S region and feeds the PV
 // MMA straight from TMEM.  The MMA issue order per key tile j is
 //   PV0(j-1), S0(j), PV1(j-1), S1(j)
-// so one tile's softmax overlaps the other tile's MMAs; tcgen05.mma ops from
+// so one lane's softmax overlaps the other lane's MMAs; tcgen05.mma ops from
 // one thread execute in order, which makes S_i(j+1) safe after PV_i(j).
 #pragma once
 
@@ -42,13 +46,17 @@ enum : int { UNIT_STAGE1 = 1, UNIT_STAGE2 = 2 };
 
 struct TcParams {
     int B, heads, T, H, W, HW;
+    long long N;                    // tokens per (batch, head)
     int fact;                       // 0 frame, 1 tiled
     int tile_h, tile_w, tiles_h, tiles_w;
     int rows_per_tile;              // tiled: tile rows per 128-row query/key tile
     int m;                          // tokens per stage-1 block
     int nblk_bh;                    // stage-1 blocks per (batch, head)
+    int nblocks;                    // stage-1 blocks in all
     int nqt;                        // 128-row query (= key) tiles per stage-1 block
-    int s1_pairs;                   // ceil(nqt / 2)
+    int ns;                         // shared pairs per block: nqt / 2
+    int odd;                        // nqt % 2
+    int upg;                        // units per group of two blocks: 2*ns + odd
     int npos;                       // stage-2 positions per chunk
     int s2_chunks;                  // chunks per (batch, head)
     int s2_pairs;                   // ceil(s2_chunks / 2)
@@ -57,60 +65,84 @@ struct TcParams {
     float scale_log2;               // d^-1/2 * log2(e)
     long long timeout_cycles;
     unsigned *status;
+    void *out;                      // bf16 output (epilogue stores)
+};
+
+struct Lane {
+    int blk;   // stage 1: global block index; stage 2: batch-head
+    int tile;  // stage 1: query tile inside the block; stage 2: chunk
 };
 
 struct Unit {
     int kind;
-    int nq;          // query tiles present (1 or 2)
-    int nk;          // key/value tiles
-    int bh;
-    // stage 1
-    int blk;         // global stage-1 block index
-    int qt0;         // first query tile index inside the block
-    // stage 2
-    int chunk0;
+    int nq;      // lanes present (1 or 2)
+    int nk;      // key/value tiles per lane
+    int shared;  // lanes share key/value tiles
+    Lane ln[2];
 };
 
 __device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
     Unit r;
     if (u < p.s1_units) {
         r.kind = UNIT_STAGE1;
-        long long blk = u / p.s1_pairs;
-        int pair = static_cast<int>(u % p.s1_pairs);
-        r.blk = static_cast<int>(blk);
-        r.bh = static_cast<int>(blk / p.nblk_bh);
-        r.qt0 = 2 * pair;
-        r.nq = (r.qt0 + 1 < p.nqt) ? 2 : 1;
         r.nk = p.nqt;
-        r.chunk0 = 0;
+        const long long g = u / p.upg;
+        const int rr = static_cast<int>(u - g * p.upg);
+        const int b0 = static_cast<int>(2 * g);
+        const bool two = b0 + 1 < p.nblocks;
+        if (rr < p.ns || (two && rr < 2 * p.ns)) {
+            const int blk = rr < p.ns ? b0 : b0 + 1;
+            const int pr = rr < p.ns ? rr : rr - p.ns;
+            r.shared = 1;
+            r.nq = 2;
+            r.ln[0] = {blk, 2 * pr};
+            r.ln[1] = {blk, 2 * pr + 1};
+        } else {  // the odd last tiles of blocks b0 and b0+1
+            r.shared = 0;
+            r.nq = two ? 2 : 1;
+            r.ln[0] = {b0, p.nqt - 1};
+            r.ln[1] = {two ? b0 + 1 : b0, p.nqt - 1};
+        }
     } else {
-        long long v = u - p.s1_units;
+        const long long v = u - p.s1_units;
         r.kind = UNIT_STAGE2;
-        r.bh = static_cast<int>(v / p.s2_pairs);
-        int pair = static_cast<int>(v % p.s2_pairs);
-        r.chunk0 = 2 * pair;
-        r.nq = (r.chunk0 + 1 < p.s2_chunks) ? 2 : 1;
         r.nk = 1;
-        r.blk = 0;
-        r.qt0 = 0;
+        r.shared = 0;
+        const int bh = static_cast<int>(v / p.s2_pairs);
+        const int c0 = 2 * static_cast<int>(v % p.s2_pairs);
+        r.nq = (c0 + 1 < p.s2_chunks) ? 2 : 1;
+        r.ln[0] = {bh, c0};
+        r.ln[1] = {bh, c0 + 1};
     }
     return r;
 }
 
-// Rows a stage-1 tile (query or key tile `tile` of block `blk`) brings in by
-// TMA, and how many of them are real tokens of the block.
-__device__ __forceinline__ void s1_tile_rows(const TcParams &p, int tile, int &loaded,
-                                             int &valid) {
+// Rows a stage-1 tile (query or key tile `tile` of a block) brings in by TMA,
+// and how many of them are real tokens of the block.
+__device__ __forceinline__ void s1_tile_rows(const TcParams &p, int tile, int &loaded, int &valid) {
     if (p.fact == 0) {
         loaded = 128;  // rows past the block end are zero-filled by TMA
-        int rem = p.m - tile * 128;
+        const int rem = p.m - tile * 128;
         valid = rem < 128 ? rem : 128;
     } else {
         loaded = p.rows_per_tile * p.tile_w;
-        int rem_rows = p.tile_h - tile * p.rows_per_tile;
-        int rows = rem_rows < p.rows_per_tile ? rem_rows : p.rows_per_tile;
+        const int rem_rows = p.tile_h - tile * p.rows_per_tile;
+        const int rows = rem_rows < p.rows_per_tile ? rem_rows : p.rows_per_tile;
         valid = rows * p.tile_w;
     }
+}
+
+// Valid key columns of key tile j of a unit, and the MMA extent covering them
+// (N of the QK^T MMA and K of the PV MMA: a multiple of 16, at most 128).
+__device__ __forceinline__ void key_extent(const TcParams &p, const Unit &un, int j, int &kvalid,
+                                           int &ext) {
+    if (un.kind == UNIT_STAGE1) {
+        int loaded;
+        s1_tile_rows(p, j, loaded, kvalid);
+    } else {
+        kvalid = p.npos * p.T;
+    }
+    ext = (kvalid + 15) & ~15;
 }
 
 // Issue the TMA load of one stage-1 tile (all panels) into dst.
@@ -119,12 +151,11 @@ __device__ __forceinline__ void s1_load(const TcParams &p, const CUtensorMap *ma
                                         uint32_t bar, int blk, int tile) {
     if (p.fact == 0) {
 #pragma unroll
-        for (int pn = 0; pn < NP; ++pn)
-            tma_load_3d(dst + pn * 16384, map, bar, pn * 64, tile * 128, blk);
+        for (int pn = 0; pn < NP; ++pn) tma_load_3d(dst + pn * 16384, map, bar, pn * 64, tile * 128, blk);
     } else {
-        int tpf = p.tiles_h * p.tiles_w;
-        int frame = blk / tpf, tif = blk % tpf;
-        int ti = tif / p.tiles_w, tj = tif % p.tiles_w;
+        const int tpf = p.tiles_h * p.tiles_w;
+        const int frame = blk / tpf, tif = blk % tpf;
+        const int ti = tif / p.tiles_w, tj = tif % p.tiles_w;
 #pragma unroll
         for (int pn = 0; pn < NP; ++pn)
             tma_load_5d(dst + pn * 16384, map, bar, pn * 64, 0, tj, tile * p.rows_per_tile,
@@ -133,50 +164,52 @@ __device__ __forceinline__ void s1_load(const TcParams &p, const CUtensorMap *ma
 }
 
 template <int NP>
-__device__ __forceinline__ void s1_store(const TcParams &p, const CUtensorMap *map, uint32_t src,
-                                         int blk, int tile) {
-    if (p.fact == 0) {
+__device__ __forceinline__ void s2_load(const CUtensorMap *map, uint32_t dst, uint32_t bar, int npos,
+                                        int bh, int chunk) {
 #pragma unroll
-        for (int pn = 0; pn < NP; ++pn) tma_store_3d(map, src + pn * 16384, pn * 64, tile * 128, blk);
-    } else {
-        int tpf = p.tiles_h * p.tiles_w;
-        int frame = blk / tpf, tif = blk % tpf;
-        int ti = tif / p.tiles_w, tj = tif % p.tiles_w;
-#pragma unroll
-        for (int pn = 0; pn < NP; ++pn)
-            tma_store_5d(map, src + pn * 16384, pn * 64, 0, tj, tile * p.rows_per_tile,
-                         frame * p.tiles_h + ti);
+    for (int pn = 0; pn < NP; ++pn) tma_load_4d(dst + pn * 16384, map, bar, pn * 64, chunk * npos, 0, bh);
+}
+
+// Output token (index inside its batch-head) of row `row` of a lane, or -1
+// when the row is padding.  bh receives the lane's batch-head.
+__device__ __forceinline__ long long lane_row_token(const TcParams &p, int kind, const Lane &ln, int row,
+                                                    int &bh) {
+    if (kind == UNIT_STAGE1) {
+        bh = ln.blk / p.nblk_bh;
+        const int b = ln.blk - bh * p.nblk_bh;
+        if (p.fact == 0) {
+            const int i = ln.tile * 128 + row;
+            if (i >= p.m) return -1;
+            return static_cast<long long>(b) * p.HW + i;
+        }
+        const int tpf = p.tiles_h * p.tiles_w;
+        const int t = b / tpf, tif = b % tpf;
+        const int ti = tif / p.tiles_w, tj = tif % p.tiles_w;
+        const int rr = row / p.tile_w, wl = row - rr * p.tile_w;
+        const int hl = ln.tile * p.rows_per_tile + rr;
+        if (rr >= p.rows_per_tile || hl >= p.tile_h) return -1;
+        return static_cast<long long>(t) * p.HW + static_cast<long long>(ti * p.tile_h + hl) * p.W +
+               tj * p.tile_w + wl;
     }
-}
-
-template <int NP>
-__device__ __forceinline__ void s2_load(const CUtensorMap *map, uint32_t dst, uint32_t bar,
-                                        int npos, int bh, int chunk) {
-#pragma unroll
-    for (int pn = 0; pn < NP; ++pn)
-        tma_load_4d(dst + pn * 16384, map, bar, pn * 64, chunk * npos, 0, bh);
-}
-
-template <int NP>
-__device__ __forceinline__ void s2_store(const CUtensorMap *map, uint32_t src, int npos, int bh,
-                                         int chunk) {
-#pragma unroll
-    for (int pn = 0; pn < NP; ++pn) tma_store_4d(map, src + pn * 16384, pn * 64, chunk * npos, 0, bh);
+    bh = ln.blk;
+    const int t = row / p.npos, pl = row - t * p.npos;
+    const int pos = ln.tile * p.npos + pl;
+    if (t >= p.T || pos >= p.HW) return -1;
+    return static_cast<long long>(t) * p.HW + pos;
 }
 
 template <int D>
 struct TcLayout {
     static constexpr int NP = D / 64;                 // 64-element (128-byte) panels per row
     static constexpr int TILE = 128 * D * 2;          // bytes of one 128-row tile
-    static constexpr int NS = (D == 128) ? 3 : 6;     // K/V ring slots
+    static constexpr int NS = (D == 128) ? 5 : 8;     // K/V ring slots
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = OFF_Q + 2 * TILE;
-    static constexpr int OFF_STG = OFF_KV + NS * TILE;
-    static constexpr int OFF_BAR = OFF_STG + 2 * TILE;
+    static constexpr int OFF_BAR = OFF_KV + NS * TILE;
     // barriers: q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2]
     //           o_full[2] o_free[2] l_full[2] l_free[2]
     static constexpr int NBAR = 16 + 2 * NS;
-    static constexpr int OFF_L = OFF_BAR + NBAR * 8;     // row sums l, [2 tiles][128 rows] fp32
+    static constexpr int OFF_L = OFF_BAR + NBAR * 8;     // row sums l, [2 lanes][128 rows] fp32
     static constexpr int OFF_MISC = OFF_L + 2 * 128 * 4; // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;        // slack to align the base to 1024
@@ -184,11 +217,11 @@ struct TcLayout {
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
 };
 
-// Zero rows [from, 128) of every panel of a 128-row tile (generic proxy),
-// so that the PV MMA reads exact zeros where no value row was loaded.
+// Zero rows [from, to) of every panel of a 128-row tile (generic proxy), so
+// that the PV MMA reads exact zeros where no value row was loaded.
 template <int NP>
-__device__ __forceinline__ void zero_tail_rows(uint32_t tile, int from) {
-    for (int r = from; r < 128; ++r)
+__device__ __forceinline__ void zero_rows(uint32_t tile, int from, int to) {
+    for (int r = from; r < to; ++r)
 #pragma unroll
         for (int pn = 0; pn < NP; ++pn)
 #pragma unroll
@@ -198,19 +231,74 @@ __device__ __forceinline__ void zero_tail_rows(uint32_t tile, int from) {
 __device__ __forceinline__ void setmaxnreg_inc192() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
 }
-__device__ __forceinline__ void setmaxnreg_dec72() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
+__device__ __forceinline__ void setmaxnreg_dec64() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
 }
-__device__ __forceinline__ void setmaxnreg_dec56() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+
+// ---------------------------------------------------------------- softmax math
+
+// 2^x for a pair of floats on the FMA pipe (offloads the MUFU unit).
+// Range reduction 2^x = 2^j * 2^f, j = floor(x), f in [0, 1): j comes from a
+// round-down add of 1.5*2^23 (the integer lands in the low mantissa bits, and
+// shifting those bits left by 23 puts j straight into the exponent field);
+// 2^f ~= 1 + f*(a1 + f*(a2 + f*a3)), a cubic fitted here for minimal relative
+// error with p(0) = 1, p(1) = 2 (max relative error 1.03e-4, below bf16's
+// 2^-9 rounding of P).  x is clamped to -126 so 2^j stays a normal number.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    const uint64_t x = pack_f32x2(x0, x1);
+    const uint64_t t = add_rm_f32x2(x, pack_f32x2(12582912.f, 12582912.f));
+    const uint64_t jf = add_f32x2(t, pack_f32x2(-12582912.f, -12582912.f));
+    const uint64_t f = sub_f32x2(x, jf);
+    uint64_t q = fma_f32x2(f, pack_f32x2(0.07826797f, 0.07826797f), pack_f32x2(0.22630768f, 0.22630768f));
+    q = fma_f32x2(q, f, pack_f32x2(0.6954244f, 0.6954244f));
+    q = fma_f32x2(q, f, pack_f32x2(1.f, 1.f));
+    float q0, q1, t0, t1;
+    unpack_f32x2(q, q0, q1);
+    unpack_f32x2(t, t0, t1);
+    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
+// bf16 pairs, and accumulate the rounded P into acc (two fp32 partial sums).
+// With EMULATE, 5 of the 16 pairs go through exp2_poly_pair, the rest
+// through MUFU ex2.
+template <bool EMULATE, int C>
+__device__ __forceinline__ void softmax_chunk(const float (&s)[128], float sl2, float moff,
+                                              uint32_t (&pk)[16], uint64_t &acc) {
+    const uint64_t scale = pack_f32x2(sl2, sl2);
+    const uint64_t off = pack_f32x2(-moff, -moff);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const uint64_t x = fma_f32x2(pack_f32x2(s[32 * C + 2 * e], s[32 * C + 2 * e + 1]), scale, off);
+        float x0, x1, a, b;
+        unpack_f32x2(x, x0, x1);
+        if (EMULATE && (e % 3 == 1)) {
+            exp2_poly_pair(x0, x1, a, b);
+        } else {
+            a = fast_exp2(x0);
+            b = fast_exp2(x1);
+        }
+        const uint32_t w = pack_bf16x2(a, b);
+        pk[e] = w;
+        // the denominator sums the bf16-rounded weights the PV MMA uses
+        acc = add_f32x2(acc, pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
+    }
 }
 
 template <int D>
 __global__ void __launch_bounds__(512, 1)
 monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant__ CUtensorMap mk1,
-                  const __grid_constant__ CUtensorMap mv1, const __grid_constant__ CUtensorMap mo1,
-                  const __grid_constant__ CUtensorMap mq2, const __grid_constant__ CUtensorMap mk2,
-                  const __grid_constant__ CUtensorMap my2, const __grid_constant__ CUtensorMap mo2,
+                  const __grid_constant__ CUtensorMap mv1, const __grid_constant__ CUtensorMap mq2,
+                  const __grid_constant__ CUtensorMap mk2, const __grid_constant__ CUtensorMap my2,
                   const TcParams p) {
     using L = TcLayout<D>;
     constexpr int NP = L::NP;
@@ -260,8 +348,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     }
     if (warp == 12 && lane == 0) {
         tma_prefetch_desc(&mq1); tma_prefetch_desc(&mk1); tma_prefetch_desc(&mv1);
-        tma_prefetch_desc(&mo1); tma_prefetch_desc(&mq2); tma_prefetch_desc(&mk2);
-        tma_prefetch_desc(&my2); tma_prefetch_desc(&mo2);
+        tma_prefetch_desc(&mq2); tma_prefetch_desc(&mk2); tma_prefetch_desc(&my2);
     }
     if (warp == 13) {
         tmem_alloc(smem_addr(tmem_slot), L::TMEM_COLS);
@@ -273,7 +360,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     const uint32_t tmem = *tmem_slot;
 
     if (wg == 3) {
-        setmaxnreg_dec56();
+        setmaxnreg_dec64();
         if (warp == 12 && lane == 0) {
             // -------------------------------------------------------- TMA producer
             uint32_t qe_par = 3u;  // bit i: parity to wait for on q_empty(i)
@@ -282,9 +369,33 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             bool ok = true;
             auto acquire_slot = [&](int &s) -> bool {
                 s = slot;
-                bool r = mbar_wait(kv_empty(slot), (kv_round & 1u) ^ 1u, ctl);
+                const bool r = mbar_wait(kv_empty(slot), (kv_round & 1u) ^ 1u, ctl);
                 if (++slot == NS) { slot = 0; ++kv_round; }
                 return r;
+            };
+            // one key or value tile of lane `ln` (stage 1: block tile j; stage 2: chunk)
+            auto load_kv = [&](const Unit &un, const Lane &ln, int j, bool is_v) -> bool {
+                int s;
+                if (!acquire_slot(s)) return false;
+                const uint32_t dst = base + L::OFF_KV + s * L::TILE;
+                int loaded, kvalid, ext;
+                key_extent(p, un, j, kvalid, ext);
+                if (un.kind == UNIT_STAGE1) {
+                    int valid;
+                    s1_tile_rows(p, j, loaded, valid);
+                } else {
+                    loaded = p.npos * p.T;
+                }
+                if (is_v && loaded < ext) {  // rows the PV MMA reads but TMA does not write
+                    zero_rows<NP>(dst, loaded, ext);
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive_expect_tx(kv_full(s), NP * loaded * 128);
+                if (un.kind == UNIT_STAGE1)
+                    s1_load<NP>(p, is_v ? &mv1 : &mk1, dst, kv_full(s), ln.blk, j);
+                else
+                    s2_load<NP>(is_v ? &my2 : &mk2, dst, kv_full(s), p.npos, ln.blk, ln.tile);
+                return true;
             };
             for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
@@ -295,59 +406,25 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     const uint32_t dst = base + L::OFF_Q + i * L::TILE;
                     if (un.kind == UNIT_STAGE1) {
                         int loaded, valid;
-                        s1_tile_rows(p, un.qt0 + i, loaded, valid);
+                        s1_tile_rows(p, un.ln[i].tile, loaded, valid);
                         mbar_arrive_expect_tx(q_full(i), NP * loaded * 128);
-                        s1_load<NP>(p, &mq1, dst, q_full(i), un.blk, un.qt0 + i);
+                        s1_load<NP>(p, &mq1, dst, q_full(i), un.ln[i].blk, un.ln[i].tile);
                     } else {
                         mbar_arrive_expect_tx(q_full(i), NP * p.npos * p.T * 128);
-                        s2_load<NP>(&mq2, dst, q_full(i), p.npos, un.bh, un.chunk0 + i);
+                        s2_load<NP>(&mq2, dst, q_full(i), p.npos, un.ln[i].blk, un.ln[i].tile);
                     }
                 }
-                if (!ok) break;
-                if (un.kind == UNIT_STAGE1) {
-                    for (int j = 0; j < un.nk && ok; ++j) {
-                        int loaded, valid;
-                        s1_tile_rows(p, j, loaded, valid);
-                        int s;
-                        if (!(ok = acquire_slot(s))) break;
-                        uint32_t dst = base + L::OFF_KV + s * L::TILE;
-                        mbar_arrive_expect_tx(kv_full(s), NP * loaded * 128);
-                        s1_load<NP>(p, &mk1, dst, kv_full(s), un.blk, j);
-                        if (!(ok = acquire_slot(s))) break;
-                        dst = base + L::OFF_KV + s * L::TILE;
-                        if (loaded < 128) {
-                            zero_tail_rows<NP>(dst, loaded);
-                            fence_proxy_async_smem();
-                        }
-                        mbar_arrive_expect_tx(kv_full(s), NP * loaded * 128);
-                        s1_load<NP>(p, &mv1, dst, kv_full(s), un.blk, j);
-                    }
-                } else {
-                    const int rows = p.npos * p.T;
-                    for (int i = 0; i < un.nq && ok; ++i) {
-                        int s;
-                        if (!(ok = acquire_slot(s))) break;
-                        const uint32_t dst = base + L::OFF_KV + s * L::TILE;
-                        mbar_arrive_expect_tx(kv_full(s), NP * rows * 128);
-                        s2_load<NP>(&mk2, dst, kv_full(s), p.npos, un.bh, un.chunk0 + i);
-                    }
-                    for (int i = 0; i < un.nq && ok; ++i) {
-                        int s;
-                        if (!(ok = acquire_slot(s))) break;
-                        const uint32_t dst = base + L::OFF_KV + s * L::TILE;
-                        if (rows < 128) {
-                            zero_tail_rows<NP>(dst, rows);
-                            fence_proxy_async_smem();
-                        }
-                        mbar_arrive_expect_tx(kv_full(s), NP * rows * 128);
-                        s2_load<NP>(&my2, dst, kv_full(s), p.npos, un.bh, un.chunk0 + i);
+                for (int j = 0; j < un.nk && ok; ++j) {
+                    if (un.shared) {
+                        ok = load_kv(un, un.ln[0], j, false) && load_kv(un, un.ln[0], j, true);
+                    } else {
+                        for (int i = 0; i < un.nq && ok; ++i) ok = load_kv(un, un.ln[i], j, false);
+                        for (int i = 0; i < un.nq && ok; ++i) ok = load_kv(un, un.ln[i], j, true);
                     }
                 }
             }
         } else if (warp == 13 && lane == 0) {
             // -------------------------------------------------------- MMA issuer
-            constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
             uint32_t qf_par = 0u;  // bit i: parity to wait for on q_full(i)
             uint32_t pf_par = 0u;  // bit i: parity to wait for on p_full(i)
             uint32_t of_par = 3u;  // bit i: parity to wait for on o_free(i)
@@ -356,30 +433,32 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             bool ok = true;
             auto acquire_full = [&](int &s) -> bool {
                 s = slot;
-                bool r = mbar_wait(kv_full(slot), kv_round & 1u, ctl);
+                const bool r = mbar_wait(kv_full(slot), kv_round & 1u, ctl);
                 if (++slot == NS) { slot = 0; ++kv_round; }
                 return r;
             };
-            // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D.
-            auto issue_s = [&](int i, int s) {
+            // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D,
+            // N = ext key columns.
+            auto issue_s = [&](int i, int s, int ext) {
                 const uint32_t qa = base + L::OFF_Q + i * L::TILE;
                 const uint32_t kb = base + L::OFF_KV + s * L::TILE;
                 const uint32_t d_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
+                const uint32_t idesc = idesc_bf16_f32(128, ext, false, false);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_ss(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                           IDESC_S, k > 0 ? 1u : 0u);
+                    mma_ss(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc,
+                           k > 0 ? 1u : 0u);
                 }
             };
             // O_i (+)= P_i V: A = P from TMEM (bf16 pairs in the S region),
-            // B = V tile (MN-major: keys x D, D contiguous), K dim = 128 keys.
-            auto issue_pv = [&](int i, int s, uint32_t acc) {
+            // B = V tile (MN-major: keys x D, D contiguous), K dim = ext keys.
+            auto issue_pv = [&](int i, int s, int ext, uint32_t acc) {
+                constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
                 const uint32_t vb = base + L::OFF_KV + s * L::TILE;
                 const uint32_t p_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
                 const uint32_t d_tmem = tmem + (i ? L::COL_O1 : L::COL_O0);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
+                for (int k = 0; k < ext / 16; ++k)
                     mma_ts(d_tmem, p_tmem + k * 8, sdesc_sw128(vb + k * 2048, 16384, 1024), IDESC_O,
                            acc | (k > 0 ? 1u : 0u));
             };
@@ -402,66 +481,75 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 }
                 if (!ok) break;
                 tc_fence_after();
-                if (un.kind == UNIT_STAGE1) {
-                    int sK, sV;
-                    if (!acquire_full(sK)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int i = 0; i < un.nq; ++i) {
-                        issue_s(i, sK);
-                        mma_commit(s_full(i));
-                    }
-                    mma_commit(kv_empty(sK));
-                    if (un.nk == 1)
-                        for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
-                    for (int j = 1; j < un.nk && ok; ++j) {
-                        if (!acquire_full(sV) || !acquire_full(sK)) { ok = false; break; }
-                        tc_fence_after();
-                        for (int i = 0; i < un.nq; ++i) {
-                            if (!wait_p_and_o(i, j == 1)) { ok = false; break; }
-                            issue_pv(i, sV, j > 1 ? 1u : 0u);
-                            issue_s(i, sK);
-                            mma_commit(s_full(i));
-                        }
-                        if (!ok) break;
-                        mma_commit(kv_empty(sV));
-                        mma_commit(kv_empty(sK));
-                        if (j == un.nk - 1)
-                            for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
-                    }
-                    if (!ok) break;
-                    if (!acquire_full(sV)) { ok = false; break; }
-                    tc_fence_after();
-                    for (int i = 0; i < un.nq; ++i) {
-                        if (!wait_p_and_o(i, un.nk == 1)) { ok = false; break; }
-                        issue_pv(i, sV, un.nk > 1 ? 1u : 0u);
-                        mma_commit(o_full(i));
-                    }
-                    if (!ok) break;
-                    mma_commit(kv_empty(sV));
-                } else {
-                    for (int i = 0; i < un.nq; ++i) {
-                        int sK;
-                        if (!acquire_full(sK)) { ok = false; break; }
-                        tc_fence_after();
-                        issue_s(i, sK);
-                        mma_commit(s_full(i));
-                        mma_commit(kv_empty(sK));
-                    }
-                    if (!ok) break;
-                    for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
-                    for (int i = 0; i < un.nq; ++i) {
-                        int sV;
-                        if (!acquire_full(sV)) { ok = false; break; }
-                        if (!wait_p_and_o(i, true)) { ok = false; break; }
-                        issue_pv(i, sV, 0u);
-                        mma_commit(o_full(i));
-                        mma_commit(kv_empty(sV));
-                    }
+                const int nkv = un.shared ? 1 : un.nq;  // K (or V) tiles per key step
+                int kvalid, ext;
+                int sK0, sK1, sV0, sV1;
+                // j = 0: S_i(0)
+                key_extent(p, un, 0, kvalid, ext);
+                if (!acquire_full(sK0)) { ok = false; break; }
+                sK1 = sK0;
+                if (nkv == 2 && !acquire_full(sK1)) { ok = false; break; }
+                tc_fence_after();
+                issue_s(0, sK0, ext);
+                mma_commit(s_full(0));
+                if (un.nq == 2) {
+                    issue_s(1, sK1, ext);
+                    mma_commit(s_full(1));
                 }
+                if (un.nk == 1)
+                    for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
+                mma_commit(kv_empty(sK0));
+                if (nkv == 2) mma_commit(kv_empty(sK1));
+                int prev_ext = ext;
+                for (int j = 1; j < un.nk && ok; ++j) {
+                    key_extent(p, un, j, kvalid, ext);
+                    if (!acquire_full(sV0)) { ok = false; break; }
+                    sV1 = sV0;
+                    if (nkv == 2 && !acquire_full(sV1)) { ok = false; break; }
+                    if (!acquire_full(sK0)) { ok = false; break; }
+                    sK1 = sK0;
+                    if (nkv == 2 && !acquire_full(sK1)) { ok = false; break; }
+                    tc_fence_after();
+                    if (!wait_p_and_o(0, j == 1)) { ok = false; break; }
+                    issue_pv(0, sV0, prev_ext, j > 1 ? 1u : 0u);
+                    issue_s(0, sK0, ext);
+                    mma_commit(s_full(0));
+                    if (un.nq == 2) {
+                        if (!wait_p_and_o(1, j == 1)) { ok = false; break; }
+                        issue_pv(1, sV1, prev_ext, j > 1 ? 1u : 0u);
+                        issue_s(1, sK1, ext);
+                        mma_commit(s_full(1));
+                    }
+                    mma_commit(kv_empty(sV0));
+                    mma_commit(kv_empty(sK0));
+                    if (nkv == 2) {
+                        mma_commit(kv_empty(sV1));
+                        mma_commit(kv_empty(sK1));
+                    }
+                    if (j == un.nk - 1)
+                        for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
+                    prev_ext = ext;
+                }
+                if (!ok) break;
+                // tail: PV_i(nk-1)
+                if (!acquire_full(sV0)) { ok = false; break; }
+                sV1 = sV0;
+                if (nkv == 2 && !acquire_full(sV1)) { ok = false; break; }
+                tc_fence_after();
+                if (!wait_p_and_o(0, un.nk == 1)) { ok = false; break; }
+                issue_pv(0, sV0, prev_ext, un.nk > 1 ? 1u : 0u);
+                mma_commit(o_full(0));
+                if (un.nq == 2) {
+                    if (!wait_p_and_o(1, un.nk == 1)) { ok = false; break; }
+                    issue_pv(1, sV1, prev_ext, un.nk > 1 ? 1u : 0u);
+                    mma_commit(o_full(1));
+                }
+                mma_commit(kv_empty(sV0));
+                if (nkv == 2) mma_commit(kv_empty(sV1));
             }
         }
     } else if (wg == 2) {
-        setmaxnreg_dec72();
+        setmaxnreg_dec64();
         // ------------------------------------------------------------ epilogue
         const int row = threadIdx.x & 127;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -475,55 +563,40 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 const float l = l_buf[i * 128 + row];
                 mbar_arrive(l_free(i));
                 const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                int bh;
+                const long long tok = lane_row_token(p, un.kind, un.ln[i], row, bh);
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) +
+                                                       (static_cast<long long>(bh) * p.N + (tok < 0 ? 0 : tok)) * D);
                 if (!mbar_wait(o_full(i), (of_par >> i) & 1u, ctl)) { ok = false; break; }
                 of_par ^= 1u << i;
                 tc_fence_after();
-                const uint32_t stg = base + L::OFF_STG + i * L::TILE;
-                // the staging buffer is free once earlier TMA stores have read it
-                if (row == 0) bulk_wait_group_read0();
-                named_barrier_sync(1, 128);
                 const uint32_t col_o = i ? L::COL_O1 : L::COL_O0;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t r[32];
                     tmem_ld32(lane_base + col_o + 32 * c, r);
                     tmem_wait_ld();
-                    // columns [32c, 32c+32) = panel c/2, 16-byte chunks (c%2)*4 + 0..3,
-                    // placed with the 128-byte swizzle the TMA store expects
-                    const uint32_t rowaddr = stg + (c >> 1) * 16384 + row * 128;
+                    if (tok >= 0) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t chunk = static_cast<uint32_t>(((c & 1) * 4 + q) ^ (row & 7));
-                        st_shared_v4(rowaddr + chunk * 16,
-                                     pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv_l,
-                                                 __uint_as_float(r[8 * q + 1]) * inv_l),
-                                     pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv_l,
-                                                 __uint_as_float(r[8 * q + 3]) * inv_l),
-                                     pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv_l,
-                                                 __uint_as_float(r[8 * q + 5]) * inv_l),
-                                     pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv_l,
-                                                 __uint_as_float(r[8 * q + 7]) * inv_l));
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv_l, __uint_as_float(r[8 * q + 1]) * inv_l);
+                            w.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv_l, __uint_as_float(r[8 * q + 3]) * inv_l);
+                            w.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv_l, __uint_as_float(r[8 * q + 5]) * inv_l);
+                            w.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv_l, __uint_as_float(r[8 * q + 7]) * inv_l);
+                            dst[4 * c + q] = w;
+                        }
                     }
                 }
                 // O_i has been read: the next unit may overwrite it
                 tc_fence_before();
                 mbar_arrive(o_free(i));
-                fence_proxy_async_smem();
-                named_barrier_sync(1, 128);
-                if (row == 0) {
-                    if (un.kind == UNIT_STAGE1)
-                        s1_store<NP>(p, &mo1, stg, un.blk, un.qt0 + i);
-                    else
-                        s2_store<NP>(&mo2, stg, p.npos, un.bh, un.chunk0 + i);
-                    bulk_commit_group();
-                }
             }
         }
-        if (row == 0) bulk_wait_group0();
     } else {
         setmaxnreg_inc192();
         // ------------------------------------------------------------ softmax
-        const int row = threadIdx.x & 127;    // TMEM lane == tile row
+        const int row = threadIdx.x & 127;  // TMEM lane == tile row
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t col_s = wg ? L::COL_S1 : L::COL_S0;
         const uint32_t col_o = wg ? L::COL_O1 : L::COL_O0;
@@ -535,14 +608,19 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             if (wg >= un.nq) continue;
             float m_run = -INFINITY;  // running max of raw logits
             float l_run = 0.f;        // running softmax denominator
-            // stage-2 mask: the row belongs to position slot prow of the chunk
+            // stage-2 mask: the row belongs to position slot prow of its chunk
             const int prow = (un.kind == UNIT_STAGE2) ? (row % p.npos) : 0;
             int npos_valid = 0;
             if (un.kind == UNIT_STAGE2) {
-                const int rem = p.HW - (un.chunk0 + wg) * p.npos;
+                const int rem = p.HW - un.ln[wg].tile * p.npos;
                 npos_valid = rem < p.npos ? rem : p.npos;
             }
             for (int j = 0; j < un.nk; ++j) {
+                int kvalid, ext;
+                key_extent(p, un, j, kvalid, ext);
+                // S is always read in full (a variable chunk count makes the
+                // compiler spill the row); columns the MMA did not write are masked
+                const bool masked = (un.kind == UNIT_STAGE2) || (kvalid < 128);
                 if (!mbar_wait(s_full(wg), sf_par, ctl)) { ok = false; break; }
                 sf_par ^= 1u;
                 tc_fence_after();
@@ -557,27 +635,34 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
 #pragma unroll
                         for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[c][e]);
                 }
-                // mask invalid key columns
-                if (un.kind == UNIT_STAGE1) {
-                    int loaded, kvalid;
-                    s1_tile_rows(p, j, loaded, kvalid);
-                    if (kvalid < 128) {
+                if (masked) {
+                    if (un.kind == UNIT_STAGE1) {
 #pragma unroll
                         for (int c = 0; c < 128; ++c)
                             if (c >= kvalid) s[c] = -INFINITY;
-                    }
-                } else {
-                    int pc = 0, tc = 0;
+                    } else {
+                        int pc = 0, tc = 0;
 #pragma unroll
-                    for (int c = 0; c < 128; ++c) {
-                        const bool valid = (pc == prow) && (tc < p.T) && (pc < npos_valid);
-                        if (!valid) s[c] = -INFINITY;
-                        if (++pc == p.npos) { pc = 0; ++tc; }
+                        for (int c = 0; c < 128; ++c) {
+                            const bool valid = (pc == prow) && (tc < p.T) && (pc < npos_valid);
+                            if (!valid) s[c] = -INFINITY;
+                            if (++pc == p.npos) { pc = 0; ++tc; }
+                        }
                     }
                 }
-                float mx = s[0];
+                float mx;
+                {
+                    float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]);
+                    float m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
 #pragma unroll
-                for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+                    for (int c = 8; c < 128; c += 8) {
+                        m0 = max3(m0, s[c], s[c + 1]);
+                        m1 = max3(m1, s[c + 2], s[c + 3]);
+                        m2 = max3(m2, s[c + 4], s[c + 5]);
+                        m3 = max3(m3, s[c + 6], s[c + 7]);
+                    }
+                    mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                }
                 // conditional rescale: keep a stale max unless it grew by > 2^8
                 bool rescale = false;
                 float alpha = 1.f;
@@ -590,25 +675,29 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     rescale = true;
                 }
                 const float moff = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-                float lsum = 0.f;
-                // P = exp2(s*scale*log2e - m*scale*log2e) as bf16 pairs, written
-                // over the first 64 columns of this tile's S region
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                uint64_t acc = pack_f32x2(0.f, 0.f);
+                // P = 2^(s*sl2 - m*sl2) as bf16 pairs over the first 64 columns
+                // of this lane's S region; masked tiles use MUFU only, so that
+                // masked columns give exact zeros
+                {
                     uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float x0 = s[32 * c + 2 * e], x1 = s[32 * c + 2 * e + 1];
-                        const float a = (x0 == -INFINITY) ? 0.f : fast_exp2(fmaf(x0, sl2, -moff));
-                        const float b = (x1 == -INFINITY) ? 0.f : fast_exp2(fmaf(x1, sl2, -moff));
-                        pk[e] = pack_bf16x2(a, b);
-                        // the denominator sums the bf16-rounded weights the PV
-                        // MMA actually uses, so a dominant weight cancels exactly
-                        lsum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
-                    }
-                    tmem_st16(lane_base + col_s + 16 * c, pk);
+#define MONARCH_CHUNK(C)                                      \
+    {                                                         \
+        if (masked)                                           \
+            softmax_chunk<false, C>(s, sl2, moff, pk, acc);   \
+        else                                                  \
+            softmax_chunk<true, C>(s, sl2, moff, pk, acc);    \
+        tmem_st16(lane_base + col_s + 16 * (C), pk);          \
+    }
+                    MONARCH_CHUNK(0)
+                    MONARCH_CHUNK(1)
+                    MONARCH_CHUNK(2)
+                    MONARCH_CHUNK(3)
+#undef MONARCH_CHUNK
                 }
-                l_run += lsum;
+                float a0, a1;
+                unpack_f32x2(acc, a0, a1);
+                l_run += a0 + a1;
                 // O from earlier key tiles is complete here (S_i(j) was issued
                 // after PV_i(j-1)); rescale it before PV_i(j) accumulates
                 if (__any_sync(0xffffffffu, rescale)) {
@@ -618,8 +707,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         tmem_ld32(lane_base + col_o + 32 * c, r);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
                         tmem_st32(lane_base + col_o + 32 * c, r);
                     }
                 }

@@ -188,6 +188,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     }
     TcParams p{};
     p.B = s.B; p.heads = s.heads; p.T = s.T; p.H = s.H; p.W = s.W; p.HW = s.H * s.W;
+    p.N = s.N;
     p.fact = s.fact;
     if (s.fact == MONARCH_FACT_TILED) {
         p.tile_h = s.tile_h; p.tile_w = s.tile_w;
@@ -204,25 +205,31 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         p.nblk_bh = s.T;
         p.nqt = (p.m + 127) / 128;
     }
-    p.s1_pairs = (p.nqt + 1) / 2;
+    const long long bh = static_cast<long long>(s.B) * s.heads;
+    if (bh * p.nblk_bh >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+    p.nblocks = static_cast<int>(bh * p.nblk_bh);
+    p.ns = p.nqt / 2;
+    p.odd = p.nqt % 2;
+    p.upg = 2 * p.ns + p.odd;
     p.npos = 128 / s.T;
     p.s2_chunks = (p.HW + p.npos - 1) / p.npos;
     p.s2_pairs = (p.s2_chunks + 1) / 2;
-    const long long bh = static_cast<long long>(s.B) * s.heads;
-    p.s1_units = bh * p.nblk_bh * p.s1_pairs;
+    // stage-1 units: groups of two blocks, each group = the shared query-tile
+    // pairs of both blocks and one unit pairing their odd last tiles
+    p.s1_units = static_cast<long long>(p.nblocks / 2) * p.upg + (p.nblocks % 2) * (p.ns + p.odd);
     p.s2_units = bh * p.s2_pairs;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.d)));
     p.timeout_cycles = env_timeout_cycles();
+    p.out = out;
     unsigned *status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_device_status) != cudaSuccess)
         return MONARCH_ERR_CUDA;
     p.status = status;
 
-    CUtensorMap mq1, mk1, mv1, mo1, mq2, mk2, my2, mo2;
+    CUtensorMap mq1, mk1, mv1, mq2, mk2, my2;
     if ((st = stage1_map(&mq1, q, s, p)) || (st = stage1_map(&mk1, k, s, p)) ||
-        (st = stage1_map(&mv1, v, s, p)) || (st = stage1_map(&mo1, out, s, p)) ||
-        (st = stage2_map(&mq2, q, s, p)) || (st = stage2_map(&mk2, k, s, p)) ||
-        (st = stage2_map(&my2, out, s, p)) || (st = stage2_map(&mo2, out, s, p)))
+        (st = stage1_map(&mv1, v, s, p)) || (st = stage2_map(&mq2, q, s, p)) ||
+        (st = stage2_map(&mk2, k, s, p)) || (st = stage2_map(&my2, out, s, p)))
         return st;
 
     // stage 1: Y1 = B1 V into out; stage 2: out = P^T B2 P Y1 in place.
@@ -234,7 +241,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         const long long units = p.unit_end - p.unit_begin;
         if (units <= 0) continue;
         const int grid = static_cast<int>(units < di->sms ? units : di->sms);
-        monarch_tc_kernel<D><<<grid, 512, L::ALLOC, stream>>>(mq1, mk1, mv1, mo1, mq2, mk2, my2, mo2, p);
+        monarch_tc_kernel<D><<<grid, 512, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
         if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
         lev.record(++lev.launches, stream);
     }
