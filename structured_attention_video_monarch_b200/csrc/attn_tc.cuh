@@ -237,30 +237,6 @@ __device__ __forceinline__ void setmaxnreg_dec64() {
 
 // ---------------------------------------------------------------- softmax math
 
-// 2^x for a pair of floats on the FMA pipe (offloads the MUFU unit).
-// Range reduction 2^x = 2^j * 2^f, j = floor(x), f in [0, 1): j comes from a
-// round-down add of 1.5*2^23 (the integer lands in the low mantissa bits, and
-// shifting those bits left by 23 puts j straight into the exponent field);
-// 2^f ~= 1 + f*(a1 + f*(a2 + f*a3)), a cubic fitted here for minimal relative
-// error with p(0) = 1, p(1) = 2 (max relative error 1.03e-4, below bf16's
-// 2^-9 rounding of P).  x is clamped to -126 so 2^j stays a normal number.
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
-    x0 = fmaxf(x0, -126.f);
-    x1 = fmaxf(x1, -126.f);
-    const uint64_t x = pack_f32x2(x0, x1);
-    const uint64_t t = add_rm_f32x2(x, pack_f32x2(12582912.f, 12582912.f));
-    const uint64_t jf = add_f32x2(t, pack_f32x2(-12582912.f, -12582912.f));
-    const uint64_t f = sub_f32x2(x, jf);
-    uint64_t q = fma_f32x2(f, pack_f32x2(0.07826797f, 0.07826797f), pack_f32x2(0.22630768f, 0.22630768f));
-    q = fma_f32x2(q, f, pack_f32x2(0.6954244f, 0.6954244f));
-    q = fma_f32x2(q, f, pack_f32x2(1.f, 1.f));
-    float q0, q1, t0, t1;
-    unpack_f32x2(q, q0, q1);
-    unpack_f32x2(t, t0, t1);
-    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -268,29 +244,24 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
-// bf16 pairs, and accumulate the rounded P into acc (two fp32 partial sums).
-// With EMULATE, 5 of the 16 pairs go through exp2_poly_pair, the rest
-// through MUFU ex2.
-template <bool EMULATE, int C>
-__device__ __forceinline__ void softmax_chunk(const float (&s)[128], float sl2, float moff,
-                                              uint32_t (&pk)[16], uint64_t &acc) {
-    const uint64_t scale = pack_f32x2(sl2, sl2);
-    const uint64_t off = pack_f32x2(-moff, -moff);
+// bf16 pairs, and accumulate the rounded P into two packed fp32 partial sums
+// (even and odd pairs, so the additions form two independent chains).
+template <int C>
+__device__ __forceinline__ void softmax_chunk(const float (&s)[128], uint64_t scale, uint64_t off,
+                                              uint32_t (&pk)[16], uint64_t &acc0, uint64_t &acc1) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const uint64_t x = fma_f32x2(pack_f32x2(s[32 * C + 2 * e], s[32 * C + 2 * e + 1]), scale, off);
-        float x0, x1, a, b;
+        float x0, x1;
         unpack_f32x2(x, x0, x1);
-        if (EMULATE && (e % 3 == 1)) {
-            exp2_poly_pair(x0, x1, a, b);
-        } else {
-            a = fast_exp2(x0);
-            b = fast_exp2(x1);
-        }
-        const uint32_t w = pack_bf16x2(a, b);
+        const uint32_t w = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
         pk[e] = w;
         // the denominator sums the bf16-rounded weights the PV MMA uses
-        acc = add_f32x2(acc, pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
+        const uint64_t r = pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        if (e & 1)
+            acc1 = add_f32x2(acc1, r);
+        else
+            acc0 = add_f32x2(acc0, r);
     }
 }
 
@@ -437,31 +408,44 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 if (++slot == NS) { slot = 0; ++kv_round; }
                 return r;
             };
+            // Descriptor halves: the low word holds the start address, so
+            // every K step below is a single 32-bit add of a constant.
+            constexpr uint32_t KM_HI = sdesc_sw128_hi(1024);  // K-major: 8-row groups 1024 B apart
+            constexpr uint32_t MN_HI = sdesc_sw128_hi(1024);  // MN-major V: 8-key groups 1024 B apart
+            const uint32_t q_lo0 = sdesc_sw128_lo(base + L::OFF_Q, 16);
+            const uint32_t kv_lo0 = sdesc_sw128_lo(base + L::OFF_KV, 16);
+            const uint32_t v_lo0 = sdesc_sw128_lo(base + L::OFF_KV, 16384);  // D panels 16 KB apart
+            constexpr uint32_t TILE16 = L::TILE >> 4;
+            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
             // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D,
-            // N = ext key columns.
-            auto issue_s = [&](int i, int s, int ext) {
-                const uint32_t qa = base + L::OFF_Q + i * L::TILE;
-                const uint32_t kb = base + L::OFF_KV + s * L::TILE;
+            // N = ext key columns (idesc_s).
+            auto issue_s = [&](int i, int s, uint32_t idesc_s) {
+                const uint32_t a = q_lo0 + i * TILE16;
+                const uint32_t b = kv_lo0 + s * TILE16;
                 const uint32_t d_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
-                const uint32_t idesc = idesc_bf16_f32(128, ext, false, false);
+                mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, idesc_s);
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                    mma_ss(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc,
-                           k > 0 ? 1u : 0u);
+                for (int k = 1; k < D / 16; ++k) {
+                    const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                    mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, idesc_s);
                 }
             };
             // O_i (+)= P_i V: A = P from TMEM (bf16 pairs in the S region),
             // B = V tile (MN-major: keys x D, D contiguous), K dim = ext keys.
             auto issue_pv = [&](int i, int s, int ext, uint32_t acc) {
-                constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-                const uint32_t vb = base + L::OFF_KV + s * L::TILE;
+                const uint32_t b = v_lo0 + s * TILE16;
                 const uint32_t p_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
                 const uint32_t d_tmem = tmem + (i ? L::COL_O1 : L::COL_O0);
-                for (int k = 0; k < ext / 16; ++k)
-                    mma_ts(d_tmem, p_tmem + k * 8, sdesc_sw128(vb + k * 2048, 16384, 1024), IDESC_O,
-                           acc | (k > 0 ? 1u : 0u));
+                mma_ts_lh(d_tmem, p_tmem, b, MN_HI, IDESC_O, acc);
+                if (ext == 128) {
+#pragma unroll
+                    for (int k = 1; k < 8; ++k) mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
+                } else {
+                    for (int k = 1; k < ext / 16; ++k)
+                        mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
+                }
             };
+            auto idesc_for = [](int ext) { return idesc_bf16_f32(128, ext, false, false); };
             // the first PV of a unit overwrites O_i: the epilogue must be done with it
             auto wait_p_and_o = [&](int i, bool first) -> bool {
                 if (first) {
@@ -490,10 +474,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 sK1 = sK0;
                 if (nkv == 2 && !acquire_full(sK1)) { ok = false; break; }
                 tc_fence_after();
-                issue_s(0, sK0, ext);
+                issue_s(0, sK0, idesc_for(ext));
                 mma_commit(s_full(0));
                 if (un.nq == 2) {
-                    issue_s(1, sK1, ext);
+                    issue_s(1, sK1, idesc_for(ext));
                     mma_commit(s_full(1));
                 }
                 if (un.nk == 1)
@@ -511,13 +495,14 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     if (nkv == 2 && !acquire_full(sK1)) { ok = false; break; }
                     tc_fence_after();
                     if (!wait_p_and_o(0, j == 1)) { ok = false; break; }
+                    const uint32_t idesc_s = idesc_for(ext);
                     issue_pv(0, sV0, prev_ext, j > 1 ? 1u : 0u);
-                    issue_s(0, sK0, ext);
+                    issue_s(0, sK0, idesc_s);
                     mma_commit(s_full(0));
                     if (un.nq == 2) {
                         if (!wait_p_and_o(1, j == 1)) { ok = false; break; }
                         issue_pv(1, sV1, prev_ext, j > 1 ? 1u : 0u);
-                        issue_s(1, sK1, ext);
+                        issue_s(1, sK1, idesc_s);
                         mma_commit(s_full(1));
                     }
                     mma_commit(kv_empty(sV0));
@@ -675,29 +660,28 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     rescale = true;
                 }
                 const float moff = (m_run == -INFINITY) ? 0.f : m_run * sl2;
-                uint64_t acc = pack_f32x2(0.f, 0.f);
+                uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
+                const uint64_t scale2 = pack_f32x2(sl2, sl2);
+                const uint64_t off2 = pack_f32x2(-moff, -moff);
                 // P = 2^(s*sl2 - m*sl2) as bf16 pairs over the first 64 columns
-                // of this lane's S region; masked tiles use MUFU only, so that
-                // masked columns give exact zeros
+                // of this lane's S region (masked columns: 2^-inf = exact 0)
                 {
                     uint32_t pk[16];
-#define MONARCH_CHUNK(C)                                      \
-    {                                                         \
-        if (masked)                                           \
-            softmax_chunk<false, C>(s, sl2, moff, pk, acc);   \
-        else                                                  \
-            softmax_chunk<true, C>(s, sl2, moff, pk, acc);    \
-        tmem_st16(lane_base + col_s + 16 * (C), pk);          \
-    }
-                    MONARCH_CHUNK(0)
-                    MONARCH_CHUNK(1)
-                    MONARCH_CHUNK(2)
-                    MONARCH_CHUNK(3)
-#undef MONARCH_CHUNK
+                    softmax_chunk<0>(s, scale2, off2, pk, acc0, acc1);
+                    tmem_st16(lane_base + col_s + 0, pk);
+                    softmax_chunk<1>(s, scale2, off2, pk, acc0, acc1);
+                    tmem_st16(lane_base + col_s + 16, pk);
+                    softmax_chunk<2>(s, scale2, off2, pk, acc0, acc1);
+                    tmem_st16(lane_base + col_s + 32, pk);
+                    softmax_chunk<3>(s, scale2, off2, pk, acc0, acc1);
+                    tmem_st16(lane_base + col_s + 48, pk);
                 }
-                float a0, a1;
-                unpack_f32x2(acc, a0, a1);
-                l_run += a0 + a1;
+                {
+                    float a0, a1, b0, b1;
+                    unpack_f32x2(acc0, a0, a1);
+                    unpack_f32x2(acc1, b0, b1);
+                    l_run += (a0 + a1) + (b0 + b1);
+                }
                 // O from earlier key tiles is complete here (S_i(j) was issued
                 // after PV_i(j-1)); rescale it before PV_i(j) accumulates
                 if (__any_sync(0xffffffffu, rescale)) {
