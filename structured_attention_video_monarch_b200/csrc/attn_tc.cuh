@@ -22,14 +22,18 @@
 // own keys ("separate" units: the odd last query tile of two blocks, and
 // every stage-2 unit).
 //
-// Warp roles (512 threads, registers rebalanced with setmaxnreg):
-//   warps 0-3   softmax for lane 0 (thread = row)                  192 regs
-//   warps 4-7   softmax for lane 1                                  192 regs
-//   warps 8-11  epilogue: O / l -> bf16 -> global stores             64 regs
-//   warp  12    TMA producer (Q tiles, K/V ring)                     64 regs
-//   warp  13    TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 14-15 idle
-// (2*128*192 + 128*64 + 128*64 = 65536, the registers the block launches with.)
+// Warp roles (640 threads, registers rebalanced with setmaxnreg):
+//   warps 0-3, 8-11    lane 0: softmax over S columns 0-63 / 64-127 of each
+//                      row (thread = row), then O/l -> bf16 -> global for
+//                      output columns [0, D/2) / [D/2, D)            104 regs
+//   warps 4-7, 12-15   the same for lane 1                            104 regs
+//   warp  16           TMA producer (Q tiles, K/V ring)                64 regs
+//   warp  17           TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 18-19        idle
+// (4*128*104 + 128*64 = 61440 = 640 threads x 96, the launch allocation.)
+// Splitting each row over two warps puts two warps of the same lane on every
+// SM sub-partition, so the exp/pack work of one tile is spread over twice the
+// warps; the halves exchange their row maxima through shared memory.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0, O1 after them.
 // P (bf16) overwrites the first 64 columns of its S region and feeds the PV
 // MMA straight from TMEM.  The MMA issue order per key tile j is
@@ -207,10 +211,14 @@ struct TcLayout {
     static constexpr int OFF_KV = OFF_Q + 2 * TILE;
     static constexpr int OFF_BAR = OFF_KV + NS * TILE;
     // barriers: q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2]
-    //           o_full[2] o_free[2] l_full[2] l_free[2]
-    static constexpr int NBAR = 16 + 2 * NS;
-    static constexpr int OFF_L = OFF_BAR + NBAR * 8;     // row sums l, [2 lanes][128 rows] fp32
-    static constexpr int OFF_MISC = OFF_L + 2 * 128 * 4; // tmem base, abort flag
+    //           o_full[2] o_free[2]
+    static constexpr int NBAR = 12 + 2 * NS;
+    // row-max exchange between the two column halves of a lane:
+    // [2 parities][2 lanes][2 halves][128 rows] fp32
+    static constexpr int OFF_MX = OFF_BAR + NBAR * 8;
+    // row-sum exchange at the end of a unit: [2 lanes][2 halves][128 rows] fp32
+    static constexpr int OFF_L = OFF_MX + 2 * 2 * 2 * 128 * 4;
+    static constexpr int OFF_MISC = OFF_L + 2 * 2 * 128 * 4;  // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     static constexpr int ALLOC = BYTES + 1024;        // slack to align the base to 1024
     static constexpr uint32_t TMEM_COLS = 512;
@@ -228,8 +236,8 @@ __device__ __forceinline__ void zero_rows(uint32_t tile, int from, int to) {
             for (int c = 0; c < 8; ++c) st_shared_v4(tile + pn * 16384 + r * 128 + c * 16, 0, 0, 0, 0);
 }
 
-__device__ __forceinline__ void setmaxnreg_inc192() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;" ::: "memory");
+__device__ __forceinline__ void setmaxnreg_inc104() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
 }
 __device__ __forceinline__ void setmaxnreg_dec64() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
@@ -247,7 +255,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // bf16 pairs, and accumulate the rounded P into two packed fp32 partial sums
 // (even and odd pairs, so the additions form two independent chains).
 template <int C>
-__device__ __forceinline__ void softmax_chunk(const float (&s)[128], uint64_t scale, uint64_t off,
+__device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t scale, uint64_t off,
                                               uint32_t (&pk)[16], uint64_t &acc0, uint64_t &acc1) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -266,7 +274,7 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[128], uint64_t sc
 }
 
 template <int D>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(640, 1)
 monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant__ CUtensorMap mk1,
                   const __grid_constant__ CUtensorMap mv1, const __grid_constant__ CUtensorMap mq2,
                   const __grid_constant__ CUtensorMap mk2, const __grid_constant__ CUtensorMap my2,
@@ -288,8 +296,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     auto p_full = [&](int i) { return bar0 + 8u * (6 + 2 * NS + i); };
     auto o_full = [&](int i) { return bar0 + 8u * (8 + 2 * NS + i); };
     auto o_free = [&](int i) { return bar0 + 8u * (10 + 2 * NS + i); };
-    auto l_full = [&](int i) { return bar0 + 8u * (12 + 2 * NS + i); };
-    auto l_free = [&](int i) { return bar0 + 8u * (14 + 2 * NS + i); };
+    float *mx_buf = reinterpret_cast<float *>(base_ptr + L::OFF_MX);
     float *l_buf = reinterpret_cast<float *>(base_ptr + L::OFF_L);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
@@ -305,11 +312,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             mbar_init(q_full(i), 1);
             mbar_init(q_empty(i), 1);
             mbar_init(s_full(i), 1);
-            mbar_init(p_full(i), 128);
+            mbar_init(p_full(i), 256);
             mbar_init(o_full(i), 1);
-            mbar_init(o_free(i), 128);
-            mbar_init(l_full(i), 128);
-            mbar_init(l_free(i), 128);
+            mbar_init(o_free(i), 256);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full(s), 1);
@@ -317,11 +322,11 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         }
         fence_barrier_init();
     }
-    if (warp == 12 && lane == 0) {
+    if (warp == 16 && lane == 0) {
         tma_prefetch_desc(&mq1); tma_prefetch_desc(&mk1); tma_prefetch_desc(&mv1);
         tma_prefetch_desc(&mq2); tma_prefetch_desc(&mk2); tma_prefetch_desc(&my2);
     }
-    if (warp == 13) {
+    if (warp == 17) {
         tmem_alloc(smem_addr(tmem_slot), L::TMEM_COLS);
         tmem_relinquish();
     }
@@ -330,9 +335,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (wg == 3) {
+    if (wg == 4) {
         setmaxnreg_dec64();
-        if (warp == 12 && lane == 0) {
+        if (warp == 16 && lane == 0) {
             // -------------------------------------------------------- TMA producer
             uint32_t qe_par = 3u;  // bit i: parity to wait for on q_empty(i)
             int slot = 0;
@@ -394,7 +399,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     }
                 }
             }
-        } else if (warp == 13 && lane == 0) {
+        } else if (warp == 17 && lane == 0) {
             // -------------------------------------------------------- MMA issuer
             uint32_t qf_par = 0u;  // bit i: parity to wait for on q_full(i)
             uint32_t pf_par = 0u;  // bit i: parity to wait for on p_full(i)
@@ -533,102 +538,58 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 if (nkv == 2) mma_commit(kv_empty(sV1));
             }
         }
-    } else if (wg == 2) {
-        setmaxnreg_dec64();
-        // ------------------------------------------------------------ epilogue
-        const int row = threadIdx.x & 127;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        uint32_t lf_par = 0u, of_par = 0u;  // bit i: parity for l_full(i) / o_full(i)
-        bool ok = true;
-        for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
-            const Unit un = decode_unit(p, u);
-            for (int i = 0; i < un.nq; ++i) {
-                if (!mbar_wait(l_full(i), (lf_par >> i) & 1u, ctl)) { ok = false; break; }
-                lf_par ^= 1u << i;
-                const float l = l_buf[i * 128 + row];
-                mbar_arrive(l_free(i));
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                int bh;
-                const long long tok = lane_row_token(p, un.kind, un.ln[i], row, bh);
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) +
-                                                       (static_cast<long long>(bh) * p.N + (tok < 0 ? 0 : tok)) * D);
-                if (!mbar_wait(o_full(i), (of_par >> i) & 1u, ctl)) { ok = false; break; }
-                of_par ^= 1u << i;
-                tc_fence_after();
-                const uint32_t col_o = i ? L::COL_O1 : L::COL_O0;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(lane_base + col_o + 32 * c, r);
-                    tmem_wait_ld();
-                    if (tok >= 0) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv_l, __uint_as_float(r[8 * q + 1]) * inv_l);
-                            w.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv_l, __uint_as_float(r[8 * q + 3]) * inv_l);
-                            w.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv_l, __uint_as_float(r[8 * q + 5]) * inv_l);
-                            w.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv_l, __uint_as_float(r[8 * q + 7]) * inv_l);
-                            dst[4 * c + q] = w;
-                        }
-                    }
-                }
-                // O_i has been read: the next unit may overwrite it
-                tc_fence_before();
-                mbar_arrive(o_free(i));
-            }
-        }
     } else {
-        setmaxnreg_inc192();
-        // ------------------------------------------------------------ softmax
+        setmaxnreg_inc104();
+        // ------------------------------------------------------------ softmax + epilogue
+        // warpgroup wg: lane li = wg & 1 (query tile of the unit), column
+        // half h = wg >> 1 (S columns [64h, 64h+64), O columns [h*D/2, (h+1)*D/2))
+        const int li = wg & 1, h = wg >> 1;
         const int row = threadIdx.x & 127;  // TMEM lane == tile row
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        const uint32_t col_s = wg ? L::COL_S1 : L::COL_S0;
-        const uint32_t col_o = wg ? L::COL_O1 : L::COL_O0;
+        const uint32_t col_s = li ? L::COL_S1 : L::COL_S0;
+        const uint32_t col_o = li ? L::COL_O1 : L::COL_O0;
         const float sl2 = p.scale_log2;
-        uint32_t sf_par = 0u, lfree_par = 1u;
+        uint32_t sf_par = 0u, of_par = 0u, mx_par = 0u;
         bool ok = true;
         for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u);
-            if (wg >= un.nq) continue;
-            float m_run = -INFINITY;  // running max of raw logits
-            float l_run = 0.f;        // running softmax denominator
+            if (li >= un.nq) continue;
+            float m_run = -INFINITY;  // running max of raw logits (whole row)
+            float l_half = 0.f;       // softmax denominator over this half's columns
             // stage-2 mask: the row belongs to position slot prow of its chunk
             const int prow = (un.kind == UNIT_STAGE2) ? (row % p.npos) : 0;
             int npos_valid = 0;
             if (un.kind == UNIT_STAGE2) {
-                const int rem = p.HW - un.ln[wg].tile * p.npos;
+                const int rem = p.HW - un.ln[li].tile * p.npos;
                 npos_valid = rem < p.npos ? rem : p.npos;
             }
             for (int j = 0; j < un.nk; ++j) {
                 int kvalid, ext;
                 key_extent(p, un, j, kvalid, ext);
-                // S is always read in full (a variable chunk count makes the
-                // compiler spill the row); columns the MMA did not write are masked
                 const bool masked = (un.kind == UNIT_STAGE2) || (kvalid < 128);
-                if (!mbar_wait(s_full(wg), sf_par, ctl)) { ok = false; break; }
+                if (!mbar_wait(s_full(li), sf_par, ctl)) { ok = false; break; }
                 sf_par ^= 1u;
                 tc_fence_after();
-                float s[128];
+                float s[64];
                 {
-                    uint32_t r[4][32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + col_s + 32 * c, r[c]);
+                    uint32_t r[2][32];
+                    tmem_ld32(lane_base + col_s + 64 * h, r[0]);
+                    tmem_ld32(lane_base + col_s + 64 * h + 32, r[1]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[c][e]);
                 }
-                if (masked) {
+                if (masked) {  // columns 64h + c
                     if (un.kind == UNIT_STAGE1) {
 #pragma unroll
-                        for (int c = 0; c < 128; ++c)
-                            if (c >= kvalid) s[c] = -INFINITY;
+                        for (int c = 0; c < 64; ++c)
+                            if (64 * h + c >= kvalid) s[c] = -INFINITY;
                     } else {
-                        int pc = 0, tc = 0;
+                        int pc = (64 * h) % p.npos, tc = (64 * h) / p.npos;
 #pragma unroll
-                        for (int c = 0; c < 128; ++c) {
+                        for (int c = 0; c < 64; ++c) {
                             const bool valid = (pc == prow) && (tc < p.T) && (pc < npos_valid);
                             if (!valid) s[c] = -INFINITY;
                             if (++pc == p.npos) { pc = 0; ++tc; }
@@ -640,7 +601,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     float m0 = fmaxf(s[0], s[1]), m1 = fmaxf(s[2], s[3]);
                     float m2 = fmaxf(s[4], s[5]), m3 = fmaxf(s[6], s[7]);
 #pragma unroll
-                    for (int c = 8; c < 128; c += 8) {
+                    for (int c = 8; c < 64; c += 8) {
                         m0 = max3(m0, s[c], s[c + 1]);
                         m1 = max3(m1, s[c + 2], s[c + 3]);
                         m2 = max3(m2, s[c + 4], s[c + 5]);
@@ -648,7 +609,16 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     }
                     mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
                 }
+                // row max over both halves (double-buffered by tile parity)
+                {
+                    float *xb = mx_buf + ((mx_par * 2 + li) * 2) * 128;
+                    xb[h * 128 + row] = mx;
+                    named_barrier_sync(1 + li, 256);
+                    mx = fmaxf(mx, xb[(1 - h) * 128 + row]);
+                    mx_par ^= 1u;
+                }
                 // conditional rescale: keep a stale max unless it grew by > 2^8
+                // (both halves see the same mx and m_run, so they agree)
                 bool rescale = false;
                 float alpha = 1.f;
                 if (j == 0) {
@@ -656,56 +626,82 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 } else if ((mx - m_run) * sl2 > 8.f) {
                     alpha = fast_exp2((m_run - mx) * sl2);
                     m_run = mx;
-                    l_run *= alpha;
+                    l_half *= alpha;
                     rescale = true;
                 }
                 const float moff = (m_run == -INFINITY) ? 0.f : m_run * sl2;
                 uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
                 const uint64_t scale2 = pack_f32x2(sl2, sl2);
                 const uint64_t off2 = pack_f32x2(-moff, -moff);
-                // P = 2^(s*sl2 - m*sl2) as bf16 pairs over the first 64 columns
-                // of this lane's S region (masked columns: 2^-inf = exact 0)
+                // P = 2^(s*sl2 - m*sl2) as bf16 pairs: this half's 64 keys go to
+                // packed columns [32h, 32h+32) of the lane's S region
                 {
                     uint32_t pk[16];
                     softmax_chunk<0>(s, scale2, off2, pk, acc0, acc1);
-                    tmem_st16(lane_base + col_s + 0, pk);
+                    tmem_st16(lane_base + col_s + 32 * h, pk);
                     softmax_chunk<1>(s, scale2, off2, pk, acc0, acc1);
-                    tmem_st16(lane_base + col_s + 16, pk);
-                    softmax_chunk<2>(s, scale2, off2, pk, acc0, acc1);
-                    tmem_st16(lane_base + col_s + 32, pk);
-                    softmax_chunk<3>(s, scale2, off2, pk, acc0, acc1);
-                    tmem_st16(lane_base + col_s + 48, pk);
+                    tmem_st16(lane_base + col_s + 32 * h + 16, pk);
                 }
                 {
                     float a0, a1, b0, b1;
                     unpack_f32x2(acc0, a0, a1);
                     unpack_f32x2(acc1, b0, b1);
-                    l_run += (a0 + a1) + (b0 + b1);
+                    l_half += (a0 + a1) + (b0 + b1);
                 }
                 // O from earlier key tiles is complete here (S_i(j) was issued
-                // after PV_i(j-1)); rescale it before PV_i(j) accumulates
+                // after PV_i(j-1)); rescale this half's columns before PV_i(j)
                 if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = 0; c < D / 64; ++c) {
                         uint32_t r[32];
-                        tmem_ld32(lane_base + col_o + 32 * c, r);
+                        const uint32_t a = lane_base + col_o + h * (D / 2) + 32 * c;
+                        tmem_ld32(a, r);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        tmem_st32(lane_base + col_o + 32 * c, r);
+                        tmem_st32(a, r);
                     }
                 }
                 tmem_wait_st();
-                if (j == un.nk - 1) {
-                    // hand the row sum to the epilogue (one-slot handshake)
-                    if (!mbar_wait(l_free(wg), lfree_par, ctl)) { ok = false; break; }
-                    lfree_par ^= 1u;
-                    l_buf[wg * 128 + row] = l_run;
-                    mbar_arrive(l_full(wg));
-                }
                 tc_fence_before();
-                mbar_arrive(p_full(wg));
+                mbar_arrive(p_full(li));
             }
+            if (!ok) break;
+            // ---------------------------------------------------- epilogue
+            // row sum over both halves, then O / l for this half's columns
+            float *lb = l_buf + li * 2 * 128;
+            lb[h * 128 + row] = l_half;
+            named_barrier_sync(1 + li, 256);
+            const float l = l_half + lb[(1 - h) * 128 + row];
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            int bh;
+            const long long tok = lane_row_token(p, un.kind, un.ln[li], row, bh);
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) +
+                                                   (static_cast<long long>(bh) * p.N + (tok < 0 ? 0 : tok)) * D +
+                                                   h * (D / 2));
+            if (!mbar_wait(o_full(li), of_par, ctl)) { ok = false; break; }
+            of_par ^= 1u;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + col_o + h * (D / 2) + 32 * c, r);
+                tmem_wait_ld();
+                if (tok >= 0) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv_l, __uint_as_float(r[8 * q + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv_l, __uint_as_float(r[8 * q + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv_l, __uint_as_float(r[8 * q + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv_l, __uint_as_float(r[8 * q + 7]) * inv_l);
+                        dst[4 * c + q] = w;
+                    }
+                }
+            }
+            // O_i has been read: the next unit may overwrite it
+            tc_fence_before();
+            mbar_arrive(o_free(li));
         }
     }
 
@@ -718,7 +714,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         while (clock64() - t0 < (1ll << 24)) {
         }
     }
-    if (warp == 13) {
+    if (warp == 17) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);

@@ -241,7 +241,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         const long long units = p.unit_end - p.unit_begin;
         if (units <= 0) continue;
         const int grid = static_cast<int>(units < di->sms ? units : di->sms);
-        monarch_tc_kernel<D><<<grid, 512, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
+        monarch_tc_kernel<D><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
         if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
         lev.record(++lev.launches, stream);
     }
