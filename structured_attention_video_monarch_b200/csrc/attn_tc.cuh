@@ -213,14 +213,16 @@ struct TcLayout {
     // barriers: q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2]
     //           o_full[2] o_free[2]
     static constexpr int NBAR = 12 + 2 * NS;
-    // row-max exchange between the two column halves of a lane:
-    // [2 parities][2 lanes][2 halves][128 rows] fp32
-    static constexpr int OFF_MX = OFF_BAR + NBAR * 8;
-    // row-sum exchange at the end of a unit: [2 lanes][2 halves][128 rows] fp32
-    static constexpr int OFF_L = OFF_MX + 2 * 2 * 2 * 128 * 4;
-    static constexpr int OFF_MISC = OFF_L + 2 * 2 * 128 * 4;  // tmem base, abort flag
+    // exchange of per-row values (partial maxima, partial sums) between the two
+    // column halves of a lane: [2 lanes][2 halves][128 rows] fp32
+    static constexpr int OFF_X = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_MISC = OFF_X + 2 * 2 * 128 * 4;  // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
-    static constexpr int ALLOC = BYTES + 1024;        // slack to align the base to 1024
+    // The dynamic shared-memory base is at least 256-byte aligned; up to 768
+    // bytes of slack realign it to the 1024 bytes the 128-byte swizzle needs.
+    static constexpr int SLACK = 768;
+    static constexpr int ALLOC = BYTES + SLACK;
+    static_assert(ALLOC <= 232448, "exceeds the 227 KB of shared memory a block may use");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
 };
@@ -286,6 +288,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (base - raw);
+    if (base - raw > static_cast<uint32_t>(L::SLACK)) {  // uniform over the block
+        if (threadIdx.x == 0) atomicOr(p.status, DEVERR_ALIGN);
+        return;
+    }
 
     const uint32_t bar0 = base + L::OFF_BAR;
     auto q_full = [&](int i) { return bar0 + 8u * i; };
@@ -296,8 +302,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     auto p_full = [&](int i) { return bar0 + 8u * (6 + 2 * NS + i); };
     auto o_full = [&](int i) { return bar0 + 8u * (8 + 2 * NS + i); };
     auto o_free = [&](int i) { return bar0 + 8u * (10 + 2 * NS + i); };
-    float *mx_buf = reinterpret_cast<float *>(base_ptr + L::OFF_MX);
-    float *l_buf = reinterpret_cast<float *>(base_ptr + L::OFF_L);
+    float *x_buf = reinterpret_cast<float *>(base_ptr + L::OFF_X);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
 
@@ -549,8 +554,18 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         const uint32_t col_s = li ? L::COL_S1 : L::COL_S0;
         const uint32_t col_o = li ? L::COL_O1 : L::COL_O0;
         const float sl2 = p.scale_log2;
-        uint32_t sf_par = 0u, of_par = 0u, mx_par = 0u;
+        uint32_t sf_par = 0u, of_par = 0u;
         bool ok = true;
+        // value of this row in the other column half of the lane: barrier
+        // 3+li makes sure the other half has read the previous value before
+        // it is overwritten, barrier 1+li publishes the new one
+        float *xb = x_buf + li * 2 * 128;
+        auto exchange = [&](float v) -> float {
+            named_barrier_sync(3 + li, 256);
+            xb[h * 128 + row] = v;
+            named_barrier_sync(1 + li, 256);
+            return xb[(1 - h) * 128 + row];
+        };
         for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u);
             if (li >= un.nq) continue;
@@ -609,14 +624,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     }
                     mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
                 }
-                // row max over both halves (double-buffered by tile parity)
-                {
-                    float *xb = mx_buf + ((mx_par * 2 + li) * 2) * 128;
-                    xb[h * 128 + row] = mx;
-                    named_barrier_sync(1 + li, 256);
-                    mx = fmaxf(mx, xb[(1 - h) * 128 + row]);
-                    mx_par ^= 1u;
-                }
+                mx = fmaxf(mx, exchange(mx));  // row max over both halves
                 // conditional rescale: keep a stale max unless it grew by > 2^8
                 // (both halves see the same mx and m_run, so they agree)
                 bool rescale = false;
@@ -669,10 +677,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             if (!ok) break;
             // ---------------------------------------------------- epilogue
             // row sum over both halves, then O / l for this half's columns
-            float *lb = l_buf + li * 2 * 128;
-            lb[h * 128 + row] = l_half;
-            named_barrier_sync(1 + li, 256);
-            const float l = l_half + lb[(1 - h) * 128 + row];
+            const float l = l_half + exchange(l_half);
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             int bh;
             const long long tok = lane_row_token(p, un.kind, un.ln[li], row, bh);

@@ -320,7 +320,9 @@ int read_status(cudaStream_t stream, int reset) {
         if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
             return MONARCH_ERR_CUDA;
     }
-    return (v & DEVERR_TIMEOUT) ? MONARCH_ERR_TIMEOUT : MONARCH_OK;
+    if (v & DEVERR_TIMEOUT) return MONARCH_ERR_TIMEOUT;
+    if (v & DEVERR_ALIGN) return MONARCH_ERR_LAUNCH;
+    return MONARCH_OK;
 }
 
 }  // namespace

@@ -47,6 +47,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Device status bits (written with atomicOr into the library's status word).
 enum : unsigned {
     DEVERR_TIMEOUT = 1u,
+    DEVERR_ALIGN = 2u,  // dynamic shared memory base not aligned as the kernel assumes
 };
 
 // Shared state for bounded waiting.  `abort_flag` lives in shared memory:
