@@ -247,6 +247,28 @@ __device__ __forceinline__ void setmaxnreg_dec64() {
 
 // ---------------------------------------------------------------- softmax math
 
+// 2^x for a pair of floats on the FMA pipe (offloads the MUFU unit).
+// Range reduction 2^x = 2^j * 2^f, j = floor(x), f in [0, 1): j comes from a
+// round-down add of 1.5*2^23 (the integer lands in the low mantissa bits, and
+// shifting those bits left by 23 puts j straight into the exponent field);
+// 2^f ~= 1 + f*(a1 + f*(a2 + f*a3)), a cubic fitted here for minimal relative
+// error with p(0) = 1, p(1) = 2 (max relative error 1.03e-4, below bf16's
+// 2^-9 rounding of P).  x is clamped to -126 so 2^j stays a normal number;
+// callers only pass finite x (masked tiles use the MUFU path).
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
+    const uint64_t x = pack_f32x2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t t = add_rm_f32x2(x, pack_f32x2(12582912.f, 12582912.f));
+    const uint64_t f = sub_f32x2(x, add_f32x2(t, pack_f32x2(-12582912.f, -12582912.f)));
+    uint64_t q = fma_f32x2(f, pack_f32x2(0.07826797f, 0.07826797f), pack_f32x2(0.22630768f, 0.22630768f));
+    q = fma_f32x2(q, f, pack_f32x2(0.6954244f, 0.6954244f));
+    q = fma_f32x2(q, f, pack_f32x2(1.f, 1.f));
+    float q0, q1, t0, t1;
+    unpack_f32x2(q, q0, q1);
+    unpack_f32x2(t, t0, t1);
+    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -255,16 +277,24 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 // Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
 // bf16 pairs, and accumulate the rounded P into two packed fp32 partial sums
-// (even and odd pairs, so the additions form two independent chains).
-template <int C>
+// (even and odd pairs, so the additions form two independent chains).  With
+// EMULATE, 6 of the 16 pairs take exp2_poly_pair on the FMA pipe and the rest
+// MUFU ex2, balancing the two units.
+template <bool EMULATE, int C>
 __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t scale, uint64_t off,
                                               uint32_t (&pk)[16], uint64_t &acc0, uint64_t &acc1) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const uint64_t x = fma_f32x2(pack_f32x2(s[32 * C + 2 * e], s[32 * C + 2 * e + 1]), scale, off);
-        float x0, x1;
+        float x0, x1, a, b;
         unpack_f32x2(x, x0, x1);
-        const uint32_t w = pack_bf16x2(fast_exp2(x0), fast_exp2(x1));
+        if (EMULATE && (e % 8 == 1 || e % 8 == 4 || e % 8 == 6)) {
+            exp2_poly_pair(x0, x1, a, b);
+        } else {
+            a = fast_exp2(x0);
+            b = fast_exp2(x1);
+        }
+        const uint32_t w = pack_bf16x2(a, b);
         pk[e] = w;
         // the denominator sums the bf16-rounded weights the PV MMA uses
         const uint64_t r = pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
@@ -624,18 +654,22 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     }
                     mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
                 }
-                mx = fmaxf(mx, exchange(mx));  // row max over both halves
-                // conditional rescale: keep a stale max unless it grew by > 2^8
-                // (both halves see the same mx and m_run, so they agree)
+                // The row max spans both halves.  Tile 0 exchanges it; later
+                // tiles keep the running max unless some row of the lane grew
+                // by more than 2^8 (one OR-barrier tells), and only then
+                // exchange partial maxima and rescale O.
                 bool rescale = false;
                 float alpha = 1.f;
                 if (j == 0) {
-                    m_run = mx;
-                } else if ((mx - m_run) * sl2 > 8.f) {
-                    alpha = fast_exp2((m_run - mx) * sl2);
-                    m_run = mx;
-                    l_half *= alpha;
-                    rescale = true;
+                    m_run = fmaxf(mx, exchange(mx));
+                } else if (named_barrier_or(5 + li, 256, (mx - m_run) * sl2 > 8.f)) {
+                    mx = fmaxf(mx, exchange(mx));
+                    if ((mx - m_run) * sl2 > 8.f) {
+                        alpha = fast_exp2((m_run - mx) * sl2);
+                        m_run = mx;
+                        l_half *= alpha;
+                        rescale = true;
+                    }
                 }
                 const float moff = (m_run == -INFINITY) ? 0.f : m_run * sl2;
                 uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
@@ -645,10 +679,17 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 // packed columns [32h, 32h+32) of the lane's S region
                 {
                     uint32_t pk[16];
-                    softmax_chunk<0>(s, scale2, off2, pk, acc0, acc1);
-                    tmem_st16(lane_base + col_s + 32 * h, pk);
-                    softmax_chunk<1>(s, scale2, off2, pk, acc0, acc1);
-                    tmem_st16(lane_base + col_s + 32 * h + 16, pk);
+                    if (masked) {  // masked columns need MUFU's exact 2^-inf = 0
+                        softmax_chunk<false, 0>(s, scale2, off2, pk, acc0, acc1);
+                        tmem_st16(lane_base + col_s + 32 * h, pk);
+                        softmax_chunk<false, 1>(s, scale2, off2, pk, acc0, acc1);
+                        tmem_st16(lane_base + col_s + 32 * h + 16, pk);
+                    } else {
+                        softmax_chunk<true, 0>(s, scale2, off2, pk, acc0, acc1);
+                        tmem_st16(lane_base + col_s + 32 * h, pk);
+                        softmax_chunk<true, 1>(s, scale2, off2, pk, acc0, acc1);
+                        tmem_st16(lane_base + col_s + 32 * h + 16, pk);
+                    }
                 }
                 {
                     float a0, a1, b0, b1;
