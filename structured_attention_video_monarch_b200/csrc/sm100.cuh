@@ -44,6 +44,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same, but a thread whose phase has not completed is suspended in hardware
+// for up to `hint_ns` nanoseconds (woken early when the phase completes), so
+// waiting warps do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Device status bits (written with atomicOr into the library's status word).
 enum : unsigned {
     DEVERR_TIMEOUT = 1u,
@@ -60,19 +75,18 @@ struct WaitCtl {
 
 // Waits until the phase with parity `parity` of the barrier has completed.
 // Returns false (and raises the CTA's abort flag) when the wait gives up.
+// Each try suspends the thread for at most 0.5 ms, so the time limit and the
+// abort flag are checked at least that often.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl &ctl) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
-    uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((++spins & 63u) == 0) {
-            if (*ctl.abort_flag) return false;
-            if (clock64() - t0 > ctl.limit_cycles) {
-                atomicOr(ctl.status, DEVERR_TIMEOUT);
-                *ctl.abort_flag = 1u;
-                return false;
-            }
+        if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
+        if (*ctl.abort_flag) return false;
+        if (clock64() - t0 > ctl.limit_cycles) {
+            atomicOr(ctl.status, DEVERR_TIMEOUT);
+            *ctl.abort_flag = 1u;
+            return false;
         }
     }
 }
