@@ -19,7 +19,10 @@
  * with the stage-1 outputs as values.
  *
  * Every entry point is plain C: raw pointers, ints, and a cudaStream_t passed
- * as void*.  No entry point allocates device memory.
+ * as void*.  The bf16 path keeps a small per-(device, stream) buffer of
+ * completion counters (one 32-bit word per batch-head, at least 4 KB),
+ * allocated with cudaMalloc by the first call on that stream and reused
+ * afterwards; a call needing more drains the stream and reallocates it.
  */
 #ifndef MONARCH_ATTN_H
 #define MONARCH_ATTN_H
@@ -60,8 +63,8 @@ typedef enum {
  *             `dtype`.  Read only.
  *   out       device pointer, output, same layout and type.  Must not overlap
  *             q, k or v.  The stage-1 result is kept in `out` between the two
- *             stages (stage 2 reads and overwrites it group by group), so no
- *             scratch buffer is needed; out's prior contents are ignored.
+ *             stages (stage 2 reads and overwrites it group by group); out's
+ *             prior contents are ignored.
  *   B, heads  batch size and head count, >= 1.
  *   T, H, W   frames, height and width of the token grid, >= 1.
  *   d         head width: 64 or 128.
@@ -114,8 +117,9 @@ int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, voi
  * `events` holds `nevents` cudaEvent_t handles created by the caller
  * (entries beyond what the call needs are left untouched; NULL entries are
  * skipped).  *nlaunch (if not NULL) receives the number of kernel launches
- * the call queued: 2 (stage 1, then stage 2).  Same arguments, rules and
- * status codes as monarch_attn_fwd otherwise.
+ * the call queued: 1 for bf16 (both stages in one persistent kernel), 2 for
+ * fp32 (stage 1, then stage 2).  Same arguments, rules and status codes as
+ * monarch_attn_fwd otherwise.
  */
 int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void *out,
                               int B, int heads, int T, int H, int W, int d,

@@ -63,9 +63,13 @@ struct TcParams {
     int upg;                        // units per group of two blocks: 2*ns + odd
     int npos;                       // stage-2 positions per chunk
     int s2_chunks;                  // chunks per (batch, head)
-    int s2_pairs;                   // ceil(s2_chunks / 2)
-    long long s1_units, s2_units;
-    long long unit_begin, unit_end; // [begin, end) over stage-1 units then stage-2 units
+    int s2_pairs;                   // ceil(s2_chunks / 2) = stage-2 units per (batch, head)
+    int BH;                         // batch x heads
+    int u1_bh;                      // stage-1 units per (batch, head)
+    int lag;                        // stage-2 units of bh follow the stage-1 units of bh + lag
+    long long units;                // all units of the call
+    unsigned *s1_done;              // per batch-head: stage-1 lanes whose Y1 rows are stored
+    unsigned s1_target;             // stage-1 lanes per batch-head
     float scale_log2;               // d^-1/2 * log2(e)
     long long timeout_cycles;
     unsigned *status;
@@ -85,40 +89,62 @@ struct Unit {
     Lane ln[2];
 };
 
-__device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
-    Unit r;
-    if (u < p.s1_units) {
-        r.kind = UNIT_STAGE1;
-        r.nk = p.nqt;
-        const long long g = u / p.upg;
-        const int rr = static_cast<int>(u - g * p.upg);
-        const int b0 = static_cast<int>(2 * g);
-        const bool two = b0 + 1 < p.nblocks;
-        if (rr < p.ns || (two && rr < 2 * p.ns)) {
-            const int blk = rr < p.ns ? b0 : b0 + 1;
-            const int pr = rr < p.ns ? rr : rr - p.ns;
-            r.shared = 1;
-            r.nq = 2;
-            r.ln[0] = {blk, 2 * pr};
-            r.ln[1] = {blk, 2 * pr + 1};
-        } else {  // the odd last tiles of blocks b0 and b0+1
-            r.shared = 0;
-            r.nq = two ? 2 : 1;
-            r.ln[0] = {b0, p.nqt - 1};
-            r.ln[1] = {two ? b0 + 1 : b0, p.nqt - 1};
-        }
+// Stage-1 unit r of batch-head bh: blocks are taken in pairs (lb0, lb0+1) of
+// this batch-head; a pair's units are the shared query-tile pairs of both
+// blocks, then one unit joining their odd last query tiles.
+__device__ __forceinline__ Unit decode_stage1(const TcParams &p, int bh, int r) {
+    Unit un;
+    un.kind = UNIT_STAGE1;
+    un.nk = p.nqt;
+    const int g = r / p.upg, rr = r - g * p.upg;
+    const int lb0 = 2 * g;
+    const bool two = lb0 + 1 < p.nblk_bh;
+    const int b0 = bh * p.nblk_bh + lb0;
+    if (rr < p.ns || (two && rr < 2 * p.ns)) {
+        const int blk = rr < p.ns ? b0 : b0 + 1;
+        const int pr = rr < p.ns ? rr : rr - p.ns;
+        un.shared = 1;
+        un.nq = 2;
+        un.ln[0] = {blk, 2 * pr};
+        un.ln[1] = {blk, 2 * pr + 1};
     } else {
-        const long long v = u - p.s1_units;
-        r.kind = UNIT_STAGE2;
-        r.nk = 1;
-        r.shared = 0;
-        const int bh = static_cast<int>(v / p.s2_pairs);
-        const int c0 = 2 * static_cast<int>(v % p.s2_pairs);
-        r.nq = (c0 + 1 < p.s2_chunks) ? 2 : 1;
-        r.ln[0] = {bh, c0};
-        r.ln[1] = {bh, c0 + 1};
+        un.shared = 0;
+        un.nq = two ? 2 : 1;
+        un.ln[0] = {b0, p.nqt - 1};
+        un.ln[1] = {two ? b0 + 1 : b0, p.nqt - 1};
     }
-    return r;
+    return un;
+}
+
+__device__ __forceinline__ Unit decode_stage2(const TcParams &p, int bh, int r) {
+    Unit un;
+    un.kind = UNIT_STAGE2;
+    un.nk = 1;
+    un.shared = 0;
+    const int c0 = 2 * r;
+    un.nq = (c0 + 1 < p.s2_chunks) ? 2 : 1;
+    un.ln[0] = {bh, c0};
+    un.ln[1] = {bh, c0 + 1};
+    return un;
+}
+
+// Unit u of the call.  Units are ordered in slots s = 0, 1, ...: slot s holds
+// the stage-1 units of batch-head s (while s < BH) followed by the stage-2
+// units of batch-head s - lag (once s >= lag), so a batch-head's stage-2
+// units come about `lag` batch-heads of work after its stage-1 units.
+__device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
+    const long long U1 = p.u1_bh, U2 = p.s2_pairs;
+    const long long L = p.lag < p.BH ? p.lag : p.BH;
+    if (u < L * U1) return decode_stage1(p, static_cast<int>(u / U1), static_cast<int>(u % U1));
+    u -= L * U1;
+    const long long nB = p.BH - L;  // slots holding both kinds
+    if (u < nB * (U1 + U2)) {
+        const long long s = u / (U1 + U2), r = u - s * (U1 + U2);
+        if (r < U1) return decode_stage1(p, static_cast<int>(L + s), static_cast<int>(r));
+        return decode_stage2(p, static_cast<int>(s), static_cast<int>(r - U1));
+    }
+    u -= nB * (U1 + U2);
+    return decode_stage2(p, static_cast<int>(nB + u / U2), static_cast<int>(u % U2));
 }
 
 // Rows a stage-1 tile (query or key tile `tile` of a block) brings in by TMA,
@@ -247,28 +273,6 @@ __device__ __forceinline__ void setmaxnreg_dec64() {
 
 // ---------------------------------------------------------------- softmax math
 
-// 2^x for a pair of floats on the FMA pipe (offloads the MUFU unit).
-// Range reduction 2^x = 2^j * 2^f, j = floor(x), f in [0, 1): j comes from a
-// round-down add of 1.5*2^23 (the integer lands in the low mantissa bits, and
-// shifting those bits left by 23 puts j straight into the exponent field);
-// 2^f ~= 1 + f*(a1 + f*(a2 + f*a3)), a cubic fitted here for minimal relative
-// error with p(0) = 1, p(1) = 2 (max relative error 1.03e-4, below bf16's
-// 2^-9 rounding of P).  x is clamped to -126 so 2^j stays a normal number;
-// callers only pass finite x (masked tiles use the MUFU path).
-__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
-    const uint64_t x = pack_f32x2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-    const uint64_t t = add_rm_f32x2(x, pack_f32x2(12582912.f, 12582912.f));
-    const uint64_t f = sub_f32x2(x, add_f32x2(t, pack_f32x2(-12582912.f, -12582912.f)));
-    uint64_t q = fma_f32x2(f, pack_f32x2(0.07826797f, 0.07826797f), pack_f32x2(0.22630768f, 0.22630768f));
-    q = fma_f32x2(q, f, pack_f32x2(0.6954244f, 0.6954244f));
-    q = fma_f32x2(q, f, pack_f32x2(1.f, 1.f));
-    float q0, q1, t0, t1;
-    unpack_f32x2(q, q0, q1);
-    unpack_f32x2(t, t0, t1);
-    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -276,11 +280,9 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
-// bf16 pairs, and accumulate the rounded P into two packed fp32 partial sums
-// (even and odd pairs, so the additions form two independent chains).  With
-// EMULATE, 6 of the 16 pairs take exp2_poly_pair on the FMA pipe and the rest
-// MUFU ex2, balancing the two units.
-template <bool EMULATE, int C>
+// bf16 pairs, and accumulate P into two packed fp32 partial sums (even and
+// odd pairs, so the additions form two independent chains).
+template <int C>
 __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t scale, uint64_t off,
                                               uint32_t (&pk)[16], uint64_t &acc0, uint64_t &acc1) {
 #pragma unroll
@@ -288,16 +290,12 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t sca
         const uint64_t x = fma_f32x2(pack_f32x2(s[32 * C + 2 * e], s[32 * C + 2 * e + 1]), scale, off);
         float x0, x1, a, b;
         unpack_f32x2(x, x0, x1);
-        if (EMULATE && (e % 8 == 1 || e % 8 == 4 || e % 8 == 6)) {
-            exp2_poly_pair(x0, x1, a, b);
-        } else {
-            a = fast_exp2(x0);
-            b = fast_exp2(x1);
-        }
+        a = fast_exp2(x0);
+        b = fast_exp2(x1);
         const uint32_t w = pack_bf16x2(a, b);
         pk[e] = w;
         // the denominator sums the bf16-rounded weights the PV MMA uses
-        const uint64_t r = pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+        const uint64_t r = pack_f32x2(a, b);  // softmax denominator
         if (e & 1)
             acc1 = add_f32x2(acc1, r);
         else
@@ -408,7 +406,15 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     s2_load<NP>(is_v ? &my2 : &mk2, dst, kv_full(s), p.npos, ln.blk, ln.tile);
                 return true;
             };
-            for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
+            // Stage 2 reads Y1 rows that stage-1 lanes of this batch-head (on
+            // any SM) stored with plain stores: wait until all of them have
+            // published (acquire), then order the TMA reads after that.
+            auto wait_stage1 = [&](int bh) -> bool {
+                if (!wait_counter(p.s1_done + bh, p.s1_target, ctl)) return false;
+                fence_proxy_async_global();
+                return true;
+            };
+            for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
                 for (int i = 0; i < un.nq && ok; ++i) {
                     ok = mbar_wait(q_empty(i), (qe_par >> i) & 1u, ctl);
@@ -430,6 +436,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         ok = load_kv(un, un.ln[0], j, false) && load_kv(un, un.ln[0], j, true);
                     } else {
                         for (int i = 0; i < un.nq && ok; ++i) ok = load_kv(un, un.ln[i], j, false);
+                        if (ok && un.kind == UNIT_STAGE2) ok = wait_stage1(un.ln[0].blk);
                         for (int i = 0; i < un.nq && ok; ++i) ok = load_kv(un, un.ln[i], j, true);
                     }
                 }
@@ -497,7 +504,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 tc_fence_after();
                 return true;
             };
-            for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
+            for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
                 for (int i = 0; i < un.nq && ok; ++i) {
                     ok = mbar_wait(q_full(i), (qf_par >> i) & 1u, ctl);
@@ -596,7 +603,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             named_barrier_sync(1 + li, 256);
             return xb[(1 - h) * 128 + row];
         };
-        for (long long u = p.unit_begin + blockIdx.x; u < p.unit_end && ok; u += gridDim.x) {
+        for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u);
             if (li >= un.nq) continue;
             float m_run = -INFINITY;  // running max of raw logits (whole row)
@@ -679,17 +686,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 // packed columns [32h, 32h+32) of the lane's S region
                 {
                     uint32_t pk[16];
-                    if (masked) {  // masked columns need MUFU's exact 2^-inf = 0
-                        softmax_chunk<false, 0>(s, scale2, off2, pk, acc0, acc1);
-                        tmem_st16(lane_base + col_s + 32 * h, pk);
-                        softmax_chunk<false, 1>(s, scale2, off2, pk, acc0, acc1);
-                        tmem_st16(lane_base + col_s + 32 * h + 16, pk);
-                    } else {
-                        softmax_chunk<true, 0>(s, scale2, off2, pk, acc0, acc1);
-                        tmem_st16(lane_base + col_s + 32 * h, pk);
-                        softmax_chunk<true, 1>(s, scale2, off2, pk, acc0, acc1);
-                        tmem_st16(lane_base + col_s + 32 * h + 16, pk);
-                    }
+                    softmax_chunk<0>(s, scale2, off2, pk, acc0, acc1);  // masked: 2^-inf = 0
+                    tmem_st16(lane_base + col_s + 32 * h, pk);
+                    softmax_chunk<1>(s, scale2, off2, pk, acc0, acc1);
+                    tmem_st16(lane_base + col_s + 32 * h + 16, pk);
                 }
                 {
                     float a0, a1, b0, b1;
@@ -748,6 +748,17 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             // O_i has been read: the next unit may overwrite it
             tc_fence_before();
             mbar_arrive(o_free(li));
+            if (un.kind == UNIT_STAGE1) {
+                // publish this lane's Y1 rows to the stage-2 units of its
+                // batch-head: every storing thread orders its stores for the
+                // async proxy, the lane's 256 threads meet, one releases
+                fence_proxy_async_global();
+                named_barrier_sync(7 + li, 256);
+                if (h == 0 && row == 0) {
+                    __threadfence();
+                    atomicAdd(p.s1_done + bh, 1u);
+                }
+            }
         }
     }
 

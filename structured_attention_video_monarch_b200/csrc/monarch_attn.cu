@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/monarch_attn.h"
 #include "attn_f32.cuh"
@@ -30,6 +31,17 @@ struct DeviceInfo {
     bool tc_attr[2] = {false, false};
     bool f32_attr[2] = {false, false};
 };
+
+// Per (device, stream) buffer of per-batch-head stage-1 completion counters:
+// calls queued on one stream run in order, so each buffer is used by one call
+// at a time; calls on different streams get different buffers.
+struct CounterBuf {
+    int dev;
+    cudaStream_t stream;
+    unsigned *ptr;
+    size_t cap;  // elements
+};
+std::vector<CounterBuf> g_counters;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 
@@ -63,6 +75,36 @@ int device_info(DeviceInfo **out) {
         di.init = true;
     }
     *out = &di;
+    return MONARCH_OK;
+}
+
+// Counter buffer of at least n elements for (current device, stream),
+// allocated on first use; when a call needs more, the stream is drained and
+// the buffer replaced.
+int counters_for(cudaStream_t stream, size_t n, unsigned **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    CounterBuf *cb = nullptr;
+    for (auto &c : g_counters)
+        if (c.dev == dev && c.stream == stream) cb = &c;
+    if (!cb) {
+        g_counters.push_back(CounterBuf{dev, stream, nullptr, 0});
+        cb = &g_counters.back();
+    }
+    if (cb->cap < n) {
+        const size_t cap = n < 1024 ? 1024 : n;
+        if (cb->ptr) {
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return MONARCH_ERR_CUDA;
+            cudaFree(cb->ptr);
+            cb->ptr = nullptr;
+            cb->cap = 0;
+        }
+        if (cudaMalloc(reinterpret_cast<void **>(&cb->ptr), cap * sizeof(unsigned)) != cudaSuccess)
+            return MONARCH_ERR_CUDA;
+        cb->cap = cap;
+    }
+    *out = cb->ptr;
     return MONARCH_OK;
 }
 
@@ -208,16 +250,27 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     const long long bh = static_cast<long long>(s.B) * s.heads;
     if (bh * p.nblk_bh >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
     p.nblocks = static_cast<int>(bh * p.nblk_bh);
+    p.BH = static_cast<int>(bh);
     p.ns = p.nqt / 2;
     p.odd = p.nqt % 2;
     p.upg = 2 * p.ns + p.odd;
     p.npos = 128 / s.T;
     p.s2_chunks = (p.HW + p.npos - 1) / p.npos;
     p.s2_pairs = (p.s2_chunks + 1) / 2;
-    // stage-1 units: groups of two blocks, each group = the shared query-tile
-    // pairs of both blocks and one unit pairing their odd last tiles
-    p.s1_units = static_cast<long long>(p.nblocks / 2) * p.upg + (p.nblocks % 2) * (p.ns + p.odd);
-    p.s2_units = bh * p.s2_pairs;
+    // stage-1 units per batch-head: blocks in pairs, each pair = the shared
+    // query-tile pairs of both blocks plus one unit joining their odd tiles
+    p.u1_bh = (p.nblk_bh / 2) * p.upg + (p.nblk_bh % 2) * (p.ns + p.odd);
+    p.units = bh * (p.u1_bh + p.s2_pairs);
+    p.s1_target = static_cast<unsigned>(p.nblk_bh) * static_cast<unsigned>(p.nqt);
+    // Stage-2 units of a batch-head trail its stage-1 units by about two
+    // waves of the persistent grid, so they rarely wait on their inputs.
+    {
+        const long long wave = di->sms;
+        long long lag = (2 * wave + p.u1_bh - 1) / p.u1_bh;
+        if (lag < 1) lag = 1;
+        if (lag > bh) lag = bh;
+        p.lag = static_cast<int>(lag);
+    }
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.d)));
     p.timeout_cycles = env_timeout_cycles();
     p.out = out;
@@ -232,19 +285,20 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         (st = stage2_map(&mk2, k, s, p)) || (st = stage2_map(&my2, out, s, p)))
         return st;
 
-    // stage 1: Y1 = B1 V into out; stage 2: out = P^T B2 P Y1 in place.
-    const long long ranges[2][2] = {{0, p.s1_units}, {p.s1_units, p.s1_units + p.s2_units}};
+    // One persistent launch runs both stages: stage-1 units write Y1 = B1 V
+    // into out; stage-2 units overwrite it in place with P^T B2 P Y1 once the
+    // stage-1 lanes of their batch-head have published (per-batch-head
+    // counters, zeroed for every call).
+    unsigned *counters = nullptr;
+    if ((st = counters_for(stream, static_cast<size_t>(bh), &counters))) return st;
+    p.s1_done = counters;
+    if (cudaMemsetAsync(counters, 0, static_cast<size_t>(bh) * sizeof(unsigned), stream) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
     lev.record(0, stream);
-    for (int r = 0; r < 2; ++r) {
-        p.unit_begin = ranges[r][0];
-        p.unit_end = ranges[r][1];
-        const long long units = p.unit_end - p.unit_begin;
-        if (units <= 0) continue;
-        const int grid = static_cast<int>(units < di->sms ? units : di->sms);
-        monarch_tc_kernel<D><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
-        if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
-        lev.record(++lev.launches, stream);
-    }
+    const int grid = static_cast<int>(p.units < di->sms ? p.units : di->sms);
+    monarch_tc_kernel<D><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    lev.record(++lev.launches, stream);
     return MONARCH_OK;
 }
 

@@ -91,6 +91,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
 }
 
+// Waits until *counter >= target (acquire at GPU scope), sleeping between
+// polls; gives up like mbar_wait.
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ bool wait_counter(const unsigned *counter, unsigned target, const WaitCtl &ctl) {
+    if (ld_acquire_gpu(counter) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(200);
+        if (ld_acquire_gpu(counter) >= target) return true;
+        if (*ctl.abort_flag) return false;
+        if (clock64() - t0 > ctl.limit_cycles) {
+            atomicOr(ctl.status, DEVERR_TIMEOUT);
+            *ctl.abort_flag = 1u;
+            return false;
+        }
+    }
+}
+
 // ----------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
@@ -161,6 +183,11 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 // Wait until all committed bulk stores have completed (writes visible).
 __device__ __forceinline__ void bulk_wait_group0() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Orders this thread's generic-proxy global-memory accesses with async-proxy
+// (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA, tensor core) accesses.
