@@ -29,7 +29,8 @@
 //   warps 4-7, 12-15   the same for lane 1                            104 regs
 //   warp  16           TMA producer (Q tiles, K/V ring)                64 regs
 //   warp  17           TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 18-19        idle
+//   warp  18           publishes finished stage-1 lanes to stage-2 units
+//   warp  19           idle
 // (4*128*104 + 128*64 = 61440 = 640 threads x 96, the launch allocation.)
 // Splitting each row over two warps puts two warps of the same lane on every
 // SM sub-partition, so the exp/pack work of one tile is spread over twice the
@@ -237,8 +238,8 @@ struct TcLayout {
     static constexpr int OFF_KV = OFF_Q + 2 * TILE;
     static constexpr int OFF_BAR = OFF_KV + NS * TILE;
     // barriers: q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2]
-    //           o_full[2] o_free[2]
-    static constexpr int NBAR = 12 + 2 * NS;
+    //           o_full[2] o_free[2] y_done[2] y_free[2]
+    static constexpr int NBAR = 16 + 2 * NS;
     // exchange of per-row values (partial maxima, partial sums) between the two
     // column halves of a lane: [2 lanes][2 halves][128 rows] fp32
     static constexpr int OFF_X = OFF_BAR + NBAR * 8;
@@ -330,6 +331,8 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     auto p_full = [&](int i) { return bar0 + 8u * (6 + 2 * NS + i); };
     auto o_full = [&](int i) { return bar0 + 8u * (8 + 2 * NS + i); };
     auto o_free = [&](int i) { return bar0 + 8u * (10 + 2 * NS + i); };
+    auto y_done = [&](int i) { return bar0 + 8u * (12 + 2 * NS + i); };
+    auto y_free = [&](int i) { return bar0 + 8u * (14 + 2 * NS + i); };
     float *x_buf = reinterpret_cast<float *>(base_ptr + L::OFF_X);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
@@ -348,6 +351,8 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             mbar_init(p_full(i), 256);
             mbar_init(o_full(i), 1);
             mbar_init(o_free(i), 256);
+            mbar_init(y_done(i), 256);
+            mbar_init(y_free(i), 1);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full(s), 1);
@@ -370,6 +375,27 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
 
     if (wg == 4) {
         setmaxnreg_dec64();
+        if (warp == 18 && lane == 0) {
+            // ------------------------------------------------------ Y1 publisher
+            // Once the 256 threads of a stage-1 lane have stored its Y1 rows
+            // (y_done), make them visible at GPU scope and count the lane for
+            // its batch-head; stage-2 units acquire that count.  Kept off the
+            // softmax warps so the fence latency is not on their path.
+            uint32_t yd_par = 0u;  // bit i: parity to wait for on y_done(i)
+            bool ok = true;
+            for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+                const Unit un = decode_unit(p, u);
+                if (un.kind != UNIT_STAGE1) continue;
+                for (int i = 0; i < un.nq && ok; ++i) {
+                    ok = mbar_wait(y_done(i), (yd_par >> i) & 1u, ctl);
+                    yd_par ^= 1u << i;
+                    if (!ok) break;
+                    __threadfence();
+                    atomicAdd(p.s1_done + un.ln[i].blk / p.nblk_bh, 1u);
+                    mbar_arrive(y_free(i));
+                }
+            }
+        }
         if (warp == 16 && lane == 0) {
             // -------------------------------------------------------- TMA producer
             uint32_t qe_par = 3u;  // bit i: parity to wait for on q_empty(i)
@@ -591,7 +617,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         const uint32_t col_s = li ? L::COL_S1 : L::COL_S0;
         const uint32_t col_o = li ? L::COL_O1 : L::COL_O0;
         const float sl2 = p.scale_log2;
-        uint32_t sf_par = 0u, of_par = 0u;
+        uint32_t sf_par = 0u, of_par = 0u, yf_par = 1u;
         bool ok = true;
         // value of this row in the other column half of the lane: barrier
         // 3+li makes sure the other half has read the previous value before
@@ -749,15 +775,11 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             tc_fence_before();
             mbar_arrive(o_free(li));
             if (un.kind == UNIT_STAGE1) {
-                // publish this lane's Y1 rows to the stage-2 units of its
-                // batch-head: every storing thread orders its stores for the
-                // async proxy, the lane's 256 threads meet, one releases
-                fence_proxy_async_global();
-                named_barrier_sync(7 + li, 256);
-                if (h == 0 && row == 0) {
-                    __threadfence();
-                    atomicAdd(p.s1_done + bh, 1u);
-                }
+                // Y1 rows stored: hand them to the publisher (one-slot
+                // handshake, so y_done never runs a phase ahead of it)
+                if (!mbar_wait(y_free(li), yf_par, ctl)) { ok = false; break; }
+                yf_par ^= 1u;
+                mbar_arrive(y_done(li));
             }
         }
     }

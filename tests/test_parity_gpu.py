@@ -144,7 +144,14 @@ def test_tiled_edge_cases(B, heads, T, H, W, d, th, tw, dtype):
 
 
 def test_large_logits_rescale_path():
-    """Peaked softmax rows (large |q.k|) exercise the running-max rescale."""
+    """Peaked softmax rows (large |q.k|) exercise the running-max rescale.
+
+    This input lies far outside the workloads (logit spread ~6x theirs), so it
+    is held to a bound derived from the arithmetic rather than the workloads'
+    2e-2: when one weight dominates a row, the bf16 rounding of that weight
+    (relative 2^-9) reaches the output once in each stage, and the bf16 output
+    rounding adds one more half-ulp: 3 * 2^-9 * max|V|.
+    """
     B, heads, T, H, W, d = 1, 2, 3, 30, 52, 128
     q, k, v = workloads.random_inputs(B, heads, T, H, W, d, seed=77)
     # make later key tiles of each frame dominate so the running max grows
@@ -152,8 +159,12 @@ def test_large_logits_rescale_path():
     k.view(B, heads, T, H * W, d)[:, :, :, 1000:] *= 3.0
     k = k.to(torch.bfloat16)
     q = (q.float() * 2.0).to(torch.bfloat16)
-    got = _run(q, k, v, T, H, W)
-    _check(got, oracle.monarch_fwd(q, k, v, T, H, W), torch.bfloat16)
+    got = _run(q, k, v, T, H, W).double().numpy()
+    ref = oracle.monarch_fwd(q, k, v, T, H, W)
+    assert np.isfinite(got).all()
+    atol = 3 * 2.0 ** -9 * float(v.float().abs().max())
+    assert np.abs(got - ref).max() <= atol
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= BF16_RL2
 
 
 def test_constant_values_and_zero_qk():
