@@ -68,7 +68,10 @@ struct TcParams {
     int BH;                         // batch x heads
     int u1_bh;                      // stage-1 units per (batch, head)
     int lag;                        // stage-2 units of bh follow the stage-1 units of bh + lag
-    long long units;                // all units of the call
+    int units;                      // all units of the call
+    // divisions by launch constants, as multiply-shift
+    FastDiv fd_u1, fd_u12, fd_u2;   // u1_bh, u1_bh + s2_pairs, s2_pairs
+    FastDiv fd_upg, fd_nblk_bh, fd_tpf, fd_tiles_w, fd_tile_w, fd_npos;
     unsigned *s1_done;              // per batch-head: stage-1 lanes whose Y1 rows are stored
     unsigned s1_target;             // stage-1 lanes per batch-head
     float scale_log2;               // d^-1/2 * log2(e)
@@ -97,7 +100,7 @@ __device__ __forceinline__ Unit decode_stage1(const TcParams &p, int bh, int r) 
     Unit un;
     un.kind = UNIT_STAGE1;
     un.nk = p.nqt;
-    const int g = r / p.upg, rr = r - g * p.upg;
+    const int g = static_cast<int>(fdiv(r, p.fd_upg)), rr = r - g * p.upg;
     const int lb0 = 2 * g;
     const bool two = lb0 + 1 < p.nblk_bh;
     const int b0 = bh * p.nblk_bh + lb0;
@@ -133,19 +136,23 @@ __device__ __forceinline__ Unit decode_stage2(const TcParams &p, int bh, int r) 
 // the stage-1 units of batch-head s (while s < BH) followed by the stage-2
 // units of batch-head s - lag (once s >= lag), so a batch-head's stage-2
 // units come about `lag` batch-heads of work after its stage-1 units.
-__device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
-    const long long U1 = p.u1_bh, U2 = p.s2_pairs;
-    const long long L = p.lag < p.BH ? p.lag : p.BH;
-    if (u < L * U1) return decode_stage1(p, static_cast<int>(u / U1), static_cast<int>(u % U1));
+__device__ __forceinline__ Unit decode_unit(const TcParams &p, int u) {
+    const int U1 = p.u1_bh, U2 = p.s2_pairs;
+    const int L = p.lag < p.BH ? p.lag : p.BH;
+    if (u < L * U1) {
+        const int s = static_cast<int>(fdiv(u, p.fd_u1));
+        return decode_stage1(p, s, u - s * U1);
+    }
     u -= L * U1;
-    const long long nB = p.BH - L;  // slots holding both kinds
+    const int nB = p.BH - L;  // slots holding both kinds
     if (u < nB * (U1 + U2)) {
-        const long long s = u / (U1 + U2), r = u - s * (U1 + U2);
-        if (r < U1) return decode_stage1(p, static_cast<int>(L + s), static_cast<int>(r));
-        return decode_stage2(p, static_cast<int>(s), static_cast<int>(r - U1));
+        const int s = static_cast<int>(fdiv(u, p.fd_u12)), r = u - s * (U1 + U2);
+        if (r < U1) return decode_stage1(p, L + s, r);
+        return decode_stage2(p, s, r - U1);
     }
     u -= nB * (U1 + U2);
-    return decode_stage2(p, static_cast<int>(nB + u / U2), static_cast<int>(u % U2));
+    const int s = static_cast<int>(fdiv(u, p.fd_u2));
+    return decode_stage2(p, nB + s, u - s * U2);
 }
 
 // Rows a stage-1 tile (query or key tile `tile` of a block) brings in by TMA,
@@ -184,9 +191,9 @@ __device__ __forceinline__ void s1_load(const TcParams &p, const CUtensorMap *ma
 #pragma unroll
         for (int pn = 0; pn < NP; ++pn) tma_load_3d(dst + pn * 16384, map, bar, pn * 64, tile * 128, blk);
     } else {
-        const int tpf = p.tiles_h * p.tiles_w;
-        const int frame = blk / tpf, tif = blk % tpf;
-        const int ti = tif / p.tiles_w, tj = tif % p.tiles_w;
+        const int frame = static_cast<int>(fdiv(blk, p.fd_tpf));
+        const int tif = blk - frame * p.tiles_h * p.tiles_w;
+        const int ti = static_cast<int>(fdiv(tif, p.fd_tiles_w)), tj = tif - ti * p.tiles_w;
 #pragma unroll
         for (int pn = 0; pn < NP; ++pn)
             tma_load_5d(dst + pn * 16384, map, bar, pn * 64, 0, tj, tile * p.rows_per_tile,
@@ -206,24 +213,23 @@ __device__ __forceinline__ void s2_load(const CUtensorMap *map, uint32_t dst, ui
 __device__ __forceinline__ long long lane_row_token(const TcParams &p, int kind, const Lane &ln, int row,
                                                     int &bh) {
     if (kind == UNIT_STAGE1) {
-        bh = ln.blk / p.nblk_bh;
+        bh = static_cast<int>(fdiv(ln.blk, p.fd_nblk_bh));
         const int b = ln.blk - bh * p.nblk_bh;
         if (p.fact == 0) {
             const int i = ln.tile * 128 + row;
             if (i >= p.m) return -1;
             return static_cast<long long>(b) * p.HW + i;
         }
-        const int tpf = p.tiles_h * p.tiles_w;
-        const int t = b / tpf, tif = b % tpf;
-        const int ti = tif / p.tiles_w, tj = tif % p.tiles_w;
-        const int rr = row / p.tile_w, wl = row - rr * p.tile_w;
+        const int t = static_cast<int>(fdiv(b, p.fd_tpf)), tif = b - t * p.tiles_h * p.tiles_w;
+        const int ti = static_cast<int>(fdiv(tif, p.fd_tiles_w)), tj = tif - ti * p.tiles_w;
+        const int rr = static_cast<int>(fdiv(row, p.fd_tile_w)), wl = row - rr * p.tile_w;
         const int hl = ln.tile * p.rows_per_tile + rr;
         if (rr >= p.rows_per_tile || hl >= p.tile_h) return -1;
         return static_cast<long long>(t) * p.HW + static_cast<long long>(ti * p.tile_h + hl) * p.W +
                tj * p.tile_w + wl;
     }
     bh = ln.blk;
-    const int t = row / p.npos, pl = row - t * p.npos;
+    const int t = static_cast<int>(fdiv(row, p.fd_npos)), pl = row - t * p.npos;
     const int pos = ln.tile * p.npos + pl;
     if (t >= p.T || pos >= p.HW) return -1;
     return static_cast<long long>(t) * p.HW + pos;
@@ -383,7 +389,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             // softmax warps so the fence latency is not on their path.
             uint32_t yd_par = 0u;  // bit i: parity to wait for on y_done(i)
             bool ok = true;
-            for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
                 if (un.kind != UNIT_STAGE1) continue;
                 for (int i = 0; i < un.nq && ok; ++i) {
@@ -391,7 +397,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     yd_par ^= 1u << i;
                     if (!ok) break;
                     __threadfence();
-                    atomicAdd(p.s1_done + un.ln[i].blk / p.nblk_bh, 1u);
+                    atomicAdd(p.s1_done + fdiv(un.ln[i].blk, p.fd_nblk_bh), 1u);
                     mbar_arrive(y_free(i));
                 }
             }
@@ -440,7 +446,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 fence_proxy_async_global();
                 return true;
             };
-            for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
                 for (int i = 0; i < un.nq && ok; ++i) {
                     ok = mbar_wait(q_empty(i), (qe_par >> i) & 1u, ctl);
@@ -530,7 +536,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 tc_fence_after();
                 return true;
             };
-            for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
                 for (int i = 0; i < un.nq && ok; ++i) {
                     ok = mbar_wait(q_full(i), (qf_par >> i) & 1u, ctl);
@@ -629,13 +635,13 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             named_barrier_sync(1 + li, 256);
             return xb[(1 - h) * 128 + row];
         };
-        for (long long u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u);
             if (li >= un.nq) continue;
             float m_run = -INFINITY;  // running max of raw logits (whole row)
             float l_half = 0.f;       // softmax denominator over this half's columns
             // stage-2 mask: the row belongs to position slot prow of its chunk
-            const int prow = (un.kind == UNIT_STAGE2) ? (row % p.npos) : 0;
+            const int prow = (un.kind == UNIT_STAGE2) ? static_cast<int>(fmod_(row, p.fd_npos)) : 0;
             int npos_valid = 0;
             if (un.kind == UNIT_STAGE2) {
                 const int rem = p.HW - un.ln[li].tile * p.npos;
@@ -665,7 +671,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         for (int c = 0; c < 64; ++c)
                             if (64 * h + c >= kvalid) s[c] = -INFINITY;
                     } else {
-                        int pc = (64 * h) % p.npos, tc = (64 * h) / p.npos;
+                        int tc = static_cast<int>(fdiv(64 * h, p.fd_npos)), pc = 64 * h - tc * p.npos;
 #pragma unroll
                         for (int c = 0; c < 64; ++c) {
                             const bool valid = (pc == prow) && (tc < p.T) && (pc < npos_valid);

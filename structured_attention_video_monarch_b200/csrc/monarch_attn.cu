@@ -260,7 +260,9 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     // stage-1 units per batch-head: blocks in pairs, each pair = the shared
     // query-tile pairs of both blocks plus one unit joining their odd tiles
     p.u1_bh = (p.nblk_bh / 2) * p.upg + (p.nblk_bh % 2) * (p.ns + p.odd);
-    p.units = bh * (p.u1_bh + p.s2_pairs);
+    const long long units = bh * (p.u1_bh + p.s2_pairs);
+    if (units >= (1ll << 31) - 1) return MONARCH_ERR_UNSUPPORTED;
+    p.units = static_cast<int>(units);
     p.s1_target = static_cast<unsigned>(p.nblk_bh) * static_cast<unsigned>(p.nqt);
     // Stage-2 units of a batch-head trail its stage-1 units by about two
     // waves of the persistent grid, so they rarely wait on their inputs.
@@ -271,6 +273,15 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         if (lag > bh) lag = bh;
         p.lag = static_cast<int>(lag);
     }
+    p.fd_u1 = make_fastdiv(static_cast<uint32_t>(p.u1_bh));
+    p.fd_u12 = make_fastdiv(static_cast<uint32_t>(p.u1_bh + p.s2_pairs));
+    p.fd_u2 = make_fastdiv(static_cast<uint32_t>(p.s2_pairs));
+    p.fd_upg = make_fastdiv(static_cast<uint32_t>(p.upg));
+    p.fd_nblk_bh = make_fastdiv(static_cast<uint32_t>(p.nblk_bh));
+    p.fd_tpf = make_fastdiv(static_cast<uint32_t>(p.fact ? p.tiles_h * p.tiles_w : 1));
+    p.fd_tiles_w = make_fastdiv(static_cast<uint32_t>(p.fact ? p.tiles_w : 1));
+    p.fd_tile_w = make_fastdiv(static_cast<uint32_t>(p.fact ? p.tile_w : 1));
+    p.fd_npos = make_fastdiv(static_cast<uint32_t>(p.npos));
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.d)));
     p.timeout_cycles = env_timeout_cycles();
     p.out = out;
@@ -295,7 +306,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     if (cudaMemsetAsync(counters, 0, static_cast<size_t>(bh) * sizeof(unsigned), stream) != cudaSuccess)
         return MONARCH_ERR_CUDA;
     lev.record(0, stream);
-    const int grid = static_cast<int>(p.units < di->sms ? p.units : di->sms);
+    const int grid = p.units < di->sms ? p.units : di->sms;
     monarch_tc_kernel<D><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
     lev.record(++lev.launches, stream);

@@ -13,6 +13,31 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ----------------------------------------------------------------- division
+
+// Division of n < 2^31 by a divisor fixed at launch: with s = ceil(log2 d)
+// and m = ceil(2^(31+s) / d) (m <= 2^32 - 1 for d >= 2), floor(n / d) =
+// umulhi(n, m) >> (s - 1): the rounding error of m adds less than
+// n / 2^(31+s) < 2^-s <= 1/d to n/d, which cannot cross an integer.
+struct FastDiv {
+    uint32_t d, m, s1;  // divisor, multiplier, shift (s - 1); m == 0 means d == 1
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f{d, 0u, 0u};
+    if (d <= 1) return f;
+    uint32_t s = 0;
+    while ((1ull << s) < d) ++s;
+    f.m = static_cast<uint32_t>(((1ull << (31 + s)) + d - 1) / d);
+    f.s1 = s - 1;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+    return f.m ? (__umulhi(n, f.m) >> f.s1) : n;
+}
+__device__ __forceinline__ uint32_t fmod_(uint32_t n, const FastDiv &f) { return n - fdiv(n, f) * f.d; }
+
 // ----------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
