@@ -235,6 +235,22 @@ __device__ __forceinline__ long long lane_row_token(const TcParams &p, int kind,
     return static_cast<long long>(t) * p.HW + pos;
 }
 
+// Bit c set when column c of a 64-column half holds a valid key: stage 1,
+// the first n columns; stage 2, the columns of the row's own position slot
+// (column 64h + c holds position slot (64h + c) % npos of frame (64h + c) / npos).
+__device__ __forceinline__ uint64_t stage1_valid_bits(int n) {
+    return n >= 64 ? ~0ull : (n <= 0 ? 0ull : ((1ull << n) - 1ull));
+}
+__device__ __noinline__ uint64_t stage2_valid_bits(const TcParams &p, int h, int prow, int npos_valid) {
+    uint64_t vm = 0;
+    if (prow >= npos_valid) return 0;
+    // first column >= 64h in slot prow, then every npos columns up to frame T-1
+    int c = prow - 64 * h;
+    if (c < 0) c += ((-c + p.npos - 1) / p.npos) * p.npos;
+    for (; c < 64 && 64 * h + c < p.npos * p.T; c += p.npos) vm |= 1ull << c;
+    return vm;
+}
+
 template <int D>
 struct TcLayout {
     static constexpr int NP = D / 64;                 // 64-element (128-byte) panels per row
@@ -404,72 +420,70 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         }
         if (warp == 16 && lane == 0) {
             // -------------------------------------------------------- TMA producer
+            // Load order per unit: Q of each lane, then per key tile j the K
+            // tile(s) then the V tile(s): one K and one V for a shared unit,
+            // K_A, K_B, V_A, V_B for a separate one.  The MMA issuer consumes
+            // the ring in exactly this order.
             uint32_t qe_par = 3u;  // bit i: parity to wait for on q_empty(i)
             int slot = 0;
             uint32_t kv_round = 0;
             bool ok = true;
-            auto acquire_slot = [&](int &s) -> bool {
-                s = slot;
-                const bool r = mbar_wait(kv_empty(slot), (kv_round & 1u) ^ 1u, ctl);
-                if (++slot == NS) { slot = 0; ++kv_round; }
-                return r;
-            };
-            // one key or value tile of lane `ln` (stage 1: block tile j; stage 2: chunk)
-            auto load_kv = [&](const Unit &un, const Lane &ln, int j, bool is_v) -> bool {
-                int s;
-                if (!acquire_slot(s)) return false;
-                const uint32_t dst = base + L::OFF_KV + s * L::TILE;
-                int loaded, kvalid, ext;
-                key_extent(p, un, j, kvalid, ext);
-                if (un.kind == UNIT_STAGE1) {
-                    int valid;
-                    s1_tile_rows(p, j, loaded, valid);
-                } else {
-                    loaded = p.npos * p.T;
-                }
-                if (is_v && loaded < ext) {  // rows the PV MMA reads but TMA does not write
-                    zero_rows<NP>(dst, loaded, ext);
-                    fence_proxy_async_smem();
-                }
-                mbar_arrive_expect_tx(kv_full(s), NP * loaded * 128);
-                if (un.kind == UNIT_STAGE1)
-                    s1_load<NP>(p, is_v ? &mv1 : &mk1, dst, kv_full(s), ln.blk, j);
-                else
-                    s2_load<NP>(is_v ? &my2 : &mk2, dst, kv_full(s), p.npos, ln.blk, ln.tile);
-                return true;
-            };
-            // Stage 2 reads Y1 rows that stage-1 lanes of this batch-head (on
-            // any SM) stored with plain stores: wait until all of them have
-            // published (acquire), then order the TMA reads after that.
-            auto wait_stage1 = [&](int bh) -> bool {
-                if (!wait_counter(p.s1_done + bh, p.s1_target, ctl)) return false;
-                fence_proxy_async_global();
-                return true;
-            };
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
+#pragma unroll 1
                 for (int i = 0; i < un.nq && ok; ++i) {
                     ok = mbar_wait(q_empty(i), (qe_par >> i) & 1u, ctl);
                     qe_par ^= 1u << i;
                     if (!ok) break;
+                    const Lane ln = i ? un.ln[1] : un.ln[0];
                     const uint32_t dst = base + L::OFF_Q + i * L::TILE;
                     if (un.kind == UNIT_STAGE1) {
                         int loaded, valid;
-                        s1_tile_rows(p, un.ln[i].tile, loaded, valid);
+                        s1_tile_rows(p, ln.tile, loaded, valid);
                         mbar_arrive_expect_tx(q_full(i), NP * loaded * 128);
-                        s1_load<NP>(p, &mq1, dst, q_full(i), un.ln[i].blk, un.ln[i].tile);
+                        s1_load<NP>(p, &mq1, dst, q_full(i), ln.blk, ln.tile);
                     } else {
                         mbar_arrive_expect_tx(q_full(i), NP * p.npos * p.T * 128);
-                        s2_load<NP>(&mq2, dst, q_full(i), p.npos, un.ln[i].blk, un.ln[i].tile);
+                        s2_load<NP>(&mq2, dst, q_full(i), p.npos, ln.blk, ln.tile);
                     }
                 }
+                const int nkv = un.shared ? 1 : un.nq;
+                int loaded = p.npos * p.T;
+#pragma unroll 1
                 for (int j = 0; j < un.nk && ok; ++j) {
-                    if (un.shared) {
-                        ok = load_kv(un, un.ln[0], j, false) && load_kv(un, un.ln[0], j, true);
-                    } else {
-                        for (int i = 0; i < un.nq && ok; ++i) ok = load_kv(un, un.ln[i], j, false);
-                        if (ok && un.kind == UNIT_STAGE2) ok = wait_stage1(un.ln[0].blk);
-                        for (int i = 0; i < un.nq && ok; ++i) ok = load_kv(un, un.ln[i], j, true);
+                    int kvalid, ext;
+                    key_extent(p, un, j, kvalid, ext);
+                    if (un.kind == UNIT_STAGE1) {
+                        int valid;
+                        s1_tile_rows(p, j, loaded, valid);
+                    }
+#pragma unroll 1
+                    for (int t = 0; t < 2 * nkv && ok; ++t) {
+                        const bool is_v = t >= nkv;
+                        const Lane ln = (t % nkv) ? un.ln[1] : un.ln[0];
+                        // stage 2 reads Y1 rows that stage-1 lanes of this
+                        // batch-head (on any SM) stored with plain stores: wait
+                        // until all have published (acquire), then order the
+                        // TMA reads after that
+                        if (t == nkv && un.kind == UNIT_STAGE2) {
+                            ok = wait_counter(p.s1_done + ln.blk, p.s1_target, ctl);
+                            if (!ok) break;
+                            fence_proxy_async_global();
+                        }
+                        const int s = slot;
+                        ok = mbar_wait(kv_empty(slot), (kv_round & 1u) ^ 1u, ctl);
+                        if (++slot == NS) { slot = 0; ++kv_round; }
+                        if (!ok) break;
+                        const uint32_t dst = base + L::OFF_KV + s * L::TILE;
+                        if (is_v && loaded < ext) {  // rows the PV MMA reads but TMA does not write
+                            zero_rows<NP>(dst, loaded, ext);
+                            fence_proxy_async_smem();
+                        }
+                        mbar_arrive_expect_tx(kv_full(s), NP * loaded * 128);
+                        if (un.kind == UNIT_STAGE1)
+                            s1_load<NP>(p, is_v ? &mv1 : &mk1, dst, kv_full(s), ln.blk, j);
+                        else
+                            s2_load<NP>(is_v ? &my2 : &mk2, dst, kv_full(s), p.npos, ln.blk, ln.tile);
                     }
                 }
             }
@@ -481,12 +495,6 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             int slot = 0;
             uint32_t kv_round = 0;
             bool ok = true;
-            auto acquire_full = [&](int &s) -> bool {
-                s = slot;
-                const bool r = mbar_wait(kv_full(slot), kv_round & 1u, ctl);
-                if (++slot == NS) { slot = 0; ++kv_round; }
-                return r;
-            };
             // Descriptor halves: the low word holds the start address, so
             // every K step below is a single 32-bit add of a constant.
             constexpr uint32_t KM_HI = sdesc_sw128_hi(1024);  // K-major: 8-row groups 1024 B apart
@@ -496,48 +504,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const uint32_t v_lo0 = sdesc_sw128_lo(base + L::OFF_KV, 16384);  // D panels 16 KB apart
             constexpr uint32_t TILE16 = L::TILE >> 4;
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
-            // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D,
-            // N = ext key columns (idesc_s).
-            auto issue_s = [&](int i, int s, uint32_t idesc_s) {
-                const uint32_t a = q_lo0 + i * TILE16;
-                const uint32_t b = kv_lo0 + s * TILE16;
-                const uint32_t d_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
-                mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, idesc_s);
-#pragma unroll
-                for (int k = 1; k < D / 16; ++k) {
-                    const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                    mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, idesc_s);
-                }
-            };
-            // O_i (+)= P_i V: A = P from TMEM (bf16 pairs in the S region),
-            // B = V tile (MN-major: keys x D, D contiguous), K dim = ext keys.
-            auto issue_pv = [&](int i, int s, int ext, uint32_t acc) {
-                const uint32_t b = v_lo0 + s * TILE16;
-                const uint32_t p_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
-                const uint32_t d_tmem = tmem + (i ? L::COL_O1 : L::COL_O0);
-                mma_ts_lh(d_tmem, p_tmem, b, MN_HI, IDESC_O, acc);
-                if (ext == 128) {
-#pragma unroll
-                    for (int k = 1; k < 8; ++k) mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
-                } else {
-                    for (int k = 1; k < ext / 16; ++k)
-                        mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
-                }
-            };
-            auto idesc_for = [](int ext) { return idesc_bf16_f32(128, ext, false, false); };
-            // the first PV of a unit overwrites O_i: the epilogue must be done with it
-            auto wait_p_and_o = [&](int i, bool first) -> bool {
-                if (first) {
-                    if (!mbar_wait(o_free(i), (of_par >> i) & 1u, ctl)) return false;
-                    of_par ^= 1u << i;
-                }
-                if (!mbar_wait(p_full(i), (pf_par >> i) & 1u, ctl)) return false;
-                pf_par ^= 1u << i;
-                tc_fence_after();
-                return true;
-            };
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
+#pragma unroll 1
                 for (int i = 0; i < un.nq && ok; ++i) {
                     ok = mbar_wait(q_full(i), (qf_par >> i) & 1u, ctl);
                     qf_par ^= 1u << i;
@@ -545,71 +514,86 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 if (!ok) break;
                 tc_fence_after();
                 const int nkv = un.shared ? 1 : un.nq;  // K (or V) tiles per key step
-                int kvalid, ext;
-                int sK0, sK1, sV0, sV1;
-                // j = 0: S_i(0)
-                key_extent(p, un, 0, kvalid, ext);
-                if (!acquire_full(sK0)) { ok = false; break; }
-                sK1 = sK0;
-                if (nkv == 2 && !acquire_full(sK1)) { ok = false; break; }
-                tc_fence_after();
-                issue_s(0, sK0, idesc_for(ext));
-                mma_commit(s_full(0));
-                if (un.nq == 2) {
-                    issue_s(1, sK1, idesc_for(ext));
-                    mma_commit(s_full(1));
-                }
-                if (un.nk == 1)
-                    for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
-                mma_commit(kv_empty(sK0));
-                if (nkv == 2) mma_commit(kv_empty(sK1));
-                int prev_ext = ext;
-                for (int j = 1; j < un.nk && ok; ++j) {
-                    key_extent(p, un, j, kvalid, ext);
-                    if (!acquire_full(sV0)) { ok = false; break; }
-                    sV1 = sV0;
-                    if (nkv == 2 && !acquire_full(sV1)) { ok = false; break; }
-                    if (!acquire_full(sK0)) { ok = false; break; }
-                    sK1 = sK0;
-                    if (nkv == 2 && !acquire_full(sK1)) { ok = false; break; }
-                    tc_fence_after();
-                    if (!wait_p_and_o(0, j == 1)) { ok = false; break; }
-                    const uint32_t idesc_s = idesc_for(ext);
-                    issue_pv(0, sV0, prev_ext, j > 1 ? 1u : 0u);
-                    issue_s(0, sK0, idesc_s);
-                    mma_commit(s_full(0));
-                    if (un.nq == 2) {
-                        if (!wait_p_and_o(1, j == 1)) { ok = false; break; }
-                        issue_pv(1, sV1, prev_ext, j > 1 ? 1u : 0u);
-                        issue_s(1, sK1, idesc_s);
-                        mma_commit(s_full(1));
+                int sK0 = 0, sK1 = 0, sV0 = 0, sV1 = 0;
+                int ext = 0, prev_ext = 0;
+                // step j: PV_i(j-1) (for j >= 1) then S_i(j) (for j < nk)
+#pragma unroll 1
+                for (int j = 0; j <= un.nk && ok; ++j) {
+                    const bool has_s = j < un.nk, has_pv = j > 0;
+                    if (has_s) {
+                        int kvalid;
+                        key_extent(p, un, j, kvalid, ext);
                     }
-                    mma_commit(kv_empty(sV0));
-                    mma_commit(kv_empty(sK0));
-                    if (nkv == 2) {
-                        mma_commit(kv_empty(sV1));
-                        mma_commit(kv_empty(sK1));
+                    // take the ring slots in load order: V(j-1) tile(s), K(j) tile(s)
+#pragma unroll 1
+                    for (int t = 0; t < 2 * nkv && ok; ++t) {
+                        const bool is_v = t < nkv;
+                        if ((is_v && !has_pv) || (!is_v && !has_s)) continue;
+                        const int s = slot;
+                        ok = mbar_wait(kv_full(slot), kv_round & 1u, ctl);
+                        if (++slot == NS) { slot = 0; ++kv_round; }
+                        if (is_v) {
+                            if (t == 0) sV0 = sV1 = s; else sV1 = s;
+                        } else {
+                            if (t == nkv) sK0 = sK1 = s; else sK1 = s;
+                        }
+                    }
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t idesc_s = idesc_bf16_f32(128, ext, false, false);
+#pragma unroll 1
+                    for (int i = 0; i < un.nq && ok; ++i) {
+                        if (has_pv) {
+                            // the first PV of a unit overwrites O_i: the epilogue must be done with it
+                            if (j == 1) {
+                                ok = mbar_wait(o_free(i), (of_par >> i) & 1u, ctl);
+                                of_par ^= 1u << i;
+                                if (!ok) break;
+                            }
+                            ok = mbar_wait(p_full(i), (pf_par >> i) & 1u, ctl);
+                            pf_par ^= 1u << i;
+                            if (!ok) break;
+                            tc_fence_after();
+                            // O_i (+)= P_i V: A = P from TMEM (bf16 pairs in the S region),
+                            // B = V tile (MN-major: keys x D), K dim = prev_ext keys
+                            const uint32_t b = v_lo0 + (i ? sV1 : sV0) * TILE16;
+                            const uint32_t p_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
+                            const uint32_t d_tmem = tmem + (i ? L::COL_O1 : L::COL_O0);
+                            mma_ts_lh(d_tmem, p_tmem, b, MN_HI, IDESC_O, j > 1 ? 1u : 0u);
+#pragma unroll 1
+                            for (int k = 1; k < prev_ext / 16; ++k)
+                                mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
+                        }
+                        if (has_s) {
+                            // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D
+                            const uint32_t a = q_lo0 + i * TILE16;
+                            const uint32_t b = kv_lo0 + (i ? sK1 : sK0) * TILE16;
+                            const uint32_t d_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
+                            mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, idesc_s);
+#pragma unroll
+                            for (int k = 1; k < D / 16; ++k) {
+                                const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                                mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, idesc_s);
+                            }
+                            mma_commit(s_full(i));
+                        } else {
+                            mma_commit(o_full(i));
+                        }
+                    }
+                    if (!ok) break;
+                    // release the slots once the MMAs reading them complete
+                    if (has_pv) {
+                        mma_commit(kv_empty(sV0));
+                        if (nkv == 2) mma_commit(kv_empty(sV1));
+                    }
+                    if (has_s) {
+                        mma_commit(kv_empty(sK0));
+                        if (nkv == 2) mma_commit(kv_empty(sK1));
                     }
                     if (j == un.nk - 1)
                         for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
                     prev_ext = ext;
                 }
-                if (!ok) break;
-                // tail: PV_i(nk-1)
-                if (!acquire_full(sV0)) { ok = false; break; }
-                sV1 = sV0;
-                if (nkv == 2 && !acquire_full(sV1)) { ok = false; break; }
-                tc_fence_after();
-                if (!wait_p_and_o(0, un.nk == 1)) { ok = false; break; }
-                issue_pv(0, sV0, prev_ext, un.nk > 1 ? 1u : 0u);
-                mma_commit(o_full(0));
-                if (un.nq == 2) {
-                    if (!wait_p_and_o(1, un.nk == 1)) { ok = false; break; }
-                    issue_pv(1, sV1, prev_ext, un.nk > 1 ? 1u : 0u);
-                    mma_commit(o_full(1));
-                }
-                mma_commit(kv_empty(sV0));
-                if (nkv == 2) mma_commit(kv_empty(sV1));
             }
         }
     } else {
@@ -665,20 +649,13 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
 #pragma unroll
                         for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[c][e]);
                 }
-                if (masked) {  // columns 64h + c
-                    if (un.kind == UNIT_STAGE1) {
+                if (masked) {  // columns 64h + c: validity bits, then -inf where 0
+                    const uint64_t vm = un.kind == UNIT_STAGE1
+                                            ? stage1_valid_bits(kvalid - 64 * h)
+                                            : stage2_valid_bits(p, h, prow, npos_valid);
 #pragma unroll
-                        for (int c = 0; c < 64; ++c)
-                            if (64 * h + c >= kvalid) s[c] = -INFINITY;
-                    } else {
-                        int tc = static_cast<int>(fdiv(64 * h, p.fd_npos)), pc = 64 * h - tc * p.npos;
-#pragma unroll
-                        for (int c = 0; c < 64; ++c) {
-                            const bool valid = (pc == prow) && (tc < p.T) && (pc < npos_valid);
-                            if (!valid) s[c] = -INFINITY;
-                            if (++pc == p.npos) { pc = 0; ++tc; }
-                        }
-                    }
+                    for (int c = 0; c < 64; ++c)
+                        if (!((vm >> c) & 1ull)) s[c] = -INFINITY;
                 }
                 float mx;
                 {

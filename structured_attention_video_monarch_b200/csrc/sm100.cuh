@@ -98,12 +98,9 @@ struct WaitCtl {
     long long limit_cycles;    // give up after this many SM cycles
 };
 
-// Waits until the phase with parity `parity` of the barrier has completed.
-// Returns false (and raises the CTA's abort flag) when the wait gives up.
-// Each try suspends the thread for at most 0.5 ms, so the time limit and the
-// abort flag are checked at least that often.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl &ctl) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait.  (It stays inline: an out-of-line function would
+// have to fit the smallest register budget of the warp roles that call it.)
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtl &ctl) {
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 500000u)) return true;
@@ -114,6 +111,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
             return false;
         }
     }
+}
+
+// Waits until the phase with parity `parity` of the barrier has completed.
+// Returns false (and raises the CTA's abort flag) when the wait gives up.
+// Each try in the slow path suspends the thread for at most 0.5 ms, so the
+// time limit and the abort flag are checked at least that often.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtl &ctl) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, ctl);
 }
 
 // Waits until *counter >= target (acquire at GPU scope), sleeping between
