@@ -126,6 +126,40 @@ int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void 
                               int factorisation, int tile_h, int tile_w, int dtype,
                               void *stream, void **events, int nevents, int *nlaunch);
 
+/* Largest B*heads monarch_attn_fwd_noalloc accepts (size of its static
+ * counter array: one 32-bit word per batch-head, 16 KB per device). */
+#define MONARCH_NOALLOC_MAX_BH 4096
+
+/*
+ * monarch_attn_fwd_noalloc -- monarch_attn_fwd for bf16 that allocates no
+ * device memory.  No counterpart in the pages: it exists for callers that
+ * cannot allocate once running (a real-time generation loop, where
+ * monarch_attn_fwd's first call on a new stream would cudaMalloc its counter
+ * buffer and growing it would drain the stream and cudaFree, which waits for
+ * the whole device; or a host whose device memory is all held by its own
+ * pool).
+ *
+ * Arguments, layout, ownership and status codes are those of
+ * monarch_attn_fwd with dtype = MONARCH_DTYPE_BF16.  Scratch: the per-batch-
+ * head completion counters live in one static device array per device of
+ * MONARCH_NOALLOC_MAX_BH words; B*heads above that returns
+ * MONARCH_ERR_UNSUPPORTED before anything is queued.  Those counters must be
+ * zero when the kernel starts; every call zeroes them with a cudaMemsetAsync
+ * on `stream` ahead of its launch.  The first call on each device does a
+ * one-time set-up on the host (the array's address, the kernel's shared-
+ * memory attribute, the tensor-map encoder); make that first call before
+ * beginning any stream capture.
+ *
+ * Calls race when they overlap: every call on a device uses the same
+ * counters, so two calls whose work can run at the same time (on different
+ * streams, or from different host threads without ordering) may let stage 2
+ * read unfinished stage-1 results, or time out.  Queue such calls on one
+ * stream, or order them with events.
+ */
+int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *out,
+                             int B, int heads, int T, int H, int W, int d,
+                             int factorisation, int tile_h, int tile_w, void *stream);
+
 /* Human-readable text of a status code; never NULL, owned by the library. */
 const char *monarch_attn_strerror(int status);
 

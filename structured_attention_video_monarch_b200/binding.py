@@ -58,6 +58,8 @@ def load_library(path: str | None = None):
     lib.monarch_attn_device_status.restype = i
     lib.monarch_attn_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.monarch_attn_selftest_timeout.restype = i
+    lib.monarch_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp] + [i] * 9 + [vp]
+    lib.monarch_attn_fwd_noalloc.restype = i
     lib.monarch_attn_version.argtypes = []
     lib.monarch_attn_version.restype = i
     if path == _build.LIB:
@@ -111,6 +113,29 @@ def monarch_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, T: int, 
         int(factorisation), int(tile_h), int(tile_w), _dtype_code(q), _stream_ptr(stream))
     if st != 0:
         raise MonarchError(st, "monarch_attn_fwd")
+    return out
+
+
+def monarch_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                             T: int, H: int, W: int, factorisation: int = FACT_FRAME, tile_h: int = 0,
+                             tile_w: int = 0, stream=None) -> torch.Tensor:
+    """bf16 monarch_attn_fwd through the entry point that allocates no device
+    memory (static per-device counters; calls on one device must not overlap).
+    ``out`` is required, since this path allocates nothing.
+    """
+    ts = (q, k, v, out)
+    if not all(t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16 for t in ts):
+        raise ValueError("q, k, v, out must be contiguous bf16 CUDA tensors")
+    if q.dim() != 4 or any(t.shape != q.shape for t in ts):
+        raise ValueError("q, k, v, out must share one [B, heads, N, d] shape")
+    B, heads, N, d = q.shape
+    if N != T * H * W:
+        raise ValueError(f"N={N} does not equal T*H*W={T * H * W}")
+    st = load_library().monarch_attn_fwd_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, heads, T, H, W, d,
+        int(factorisation), int(tile_h), int(tile_w), _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_noalloc")
     return out
 
 

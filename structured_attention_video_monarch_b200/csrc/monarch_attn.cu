@@ -108,6 +108,27 @@ int counters_for(cudaStream_t stream, size_t n, unsigned **out) {
     return MONARCH_OK;
 }
 
+// Completion counters for monarch_attn_fwd_noalloc: a file-scope device array
+// (4096 words, 16 KB) in place of the per-stream cudaMalloc buffer above, its
+// address looked up once per device.  One array per device means calls of
+// that entry point on one device must not overlap in time.
+static __device__ __align__(256) unsigned g_noalloc_counters[MONARCH_NOALLOC_MAX_BH];
+unsigned *g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_counters(unsigned **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_counters) != cudaSuccess || ptr == nullptr)
+            return MONARCH_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<unsigned *>(ptr);
+    }
+    *out = g_noalloc_ptr[dev];
+    return MONARCH_OK;
+}
+
 bool env_debug() {
     const char *e = std::getenv("MONARCH_ATTN_DEBUG");
     return e && e[0] == '1';
@@ -215,7 +236,7 @@ struct LaunchEvents {
 
 template <int D>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
-              cudaStream_t stream, LaunchEvents &lev) {
+              cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
@@ -300,8 +321,8 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     // into out; stage-2 units overwrite it in place with P^T B2 P Y1 once the
     // stage-1 lanes of their batch-head have published (per-batch-head
     // counters, zeroed for every call).
-    unsigned *counters = nullptr;
-    if ((st = counters_for(stream, static_cast<size_t>(bh), &counters))) return st;
+    unsigned *counters = fixed_counters;
+    if (!counters && (st = counters_for(stream, static_cast<size_t>(bh), &counters))) return st;
     p.s1_done = counters;
     if (cudaMemsetAsync(counters, 0, static_cast<size_t>(bh) * sizeof(unsigned), stream) != cudaSuccess)
         return MONARCH_ERR_CUDA;
@@ -453,6 +474,31 @@ int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, voi
     if (cudaMemcpyAsync(h_out, d_out, bytes, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
         return MONARCH_ERR_CUDA;
     if (cudaStreamSynchronize(cs) != cudaSuccess) return MONARCH_ERR_CUDA;
+    return MONARCH_OK;
+}
+
+// Same operator as monarch_attn_fwd for bf16, with the completion counters in
+// the static device array instead of a cudaMalloc'd per-stream buffer.  It
+// serves callers that cannot allocate device memory once running: a real-time
+// generation loop, where the first call on a stream (or a larger batch) would
+// otherwise cudaMalloc, and a reallocation drains the stream and calls
+// cudaFree, which waits for the whole device; and hosts whose device memory
+// is all held by their own pool, where a cudaMalloc can fail mid-run.
+int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *out, int B, int heads,
+                             int T, int H, int W, int d, int factorisation, int tile_h, int tile_w,
+                             void *stream) {
+    Shape s{B, heads, T, H, W, d, factorisation, tile_h, tile_w, MONARCH_DTYPE_BF16, 0, 0};
+    int st = validate(q, k, v, out, s);
+    if (st) return st;
+    if (static_cast<long long>(B) * heads > MONARCH_NOALLOC_MAX_BH) return MONARCH_ERR_UNSUPPORTED;
+    unsigned *counters = nullptr;
+    if ((st = noalloc_counters(&counters))) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    LaunchEvents lev;
+    st = d == 128 ? launch_tc<128>(q, k, v, out, s, cs, lev, counters)
+                  : launch_tc<64>(q, k, v, out, s, cs, lev, counters);
+    if (st) return st;
+    if (env_debug()) return read_status(cs, 0);
     return MONARCH_OK;
 }
 
