@@ -20,6 +20,7 @@ a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -214,6 +215,38 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ our arm
 
+def kernel_sources_sha256() -> str:
+    """Hash of the CUDA sources the dominant kernel is built from."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "structured_attention_video_monarch_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    or None when there is none or the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"monarch_tc_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            key, sep, val = line.strip().partition(":")
+            if sep and key in ("kernel_sources_sha256", "traffic_bytes_per_launch"):
+                fields[key] = val.strip()
+    if fields.get("kernel_sources_sha256") != kernel_sources_sha256():
+        return None
+    try:
+        return float(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -301,7 +334,8 @@ def run_ours(args):
     io_bytes = wl.io_bytes
     roofline = {
         "bound": "tensor", "achieved": k_tflops, "peak": peak, "unit": "TFLOP/s",
-        "frac": k_tflops / peak, "traffic": args.traffic,
+        "frac": k_tflops / peak,
+        "traffic": args.traffic if args.traffic is not None else captured_traffic(wl.name),
         "kernel": "monarch_tc_kernel<128> (both stages, one persistent launch)",
         "peak_source": f"{peak_src} bf16_tflops (burst)",
         "frac_of_sustained": k_tflops / peak_sus,
@@ -389,7 +423,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,
-                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+                    help="dram bytes per launch of the dominant kernel from an ncu capture "
+                         "(default: the committed profile summary, if the kernel is unchanged)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
