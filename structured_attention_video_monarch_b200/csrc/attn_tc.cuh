@@ -560,9 +560,12 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                             const uint32_t p_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
                             const uint32_t d_tmem = tmem + (i ? L::COL_O1 : L::COL_O0);
                             mma_ts_lh(d_tmem, p_tmem, b, MN_HI, IDESC_O, j > 1 ? 1u : 0u);
-#pragma unroll 1
-                            for (int k = 1; k < prev_ext / 16; ++k)
-                                mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
+                            // unrolled with constant offsets: the MMA issuer is latency-bound,
+                            // and a counted loop adds its own chain to every instruction
+                            const int npv = prev_ext >> 4;
+#pragma unroll
+                            for (int k = 1; k < 8; ++k)
+                                if (k < npv) mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
                         }
                         if (has_s) {
                             // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D
