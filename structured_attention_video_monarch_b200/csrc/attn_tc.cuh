@@ -28,19 +28,20 @@
 //                      output columns [0, D/2) / [D/2, D)            104 regs
 //   warps 4-7, 12-15   the same for lane 1                            104 regs
 //   warp  16           TMA producer (Q tiles, K/V ring)                64 regs
-//   warp  17           TMEM allocator and single-thread tcgen05.mma issuer
-//   warp  18           publishes finished stage-1 lanes to stage-2 units
-//   warp  19           idle
+//   warp  17           TMEM allocator; issues the S = Q K^T MMAs (shared-memory operands)
+//   warp  18           issues the O += P V MMAs (P from tensor memory)
+//   warp  19           publishes finished stage-1 lanes to stage-2 units
 // (4*128*104 + 128*64 = 61440 = 640 threads x 96, the launch allocation.)
 // Splitting each row over two warps puts two warps of the same lane on every
 // SM sub-partition, so the exp/pack work of one tile is spread over twice the
 // warps; the halves exchange their row maxima through shared memory.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0, O1 after them.
 // P (bf16) overwrites the first 64 columns of its S region and feeds the PV
-// MMA straight from TMEM.  The MMA issue order per key tile j is
-//   PV0(j-1), S0(j), PV1(j-1), S1(j)
-// so one lane's softmax overlaps the other lane's MMAs; tcgen05.mma ops from
-// one thread execute in order, which makes S_i(j+1) safe after PV_i(j).
+// MMA straight from TMEM.  Per lane i and key tile j the chain is
+//   S_i(j) -> softmax_i(j) writes P_i(j) -> PV_i(j) -> S_i(j+1) -> ...
+// with S_i(j+1) issued only once PV_i(j) has completed (it overwrites P_i(j));
+// the two lanes' chains interleave on the tensor pipe, so one lane's softmax
+// overlaps the other lane's MMAs.
 #pragma once
 
 #include "sm100.cuh"
@@ -260,8 +261,8 @@ struct TcLayout {
     static constexpr int OFF_KV = OFF_Q + 2 * TILE;
     static constexpr int OFF_BAR = OFF_KV + NS * TILE;
     // barriers: q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2]
-    //           o_full[2] o_free[2] y_done[2] y_free[2]
-    static constexpr int NBAR = 16 + 2 * NS;
+    //           o_full[2] o_free[2] y_done[2] y_free[2] pv_done[2]
+    static constexpr int NBAR = 18 + 2 * NS;
     // exchange of per-row values (partial maxima, partial sums) between the two
     // column halves of a lane: [2 lanes][2 halves][128 rows] fp32
     static constexpr int OFF_X = OFF_BAR + NBAR * 8;
@@ -355,6 +356,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     auto o_free = [&](int i) { return bar0 + 8u * (10 + 2 * NS + i); };
     auto y_done = [&](int i) { return bar0 + 8u * (12 + 2 * NS + i); };
     auto y_free = [&](int i) { return bar0 + 8u * (14 + 2 * NS + i); };
+    auto pv_done = [&](int i) { return bar0 + 8u * (16 + 2 * NS + i); };
     float *x_buf = reinterpret_cast<float *>(base_ptr + L::OFF_X);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
@@ -375,6 +377,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             mbar_init(o_free(i), 256);
             mbar_init(y_done(i), 256);
             mbar_init(y_free(i), 1);
+            mbar_init(pv_done(i), 1);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full(s), 1);
@@ -397,7 +400,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
 
     if (wg == 4) {
         setmaxnreg_dec64();
-        if (warp == 18 && lane == 0) {
+        if (warp == 19 && lane == 0) {
             // ------------------------------------------------------ Y1 publisher
             // Once the 256 threads of a stage-1 lane have stored its Y1 rows
             // (y_done), make them visible at GPU scope and count the lane for
@@ -487,11 +490,24 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     }
                 }
             }
-        } else if (warp == 17 && lane == 0) {
-            // -------------------------------------------------------- MMA issuer
-            uint32_t qf_par = 0u;  // bit i: parity to wait for on q_full(i)
-            uint32_t pf_par = 0u;  // bit i: parity to wait for on p_full(i)
-            uint32_t of_par = 3u;  // bit i: parity to wait for on o_free(i)
+        } else if ((warp == 17 || warp == 18) && lane == 0) {
+            // -------------------------------------------------------- MMA issuers
+            // Warp 17 issues every S = Q K^T MMA (both operands in shared
+            // memory), warp 18 every O += P V MMA (P in tensor memory).  One
+            // thread cannot issue a lane pair's 32 MMAs per key step plus its
+            // barrier traffic as fast as the tensor pipe runs them; two threads
+            // can, as long as one of them issues all the TMEM-operand MMAs (the
+            // pipe serialises those when two threads interleave them).
+            // S_i of a key tile overwrites the S/P region that PV_i of the
+            // previous tile reads, so the S issuer waits for that PV's
+            // completion (pv_done, committed after every PV).  Both issuers walk
+            // the K/V ring in load order; each waits for and releases only its
+            // own tiles (K tiles: S issuer, V tiles: PV issuer).
+            const bool s_role = warp == 17;
+            uint32_t qf_par = 0u;   // bit i: parity to wait for on q_full(i)
+            uint32_t pd_par = 3u;   // bit i: parity to wait for on pv_done(i) (the first S passes)
+            uint32_t pf_par = 0u;   // bit i: parity to wait for on p_full(i)
+            uint32_t of_par = 3u;   // bit i: parity to wait for on o_free(i)
             int slot = 0;
             uint32_t kv_round = 0;
             bool ok = true;
@@ -506,46 +522,65 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
+                if (s_role) {
 #pragma unroll 1
-                for (int i = 0; i < un.nq && ok; ++i) {
-                    ok = mbar_wait(q_full(i), (qf_par >> i) & 1u, ctl);
-                    qf_par ^= 1u << i;
-                }
-                if (!ok) break;
-                tc_fence_after();
-                const int nkv = un.shared ? 1 : un.nq;  // K (or V) tiles per key step
-                int sK0 = 0, sK1 = 0, sV0 = 0, sV1 = 0;
-                int ext = 0, prev_ext = 0;
-                // step j: PV_i(j-1) (for j >= 1) then S_i(j) (for j < nk)
-#pragma unroll 1
-                for (int j = 0; j <= un.nk && ok; ++j) {
-                    const bool has_s = j < un.nk, has_pv = j > 0;
-                    if (has_s) {
-                        int kvalid;
-                        key_extent(p, un, j, kvalid, ext);
+                    for (int i = 0; i < un.nq && ok; ++i) {
+                        ok = mbar_wait(q_full(i), (qf_par >> i) & 1u, ctl);
+                        qf_par ^= 1u << i;
                     }
-                    // take the ring slots in load order: V(j-1) tile(s), K(j) tile(s)
+                    if (!ok) break;
+                }
+                const int nkv = un.shared ? 1 : un.nq;  // K (or V) tiles per key step
+#pragma unroll 1
+                for (int j = 0; j < un.nk && ok; ++j) {
+                    int kvalid, ext;
+                    key_extent(p, un, j, kvalid, ext);
+                    // ring slots in load order: K(j) tile(s), then V(j) tile(s);
+                    // wait for this role's own ones
+                    int s0 = 0, s1 = 0;
 #pragma unroll 1
                     for (int t = 0; t < 2 * nkv && ok; ++t) {
-                        const bool is_v = t < nkv;
-                        if ((is_v && !has_pv) || (!is_v && !has_s)) continue;
+                        const bool mine = (t < nkv) == s_role;
                         const int s = slot;
-                        ok = mbar_wait(kv_full(slot), kv_round & 1u, ctl);
+                        if (mine) ok = mbar_wait(kv_full(slot), kv_round & 1u, ctl);
                         if (++slot == NS) { slot = 0; ++kv_round; }
-                        if (is_v) {
-                            if (t == 0) sV0 = sV1 = s; else sV1 = s;
-                        } else {
-                            if (t == nkv) sK0 = sK1 = s; else sK1 = s;
+                        if (mine) {
+                            if ((t % nkv) == 0) s0 = s1 = s; else s1 = s;
                         }
                     }
                     if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t idesc_s = idesc_bf16_f32(128, ext, false, false);
+                    if (s_role) {
+                        const uint32_t idesc_s = idesc_bf16_f32(128, ext, false, false);
 #pragma unroll 1
-                    for (int i = 0; i < un.nq && ok; ++i) {
-                        if (has_pv) {
+                        for (int i = 0; i < un.nq && ok; ++i) {
+                            // the PV that last read this lane's S/P region has completed
+                            ok = mbar_wait(pv_done(i), (pd_par >> i) & 1u, ctl);
+                            pd_par ^= 1u << i;
+                            if (!ok) break;
+                            tc_fence_after();
+                            // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D
+                            const uint32_t a = q_lo0 + i * TILE16;
+                            const uint32_t b = kv_lo0 + (i ? s1 : s0) * TILE16;
+                            const uint32_t d_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
+                            mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, idesc_s);
+#pragma unroll
+                            for (int k = 1; k < D / 16; ++k) {
+                                const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                                mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, idesc_s);
+                            }
+                            mma_commit(s_full(i));
+                        }
+                        if (!ok) break;
+                        mma_commit(kv_empty(s0));
+                        if (nkv == 2) mma_commit(kv_empty(s1));
+                        if (j == un.nk - 1)
+                            for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
+                    } else {
+                        const int npv = ext >> 4;
+#pragma unroll 1
+                        for (int i = 0; i < un.nq && ok; ++i) {
                             // the first PV of a unit overwrites O_i: the epilogue must be done with it
-                            if (j == 1) {
+                            if (j == 0) {
                                 ok = mbar_wait(o_free(i), (of_par >> i) & 1u, ctl);
                                 of_par ^= 1u << i;
                                 if (!ok) break;
@@ -555,47 +590,22 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                             if (!ok) break;
                             tc_fence_after();
                             // O_i (+)= P_i V: A = P from TMEM (bf16 pairs in the S region),
-                            // B = V tile (MN-major: keys x D), K dim = prev_ext keys
-                            const uint32_t b = v_lo0 + (i ? sV1 : sV0) * TILE16;
+                            // B = V tile (MN-major: keys x D), K dim = ext keys; unrolled
+                            // with constant offsets (the issuing thread is latency-bound)
+                            const uint32_t b = v_lo0 + (i ? s1 : s0) * TILE16;
                             const uint32_t p_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
                             const uint32_t d_tmem = tmem + (i ? L::COL_O1 : L::COL_O0);
-                            mma_ts_lh(d_tmem, p_tmem, b, MN_HI, IDESC_O, j > 1 ? 1u : 0u);
-                            // unrolled with constant offsets: the MMA issuer is latency-bound,
-                            // and a counted loop adds its own chain to every instruction
-                            const int npv = prev_ext >> 4;
+                            mma_ts_lh(d_tmem, p_tmem, b, MN_HI, IDESC_O, j > 0 ? 1u : 0u);
 #pragma unroll
                             for (int k = 1; k < 8; ++k)
                                 if (k < npv) mma_ts_lh(d_tmem, p_tmem + k * 8, b + k * 128, MN_HI, IDESC_O, 1u);
+                            mma_commit(pv_done(i));
+                            if (j == un.nk - 1) mma_commit(o_full(i));
                         }
-                        if (has_s) {
-                            // S_i = Q_i K^T: A = Q tile (K-major), B = K tile (K-major), K dim = D
-                            const uint32_t a = q_lo0 + i * TILE16;
-                            const uint32_t b = kv_lo0 + (i ? sK1 : sK0) * TILE16;
-                            const uint32_t d_tmem = tmem + (i ? L::COL_S1 : L::COL_S0);
-                            mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, idesc_s);
-#pragma unroll
-                            for (int k = 1; k < D / 16; ++k) {
-                                const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                                mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, idesc_s);
-                            }
-                            mma_commit(s_full(i));
-                        } else {
-                            mma_commit(o_full(i));
-                        }
+                        if (!ok) break;
+                        mma_commit(kv_empty(s0));
+                        if (nkv == 2) mma_commit(kv_empty(s1));
                     }
-                    if (!ok) break;
-                    // release the slots once the MMAs reading them complete
-                    if (has_pv) {
-                        mma_commit(kv_empty(sV0));
-                        if (nkv == 2) mma_commit(kv_empty(sV1));
-                    }
-                    if (has_s) {
-                        mma_commit(kv_empty(sK0));
-                        if (nkv == 2) mma_commit(kv_empty(sK1));
-                    }
-                    if (j == un.nk - 1)
-                        for (int i = 0; i < un.nq; ++i) mma_commit(q_empty(i));
-                    prev_ext = ext;
                 }
             }
         }
@@ -710,7 +720,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     l_half += (a0 + a1) + (b0 + b1);
                 }
                 // O from earlier key tiles is complete here (S_i(j) was issued
-                // after PV_i(j-1)); rescale this half's columns before PV_i(j)
+                // after PV_i(j-1) completed); rescale this half's columns before PV_i(j)
                 if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
                     for (int c = 0; c < D / 64; ++c) {
