@@ -79,6 +79,7 @@ struct TcParams {
     long long timeout_cycles;
     unsigned *status;
     void *out;                      // bf16 output (epilogue stores)
+    int out_v8;                     // out is 32-byte aligned: 32-byte epilogue stores
 };
 
 struct Lane {
@@ -750,26 +751,27 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             if (!mbar_wait(o_full(li), of_par, ctl)) { ok = false; break; }
             of_par ^= 1u;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < D / 64; ++c) {
-                uint32_t r[32];
-                tmem_ld32(lane_base + col_o + h * (D / 2) + 32 * c, r);
-                tmem_wait_ld();
-                if (tok >= 0) {
+            // read this half's O columns, then release O at once: the next
+            // unit's first PV may overwrite it while these rows are stored
+            uint32_t r[D / 2];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]) * inv_l, __uint_as_float(r[8 * q + 1]) * inv_l);
-                        w.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]) * inv_l, __uint_as_float(r[8 * q + 3]) * inv_l);
-                        w.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]) * inv_l, __uint_as_float(r[8 * q + 5]) * inv_l);
-                        w.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]) * inv_l, __uint_as_float(r[8 * q + 7]) * inv_l);
-                        dst[4 * c + q] = w;
-                    }
-                }
-            }
-            // O_i has been read: the next unit may overwrite it
+            for (int c = 0; c < D / 64; ++c) tmem_ld32(lane_base + col_o + h * (D / 2) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+            tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(o_free(li));
+            if (tok >= 0) {
+                uint32_t w[D / 4];
+#pragma unroll
+                for (int e = 0; e < D / 4; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+                if (p.out_v8) {  // 32-byte stores: each fills a whole sector
+#pragma unroll
+                    for (int q = 0; q < D / 32; ++q) st_global_v8(dst + 2 * q, w + 8 * q);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < D / 16; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                }
+            }
             if (un.kind == UNIT_STAGE1) {
                 // Y1 rows stored: hand them to the publisher (one-slot
                 // handshake, so y_done never runs a phase ahead of it)

@@ -306,6 +306,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.d)));
     p.timeout_cycles = env_timeout_cycles();
     p.out = out;
+    p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
     unsigned *status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_device_status) != cudaSuccess)
         return MONARCH_ERR_CUDA;
