@@ -623,14 +623,16 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         const float sl2 = p.scale_log2;
         uint32_t sf_par = 0u, of_par = 0u, yf_par = 1u;
         bool ok = true;
-        // value of this row in the other column half of the lane: barrier
-        // 3+li makes sure the other half has read the previous value before
-        // it is overwritten, barrier 1+li publishes the new one
+        // value of this row in the other column half of the lane.  Only the
+        // two warps holding the same 32 rows (one per half) take part: named
+        // barrier `pair_bar` (64 threads) makes sure the other half has read
+        // the previous value before it is overwritten, then publishes the new one.
         float *xb = x_buf + li * 2 * 128;
+        const uint32_t pair_bar = 1u + static_cast<uint32_t>(li * 4 + (warp & 3));
         auto exchange = [&](float v) -> float {
-            named_barrier_sync(3 + li, 256);
+            named_barrier_sync(pair_bar, 64);
             xb[h * 128 + row] = v;
-            named_barrier_sync(1 + li, 256);
+            named_barrier_sync(pair_bar, 64);
             return xb[(1 - h) * 128 + row];
         };
         for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
@@ -685,14 +687,14 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
                 }
                 // The row max spans both halves.  Tile 0 exchanges it; later
-                // tiles keep the running max unless some row of the lane grew
-                // by more than 2^8 (one OR-barrier tells), and only then
+                // tiles keep the running max unless some row of the warp pair
+                // grew by more than 2^8 (one OR-barrier tells), and only then
                 // exchange partial maxima and rescale O.
                 bool rescale = false;
                 float alpha = 1.f;
                 if (j == 0) {
                     m_run = fmaxf(mx, exchange(mx));
-                } else if (named_barrier_or(5 + li, 256, (mx - m_run) * sl2 > 8.f)) {
+                } else if (named_barrier_or(pair_bar, 64, (mx - m_run) * sl2 > 8.f)) {
                     mx = fmaxf(mx, exchange(mx));
                     if ((mx - m_run) * sl2 > 8.f) {
                         alpha = fast_exp2((m_run - mx) * sl2);
