@@ -762,16 +762,20 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             tc_fence_before();
             mbar_arrive(o_free(li));
             if (tok >= 0) {
-                uint32_t w[D / 4];
+                // pack and store 16 columns at a time (fewer live registers)
 #pragma unroll
-                for (int e = 0; e < D / 4; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (p.out_v8) {  // 32-byte stores: each fills a whole sector
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t w[8];
 #pragma unroll
-                    for (int q = 0; q < D / 32; ++q) st_global_v8(dst + 2 * q, w + 8 * q);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < D / 16; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                    for (int e = 0; e < 8; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(r[16 * q + 2 * e]) * inv_l,
+                                           __uint_as_float(r[16 * q + 2 * e + 1]) * inv_l);
+                    if (p.out_v8) {  // 32-byte stores: each fills a whole sector
+                        st_global_v8(dst + 2 * q, w);
+                    } else {
+                        dst[2 * q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        dst[2 * q + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
                 }
             }
             if (un.kind == UNIT_STAGE1) {
