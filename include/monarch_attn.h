@@ -19,7 +19,7 @@
  * with the stage-1 outputs as values.
  *
  * Every entry point is plain C: raw pointers, ints, and a cudaStream_t passed
- * as void*.  The bf16 path keeps a small per-(device, stream) buffer of
+ * as void*.  The bf16 / fp16 path keeps a small per-(device, stream) buffer of
  * completion counters (one 32-bit word per batch-head, at least 4 KB),
  * allocated with cudaMalloc by the first call on that stream and reused
  * afterwards; a call needing more drains the stream and reallocates it.
@@ -44,7 +44,8 @@ typedef enum {
 /* Element type of q, k, v and out. */
 typedef enum {
     MONARCH_DTYPE_F32 = 0,  /* fp32 in and out; exact path on CUDA cores, fp32 accumulation */
-    MONARCH_DTYPE_BF16 = 1  /* bf16 in and out; tcgen05 tensor cores, fp32 accumulation and softmax */
+    MONARCH_DTYPE_BF16 = 1, /* bf16 in and out; tcgen05 tensor cores, fp32 accumulation and softmax */
+    MONARCH_DTYPE_F16 = 2   /* fp16 in and out; as bf16 (P and Y1 held in fp16) */
 } monarch_dtype_t;
 
 /* Choice of stage-1 blocks (block alignment: every video axis lies inside one
@@ -71,7 +72,7 @@ typedef enum {
  *   factorisation  MONARCH_FACT_FRAME or MONARCH_FACT_TILED.
  *   tile_h, tile_w tile size for MONARCH_FACT_TILED; must divide H and W
  *             respectively.  Ignored for MONARCH_FACT_FRAME.
- *   dtype     MONARCH_DTYPE_BF16 or MONARCH_DTYPE_F32.
+ *   dtype     MONARCH_DTYPE_BF16, MONARCH_DTYPE_F16 or MONARCH_DTYPE_F32.
  *   stream    cudaStream_t (NULL = legacy default stream) the work is queued on.
  *
  * Limits of this build (MONARCH_ERR_UNSUPPORTED otherwise): T <= 128;
@@ -117,8 +118,8 @@ int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, voi
  * `events` holds `nevents` cudaEvent_t handles created by the caller
  * (entries beyond what the call needs are left untouched; NULL entries are
  * skipped).  *nlaunch (if not NULL) receives the number of kernel launches
- * the call queued: 1 for bf16 (both stages in one persistent kernel), 2 for
- * fp32 (stage 1, then stage 2).  Same arguments, rules and status codes as
+ * the call queued: 1 for bf16 and fp16 (both stages in one persistent
+ * kernel), 2 for fp32 (stage 1, then stage 2).  Same arguments, rules and status codes as
  * monarch_attn_fwd otherwise.
  */
 int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void *out,

@@ -18,6 +18,7 @@ FACT_FRAME = 0
 FACT_TILED = 1
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
+DTYPE_F16 = 2
 
 STATUS_NAMES = {0: "MONARCH_OK", 1: "MONARCH_ERR_INVALID_ARG", 2: "MONARCH_ERR_UNSUPPORTED",
                 3: "MONARCH_ERR_LAUNCH", 4: "MONARCH_ERR_TIMEOUT", 5: "MONARCH_ERR_CUDA"}
@@ -74,9 +75,11 @@ def strerror(status: int) -> str:
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return DTYPE_BF16
+    if t.dtype == torch.float16:
+        return DTYPE_F16
     if t.dtype == torch.float32:
         return DTYPE_F32
-    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16 or float32")
+    raise TypeError(f"unsupported dtype {t.dtype}; expected bfloat16, float16 or float32")
 
 
 def _stream_ptr(stream) -> int:

@@ -1,4 +1,4 @@
-// attn_tc.cuh -- bf16 Monarch attention stages on tcgen05 tensor cores.
+// attn_tc.cuh -- bf16 / fp16 Monarch attention stages on tcgen05 tensor cores.
 //
 // One persistent kernel runs "units" of block-diagonal softmax attention
 // (MonarchRT: Efficient Attention for Real-Time Video Generation,
@@ -78,7 +78,7 @@ struct TcParams {
     float scale_log2;               // d^-1/2 * log2(e)
     long long timeout_cycles;
     unsigned *status;
-    void *out;                      // bf16 output (epilogue stores)
+    void *out;                      // 16-bit output (epilogue stores)
     int out_v8;                     // out is 32-byte aligned: 32-byte epilogue stores
 };
 
@@ -307,7 +307,16 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
 // bf16 pairs, and accumulate P into two packed fp32 partial sums (even and
 // odd pairs, so the additions form two independent chains).
-template <int C>
+// Packs two fp32 values into the kernel's 16-bit input format (fp16 or bf16).
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_in(float lo, float hi) {
+    if constexpr (F16)
+        return pack_f16x2(lo, hi);
+    else
+        return pack_bf16x2(lo, hi);
+}
+
+template <int C, bool F16>
 __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t scale, uint64_t off,
                                               uint32_t (&pk)[16], uint64_t &acc0, uint64_t &acc1) {
 #pragma unroll
@@ -317,7 +326,7 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t sca
         unpack_f32x2(x, x0, x1);
         a = fast_exp2(x0);
         b = fast_exp2(x1);
-        const uint32_t w = pack_bf16x2(a, b);
+        const uint32_t w = pack_in<F16>(a, b);
         pk[e] = w;
         // the denominator sums the bf16-rounded weights the PV MMA uses
         const uint64_t r = pack_f32x2(a, b);  // softmax denominator
@@ -328,7 +337,7 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t sca
     }
 }
 
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(640, 1)
 monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant__ CUtensorMap mk1,
                   const __grid_constant__ CUtensorMap mv1, const __grid_constant__ CUtensorMap mq2,
@@ -520,7 +529,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const uint32_t kv_lo0 = sdesc_sw128_lo(base + L::OFF_KV, 16);
             const uint32_t v_lo0 = sdesc_sw128_lo(base + L::OFF_KV, 16384);  // D panels 16 KB apart
             constexpr uint32_t TILE16 = L::TILE >> 4;
-            constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+            constexpr uint32_t IDESC_O = F16 ? idesc_f16_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 const Unit un = decode_unit(p, u);
                 if (s_role) {
@@ -551,7 +560,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     }
                     if (!ok) break;
                     if (s_role) {
-                        const uint32_t idesc_s = idesc_bf16_f32(128, ext, false, false);
+                        const uint32_t idesc_s = F16 ? idesc_f16_f32(128, ext, false, false) : idesc_bf16_f32(128, ext, false, false);
 #pragma unroll 1
                         for (int i = 0; i < un.nq && ok; ++i) {
                             // the PV that last read this lane's S/P region has completed
@@ -711,9 +720,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 // packed columns [32h, 32h+32) of the lane's S region
                 {
                     uint32_t pk[16];
-                    softmax_chunk<0>(s, scale2, off2, pk, acc0, acc1);  // masked: 2^-inf = 0
+                    softmax_chunk<0, F16>(s, scale2, off2, pk, acc0, acc1);  // masked: 2^-inf = 0
                     tmem_st16(lane_base + col_s + 32 * h, pk);
-                    softmax_chunk<1>(s, scale2, off2, pk, acc0, acc1);
+                    softmax_chunk<1, F16>(s, scale2, off2, pk, acc0, acc1);
                     tmem_st16(lane_base + col_s + 32 * h + 16, pk);
                 }
                 {
@@ -768,8 +777,8 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                     uint32_t w[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(r[16 * q + 2 * e]) * inv_l,
-                                           __uint_as_float(r[16 * q + 2 * e + 1]) * inv_l);
+                        w[e] = pack_in<F16>(__uint_as_float(r[16 * q + 2 * e]) * inv_l,
+                                            __uint_as_float(r[16 * q + 2 * e + 1]) * inv_l);
                     if (p.out_v8) {  // 32-byte stores: each fills a whole sector
                         st_global_v8(dst + 2 * q, w);
                     } else {

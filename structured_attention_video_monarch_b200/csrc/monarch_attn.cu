@@ -28,7 +28,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     bool init = false;
     int sms = 0;
-    bool tc_attr[2] = {false, false};
+    bool tc_attr[4] = {false, false, false, false};  // [fp16][d == 128]
     bool f32_attr[2] = {false, false};
 };
 
@@ -157,7 +157,8 @@ int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
     if (!q || !k || !v || !out) return MONARCH_ERR_INVALID_ARG;
     if (s.B < 1 || s.heads < 1 || s.T < 1 || s.H < 1 || s.W < 1) return MONARCH_ERR_INVALID_ARG;
     if (s.d != 64 && s.d != 128) return MONARCH_ERR_INVALID_ARG;
-    if (s.dtype != MONARCH_DTYPE_F32 && s.dtype != MONARCH_DTYPE_BF16) return MONARCH_ERR_INVALID_ARG;
+    if (s.dtype != MONARCH_DTYPE_F32 && s.dtype != MONARCH_DTYPE_BF16 && s.dtype != MONARCH_DTYPE_F16)
+        return MONARCH_ERR_INVALID_ARG;
     if (s.fact != MONARCH_FACT_FRAME && s.fact != MONARCH_FACT_TILED) return MONARCH_ERR_INVALID_ARG;
     if (s.fact == MONARCH_FACT_TILED) {
         if (s.tile_h < 1 || s.tile_w < 1 || s.H % s.tile_h != 0 || s.W % s.tile_w != 0)
@@ -177,18 +178,20 @@ int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
     return MONARCH_OK;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides
-// in bytes for dims 1..rank-1.
+// 16-bit (bf16 or fp16) tensor map with 128-byte swizzle; dims/strides
+// innermost first, strides in bytes for dims 1..rank-1.
 int make_map(CUtensorMap *map, const void *ptr, int rank, const cuuint64_t *dims,
-             const cuuint64_t *strides, const cuuint32_t *box) {
+             const cuuint64_t *strides, const cuuint32_t *box, int dtype) {
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims,
+    const CUtensorMapDataType ty =
+        dtype == MONARCH_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = g_encode(map, ty, rank, const_cast<void *>(ptr), dims,
                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MONARCH_OK : MONARCH_ERR_CUDA;
 }
 
-// Stage-1 view of a [B*heads][N][d] bf16 tensor.
+// Stage-1 view of a [B*heads][N][d] 16-bit tensor.
 //   frame: (d, m, B*heads*T), box (64, 128, 1): one 128-token slab of a frame
 //   tiled: (d, tile_w, tiles_w, tile_h, tiles_h*B*heads*T),
 //          box (64, tile_w, 1, rows, 1): `rows` tile rows of one tile
@@ -199,7 +202,7 @@ int stage1_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams
                               static_cast<cuuint64_t>(s.B) * s.heads * s.T};
         cuuint64_t strides[2] = {d * es, static_cast<cuuint64_t>(p.m) * d * es};
         cuuint32_t box[3] = {64, 128, 1};
-        return make_map(map, ptr, 3, dims, strides, box);
+        return make_map(map, ptr, 3, dims, strides, box, s.dtype);
     }
     cuuint64_t dims[5] = {d, static_cast<cuuint64_t>(s.tile_w), static_cast<cuuint64_t>(p.tiles_w),
                           static_cast<cuuint64_t>(s.tile_h),
@@ -209,7 +212,7 @@ int stage1_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams
                              static_cast<cuuint64_t>(s.tile_h) * s.W * d * es};
     cuuint32_t box[5] = {64, static_cast<cuuint32_t>(s.tile_w), 1,
                          static_cast<cuuint32_t>(p.rows_per_tile), 1};
-    return make_map(map, ptr, 5, dims, strides, box);
+    return make_map(map, ptr, 5, dims, strides, box, s.dtype);
 }
 
 // Stage-2 view: (d, H*W, T, B*heads), box (64, npos, T, 1): npos consecutive
@@ -221,7 +224,7 @@ int stage2_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams
     cuuint64_t strides[3] = {d * es, static_cast<cuuint64_t>(p.HW) * d * es,
                              static_cast<cuuint64_t>(s.N) * d * es};
     cuuint32_t box[4] = {64, static_cast<cuuint32_t>(p.npos), static_cast<cuuint32_t>(s.T), 1};
-    return make_map(map, ptr, 4, dims, strides, box);
+    return make_map(map, ptr, 4, dims, strides, box, s.dtype);
 }
 
 // Optional per-launch events: ev[0] before the first launch, ev[i+1] after launch i.
@@ -234,7 +237,7 @@ struct LaunchEvents {
     }
 };
 
-template <int D>
+template <int D, bool F16>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
               cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr) {
     DeviceInfo *di = nullptr;
@@ -242,9 +245,9 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     if (st) return st;
     if ((st = get_encode())) return st;
     using L = TcLayout<D>;
-    const int di_idx = D == 128 ? 1 : 0;
+    const int di_idx = (F16 ? 2 : 0) + (D == 128 ? 1 : 0);
     if (!di->tc_attr[di_idx]) {
-        if (cudaFuncSetAttribute(monarch_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(monarch_tc_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  L::ALLOC) != cudaSuccess)
             return MONARCH_ERR_CUDA;
         di->tc_attr[di_idx] = true;
@@ -329,7 +332,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         return MONARCH_ERR_CUDA;
     lev.record(0, stream);
     const int grid = p.units < di->sms ? p.units : di->sms;
-    monarch_tc_kernel<D><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
+    monarch_tc_kernel<D, F16><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
     lev.record(++lev.launches, stream);
     return MONARCH_OK;
@@ -427,7 +430,9 @@ static int fwd_impl(const void *q, const void *k, const void *v, void *out, int 
     if (st) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (dtype == MONARCH_DTYPE_BF16)
-        st = d == 128 ? launch_tc<128>(q, k, v, out, s, cs, lev) : launch_tc<64>(q, k, v, out, s, cs, lev);
+        st = d == 128 ? launch_tc<128, false>(q, k, v, out, s, cs, lev) : launch_tc<64, false>(q, k, v, out, s, cs, lev);
+    else if (dtype == MONARCH_DTYPE_F16)
+        st = d == 128 ? launch_tc<128, true>(q, k, v, out, s, cs, lev) : launch_tc<64, true>(q, k, v, out, s, cs, lev);
     else
         st = d == 128 ? launch_f32<128>(q, k, v, out, s, cs, lev) : launch_f32<64>(q, k, v, out, s, cs, lev);
     if (st) return st;
@@ -496,8 +501,8 @@ int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *
     if ((st = noalloc_counters(&counters))) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     LaunchEvents lev;
-    st = d == 128 ? launch_tc<128>(q, k, v, out, s, cs, lev, counters)
-                  : launch_tc<64>(q, k, v, out, s, cs, lev, counters);
+    st = d == 128 ? launch_tc<128, false>(q, k, v, out, s, cs, lev, counters)
+                  : launch_tc<64, false>(q, k, v, out, s, cs, lev, counters);
     if (st) return st;
     if (env_debug()) return read_status(cs, 0);
     return MONARCH_OK;

@@ -60,7 +60,7 @@ def _call(lib, q=16, k=32, v=48, out=4096, B=1, heads=1, T=2, H=4, W=4, d=128, f
     dict(out=0),
     dict(B=0), dict(heads=0), dict(T=0), dict(H=0), dict(W=-1),
     dict(d=96), dict(d=256),        # unsupported head width
-    dict(dtype=2),                  # unknown dtype
+    dict(dtype=3),                  # unknown dtype
     dict(fact=2),                   # unknown factorisation
     dict(fact=1, th=3, tw=2),       # tile does not divide H
     dict(fact=1, th=2, tw=0),
