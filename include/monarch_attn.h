@@ -96,6 +96,28 @@ int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out,
                      void *stream);
 
 /*
+ * monarch_attn_fwd_strided -- monarch_attn_fwd for q, k, v and out laid out
+ * with the given element strides: element c of token n of (batch b, head h)
+ * is at b*stride_b + h*stride_h + n*stride_n + c in each of the four tensors
+ * (the d features of a token are contiguous).  [B][heads][N][d] is
+ * (heads*N*d, N*d, d); [B][N][heads][d], the layout of many video DiT
+ * codebases, is (N*heads*d, d, heads*d).  Token order within N stays
+ * n = (t*H + h)*W + w.
+ *
+ * Errors, besides monarch_attn_fwd's: MONARCH_ERR_INVALID_ARG if a stride is
+ * below 1, if token rows of one tensor would overlap (sorted by stride, each
+ * stride must be at least the next smaller stride times its extent, and the
+ * smallest at least d), or, for 16-bit dtypes, if a stride is not a multiple
+ * of 8 elements (16 bytes); MONARCH_ERR_UNSUPPORTED for MONARCH_FACT_TILED
+ * with strides other than the contiguous ones.
+ */
+int monarch_attn_fwd_strided(const void *q, const void *k, const void *v, void *out,
+                             int B, int heads, int T, int H, int W, int d,
+                             int factorisation, int tile_h, int tile_w, int dtype,
+                             long long stride_b, long long stride_h, long long stride_n,
+                             void *stream);
+
+/*
  * monarch_attn_fwd_host -- the same operator for inputs and output in host
  * memory.  Queues on `stream`: copies of h_q, h_k, h_v into the caller's
  * device buffers d_q, d_k, d_v (one cudaMemcpyAsync each), monarch_attn_fwd

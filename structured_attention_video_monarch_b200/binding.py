@@ -59,6 +59,9 @@ def load_library(path: str | None = None):
     lib.monarch_attn_device_status.restype = i
     lib.monarch_attn_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.monarch_attn_selftest_timeout.restype = i
+    ll = ctypes.c_longlong
+    lib.monarch_attn_fwd_strided.argtypes = [vp, vp, vp, vp] + [i] * 10 + [ll, ll, ll, vp]
+    lib.monarch_attn_fwd_strided.restype = i
     lib.monarch_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp] + [i] * 9 + [vp]
     lib.monarch_attn_fwd_noalloc.restype = i
     lib.monarch_attn_version.argtypes = []
@@ -116,6 +119,32 @@ def monarch_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, T: int, 
         int(factorisation), int(tile_h), int(tile_w), _dtype_code(q), _stream_ptr(stream))
     if st != 0:
         raise MonarchError(st, "monarch_attn_fwd")
+    return out
+
+
+def monarch_attn_fwd_strided(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                             T: int, H: int, W: int, factorisation: int = FACT_FRAME, tile_h: int = 0,
+                             tile_w: int = 0, stream=None) -> torch.Tensor:
+    """monarch_attn_fwd on [B, heads, N, d] views with any batch/head/token
+    strides (feature stride 1), e.g. ``x.permute(0, 2, 1, 3)`` of a [B, N, heads, d]
+    tensor.  q, k, v and out must share one shape, dtype and stride set.
+    """
+    ts = (q, k, v, out)
+    if not all(t.is_cuda for t in ts):
+        raise ValueError("q, k, v, out must be CUDA tensors")
+    if q.dim() != 4 or any(t.shape != q.shape or t.dtype != q.dtype for t in ts):
+        raise ValueError("q, k, v, out must share one [B, heads, N, d] shape and dtype")
+    if any(t.stride() != q.stride() for t in ts) or q.stride(3) != 1:
+        raise ValueError("q, k, v, out must share strides, with unit feature stride")
+    B, heads, N, d = q.shape
+    if N != T * H * W:
+        raise ValueError(f"N={N} does not equal T*H*W={T * H * W}")
+    sb, sh, sn, _ = q.stride()
+    st = load_library().monarch_attn_fwd_strided(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, heads, T, H, W, d,
+        int(factorisation), int(tile_h), int(tile_w), _dtype_code(q), sb, sh, sn, _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_strided")
     return out
 
 

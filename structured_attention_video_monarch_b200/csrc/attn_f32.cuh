@@ -22,7 +22,15 @@ struct F32Params {
     int nblk_bh;    // stage-1 blocks per (batch, head)
     int qchunks;    // 64-query chunks per stage-1 block
     float scale;
+    int heads;
+    long long sB, sH, sN;  // element strides of batch, head and token (all four tensors)
 };
+
+// Element offset of token n's row of batch-head bh.
+__device__ __forceinline__ long long f32_row(const F32Params &p, long long bh, long long n) {
+    const long long b = bh / p.heads;
+    return b * p.sB + (bh - b * p.heads) * p.sH + n * p.sN;
+}
 
 __device__ __forceinline__ long long f32_s1_token(const F32Params &p, int b, int i) {
     if (p.fact == 0) return static_cast<long long>(b) * p.HW + i;
@@ -51,12 +59,11 @@ monarch_f32_stage1(const float *__restrict__ q, const float *__restrict__ k,
     const int lrow = threadIdx.x >> 1, half = threadIdx.x & 1;
     const int i = qc * 64 + lrow;
     const bool active = i < p.m;
-    const long long base = bh * p.N;
     const long long n = active ? f32_s1_token(p, b, i) : 0;
     float qr[DH], o[DH];
 #pragma unroll
     for (int e = 0; e < DH; ++e) {
-        qr[e] = active ? q[(base + n) * D + 2 * e + half] * p.scale : 0.f;
+        qr[e] = active ? q[f32_row(p, bh, n) + 2 * e + half] * p.scale : 0.f;
         o[e] = 0.f;
     }
     float mrun = -INFINITY, l = 0.f;
@@ -66,8 +73,8 @@ monarch_f32_stage1(const float *__restrict__ q, const float *__restrict__ k,
             const int jj = idx / D, c = idx % D, j = j0 + jj;
             if (j < p.m) {
                 const long long nk = f32_s1_token(p, b, j);
-                ks[jj][c] = k[(base + nk) * D + c];
-                vs[jj][c] = v[(base + nk) * D + c];
+                ks[jj][c] = k[f32_row(p, bh, nk) + c];
+                vs[jj][c] = v[f32_row(p, bh, nk) + c];
             }
         }
         __syncthreads();
@@ -93,7 +100,7 @@ monarch_f32_stage1(const float *__restrict__ q, const float *__restrict__ k,
     if (active) {
         const float inv = 1.f / l;
 #pragma unroll
-        for (int e = 0; e < DH; ++e) out[(base + n) * D + 2 * e + half] = o[e] * inv;
+        for (int e = 0; e < DH; ++e) out[f32_row(p, bh, n) + 2 * e + half] = o[e] * inv;
     }
 }
 
@@ -110,12 +117,11 @@ monarch_f32_stage2(const float *__restrict__ q, const float *__restrict__ k, flo
     const long long g = blockIdx.x;
     const long long bh = g / p.HW;
     const int pos = static_cast<int>(g % p.HW);
-    const long long base = bh * p.N;
     for (int idx = threadIdx.x; idx < p.T * D; idx += blockDim.x) {
         const int t = idx / D, c = idx % D;
         const long long n = static_cast<long long>(t) * p.HW + pos;
-        ks[idx] = k[(base + n) * D + c];
-        ys[idx] = out[(base + n) * D + c];
+        ks[idx] = k[f32_row(p, bh, n) + c];
+        ys[idx] = out[f32_row(p, bh, n) + c];
     }
     __syncthreads();
     const int t = threadIdx.x >> 1, half = threadIdx.x & 1;
@@ -124,7 +130,7 @@ monarch_f32_stage2(const float *__restrict__ q, const float *__restrict__ k, flo
     float qr[DH], o[DH];
 #pragma unroll
     for (int e = 0; e < DH; ++e) {
-        qr[e] = active ? q[(base + n) * D + 2 * e + half] * p.scale : 0.f;
+        qr[e] = active ? q[f32_row(p, bh, n) + 2 * e + half] * p.scale : 0.f;
         o[e] = 0.f;
     }
     float mrun = -INFINITY, l = 0.f;
@@ -148,7 +154,7 @@ monarch_f32_stage2(const float *__restrict__ q, const float *__restrict__ k, flo
     if (active) {
         const float inv = 1.f / l;
 #pragma unroll
-        for (int e = 0; e < DH; ++e) out[(base + n) * D + 2 * e + half] = o[e] * inv;
+        for (int e = 0; e < DH; ++e) out[f32_row(p, bh, n) + 2 * e + half] = o[e] * inv;
     }
 }
 

@@ -79,6 +79,8 @@ struct TcParams {
     long long timeout_cycles;
     unsigned *status;
     void *out;                      // 16-bit output (epilogue stores)
+    long long sB, sH, sN;           // element strides of batch, head and token (all four tensors)
+    FastDiv fd_heads;               // batch-head index -> (batch, head)
     int out_v8;                     // out is 32-byte aligned: 32-byte epilogue stores
 };
 
@@ -191,7 +193,12 @@ __device__ __forceinline__ void s1_load(const TcParams &p, const CUtensorMap *ma
                                         uint32_t bar, int blk, int tile) {
     if (p.fact == 0) {
 #pragma unroll
-        for (int pn = 0; pn < NP; ++pn) tma_load_3d(dst + pn * 16384, map, bar, pn * 64, tile * 128, blk);
+        {
+            // map (d, m, T, heads, B): block blk = bh * T + t
+            const int bh = static_cast<int>(fdiv(blk, p.fd_nblk_bh)), t = blk - bh * p.nblk_bh;
+            const int b = static_cast<int>(fdiv(bh, p.fd_heads)), hd = bh - b * p.heads;
+            for (int pn = 0; pn < NP; ++pn) tma_load_5d(dst + pn * 16384, map, bar, pn * 64, tile * 128, t, hd, b);
+        }
     } else {
         const int frame = static_cast<int>(fdiv(blk, p.fd_tpf));
         const int tif = blk - frame * p.tiles_h * p.tiles_w;
@@ -204,10 +211,12 @@ __device__ __forceinline__ void s1_load(const TcParams &p, const CUtensorMap *ma
 }
 
 template <int NP>
-__device__ __forceinline__ void s2_load(const CUtensorMap *map, uint32_t dst, uint32_t bar, int npos,
+__device__ __forceinline__ void s2_load(const TcParams &p, const CUtensorMap *map, uint32_t dst, uint32_t bar,
                                         int bh, int chunk) {
+    // map (d, H*W, T, heads, B)
+    const int b = static_cast<int>(fdiv(bh, p.fd_heads)), hd = bh - b * p.heads;
 #pragma unroll
-    for (int pn = 0; pn < NP; ++pn) tma_load_4d(dst + pn * 16384, map, bar, pn * 64, chunk * npos, 0, bh);
+    for (int pn = 0; pn < NP; ++pn) tma_load_5d(dst + pn * 16384, map, bar, pn * 64, chunk * p.npos, 0, hd, b);
 }
 
 // Output token (index inside its batch-head) of row `row` of a lane, or -1
@@ -457,7 +466,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         s1_load<NP>(p, &mq1, dst, q_full(i), ln.blk, ln.tile);
                     } else {
                         mbar_arrive_expect_tx(q_full(i), NP * p.npos * p.T * 128);
-                        s2_load<NP>(&mq2, dst, q_full(i), p.npos, ln.blk, ln.tile);
+                        s2_load<NP>(p, &mq2, dst, q_full(i), ln.blk, ln.tile);
                     }
                 }
                 const int nkv = un.shared ? 1 : un.nq;
@@ -496,7 +505,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         if (un.kind == UNIT_STAGE1)
                             s1_load<NP>(p, is_v ? &mv1 : &mk1, dst, kv_full(s), ln.blk, j);
                         else
-                            s2_load<NP>(is_v ? &my2 : &mk2, dst, kv_full(s), p.npos, ln.blk, ln.tile);
+                            s2_load<NP>(p, is_v ? &my2 : &mk2, dst, kv_full(s), ln.blk, ln.tile);
                     }
                 }
             }
@@ -756,9 +765,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             int bh;
             const long long tok = lane_row_token(p, un.kind, un.ln[li], row, bh);
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) +
-                                                   (static_cast<long long>(bh) * p.N + (tok < 0 ? 0 : tok)) * D +
-                                                   h * (D / 2));
+            const int ob = static_cast<int>(fdiv(static_cast<uint32_t>(bh), p.fd_heads)), oh = bh - ob * p.heads;
+            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + ob * p.sB + oh * p.sH +
+                                                   (tok < 0 ? 0 : tok) * p.sN + h * (D / 2));
             if (!mbar_wait(o_full(li), of_par, ctl)) { ok = false; break; }
             of_par ^= 1u;
             tc_fence_after();

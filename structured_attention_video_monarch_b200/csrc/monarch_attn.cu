@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/monarch_attn.h"
@@ -151,6 +152,7 @@ bool overlaps(const void *a, const void *b, size_t bytes) {
 struct Shape {
     int B, heads, T, H, W, d, fact, tile_h, tile_w, dtype;
     long long N, elems;
+    long long sB = 0, sH = 0, sN = 0;  // element strides; all 0 = contiguous [B][heads][N][d]
 };
 
 int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
@@ -169,7 +171,30 @@ int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
     s.N = static_cast<long long>(s.T) * s.H * s.W;
     if (s.N > (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
     s.elems = static_cast<long long>(s.B) * s.heads * s.N * s.d;
-    const size_t bytes = static_cast<size_t>(s.elems) * (s.dtype == MONARCH_DTYPE_F32 ? 4 : 2);
+    const long long cB = static_cast<long long>(s.heads) * s.N * s.d, cH = s.N * s.d, cN = s.d;
+    if (s.sB == 0 && s.sH == 0 && s.sN == 0) {
+        s.sB = cB; s.sH = cH; s.sN = cN;
+    } else {
+        if (s.sB < 1 || s.sH < 1 || s.sN < 1) return MONARCH_ERR_INVALID_ARG;
+        // rows must not overlap: sorted by stride, each stride covers the dims below it
+        long long st[3] = {s.sN, s.sH, s.sB}, ex[3] = {s.N, s.heads, s.B};
+        for (int a = 0; a < 3; ++a)
+            for (int b = a + 1; b < 3; ++b)
+                if (st[b] < st[a]) { std::swap(st[a], st[b]); std::swap(ex[a], ex[b]); }
+        long long need = s.d;
+        for (int a = 0; a < 3; ++a) {
+            if (ex[a] == 1) continue;
+            if (st[a] < need) return MONARCH_ERR_INVALID_ARG;
+            need = st[a] * ex[a];
+        }
+        // 16-bit paths read through TMA: strides must be 16-byte multiples
+        if (s.dtype != MONARCH_DTYPE_F32 && (s.sB % 8 || s.sH % 8 || s.sN % 8)) return MONARCH_ERR_INVALID_ARG;
+        // the tiled factorisation's tensor map needs the contiguous layout
+        if (s.fact == MONARCH_FACT_TILED && (s.sB != cB || s.sH != cH || s.sN != cN))
+            return MONARCH_ERR_UNSUPPORTED;
+    }
+    const long long span = (s.B - 1) * s.sB + (s.heads - 1) * s.sH + (s.N - 1) * s.sN + s.d;
+    const size_t bytes = static_cast<size_t>(span) * (s.dtype == MONARCH_DTYPE_F32 ? 4 : 2);
     if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
         return MONARCH_ERR_INVALID_ARG;
     if (s.T > 128) return MONARCH_ERR_UNSUPPORTED;
@@ -191,18 +216,20 @@ int make_map(CUtensorMap *map, const void *ptr, int rank, const cuuint64_t *dims
     return r == CUDA_SUCCESS ? MONARCH_OK : MONARCH_ERR_CUDA;
 }
 
-// Stage-1 view of a [B*heads][N][d] 16-bit tensor.
-//   frame: (d, m, B*heads*T), box (64, 128, 1): one 128-token slab of a frame
+// Stage-1 view of a 16-bit tensor with element strides (sB, sH, sN).
+//   frame: (d, m, T, heads, B), box (64, 128, 1, 1, 1): one 128-token slab of a frame
 //   tiled: (d, tile_w, tiles_w, tile_h, tiles_h*B*heads*T),
 //          box (64, tile_w, 1, rows, 1): `rows` tile rows of one tile
 int stage1_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams &p) {
     const cuuint64_t es = 2, d = s.d;
     if (s.fact == MONARCH_FACT_FRAME) {
-        cuuint64_t dims[3] = {d, static_cast<cuuint64_t>(p.m),
-                              static_cast<cuuint64_t>(s.B) * s.heads * s.T};
-        cuuint64_t strides[2] = {d * es, static_cast<cuuint64_t>(p.m) * d * es};
-        cuuint32_t box[3] = {64, 128, 1};
-        return make_map(map, ptr, 3, dims, strides, box, s.dtype);
+        const cuuint64_t sN = static_cast<cuuint64_t>(s.sN);
+        cuuint64_t dims[5] = {d, static_cast<cuuint64_t>(p.m), static_cast<cuuint64_t>(s.T),
+                              static_cast<cuuint64_t>(s.heads), static_cast<cuuint64_t>(s.B)};
+        cuuint64_t strides[4] = {sN * es, static_cast<cuuint64_t>(p.m) * sN * es,
+                                 static_cast<cuuint64_t>(s.sH) * es, static_cast<cuuint64_t>(s.sB) * es};
+        cuuint32_t box[5] = {64, 128, 1, 1, 1};
+        return make_map(map, ptr, 5, dims, strides, box, s.dtype);
     }
     cuuint64_t dims[5] = {d, static_cast<cuuint64_t>(s.tile_w), static_cast<cuuint64_t>(p.tiles_w),
                           static_cast<cuuint64_t>(s.tile_h),
@@ -215,16 +242,16 @@ int stage1_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams
     return make_map(map, ptr, 5, dims, strides, box, s.dtype);
 }
 
-// Stage-2 view: (d, H*W, T, B*heads), box (64, npos, T, 1): npos consecutive
+// Stage-2 view: (d, H*W, T, heads, B), box (64, npos, T, 1, 1): npos consecutive
 // positions across all T frames, landing in shared memory as rows t*npos + pos.
 int stage2_map(CUtensorMap *map, const void *ptr, const Shape &s, const TcParams &p) {
-    const cuuint64_t es = 2, d = s.d;
-    cuuint64_t dims[4] = {d, static_cast<cuuint64_t>(p.HW), static_cast<cuuint64_t>(s.T),
-                          static_cast<cuuint64_t>(s.B) * s.heads};
-    cuuint64_t strides[3] = {d * es, static_cast<cuuint64_t>(p.HW) * d * es,
-                             static_cast<cuuint64_t>(s.N) * d * es};
-    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(p.npos), static_cast<cuuint32_t>(s.T), 1};
-    return make_map(map, ptr, 4, dims, strides, box, s.dtype);
+    const cuuint64_t es = 2, d = s.d, sN = static_cast<cuuint64_t>(s.sN);
+    cuuint64_t dims[5] = {d, static_cast<cuuint64_t>(p.HW), static_cast<cuuint64_t>(s.T),
+                          static_cast<cuuint64_t>(s.heads), static_cast<cuuint64_t>(s.B)};
+    cuuint64_t strides[4] = {sN * es, static_cast<cuuint64_t>(p.HW) * sN * es,
+                             static_cast<cuuint64_t>(s.sH) * es, static_cast<cuuint64_t>(s.sB) * es};
+    cuuint32_t box[5] = {64, static_cast<cuuint32_t>(p.npos), static_cast<cuuint32_t>(s.T), 1, 1};
+    return make_map(map, ptr, 5, dims, strides, box, s.dtype);
 }
 
 // Optional per-launch events: ev[0] before the first launch, ev[i+1] after launch i.
@@ -309,7 +336,10 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.d)));
     p.timeout_cycles = env_timeout_cycles();
     p.out = out;
-    p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 ? 1 : 0;
+    p.sB = s.sB; p.sH = s.sH; p.sN = s.sN;
+    p.fd_heads = make_fastdiv(static_cast<uint32_t>(s.heads));
+    p.out_v8 = ((reinterpret_cast<uintptr_t>(out) & 31u) == 0 && s.sB % 16 == 0 && s.sH % 16 == 0 &&
+                s.sN % 16 == 0) ? 1 : 0;
     unsigned *status = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_device_status) != cudaSuccess)
         return MONARCH_ERR_CUDA;
@@ -357,6 +387,8 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
         p.nblk_bh = s.T;
     }
     p.qchunks = (p.m + 63) / 64;
+    p.heads = s.heads;
+    p.sB = s.sB; p.sH = s.sH; p.sN = s.sN;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.d)));
     const long long bh = static_cast<long long>(s.B) * s.heads;
     const long long g1 = bh * p.nblk_bh * p.qchunks;
@@ -424,8 +456,9 @@ extern "C" {
 
 static int fwd_impl(const void *q, const void *k, const void *v, void *out, int B, int heads, int T,
                     int H, int W, int d, int factorisation, int tile_h, int tile_w, int dtype,
-                    void *stream, LaunchEvents &lev) {
+                    void *stream, LaunchEvents &lev, long long sb = 0, long long sh = 0, long long sn = 0) {
     Shape s{B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
+    s.sB = sb; s.sH = sh; s.sN = sn;
     int st = validate(q, k, v, out, s);
     if (st) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -446,6 +479,15 @@ int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out, int
     LaunchEvents lev;
     return fwd_impl(q, k, v, out, B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, stream,
                     lev);
+}
+
+int monarch_attn_fwd_strided(const void *q, const void *k, const void *v, void *out, int B, int heads,
+                             int T, int H, int W, int d, int factorisation, int tile_h, int tile_w, int dtype,
+                             long long stride_b, long long stride_h, long long stride_n, void *stream) {
+    if (stride_b < 1 || stride_h < 1 || stride_n < 1) return MONARCH_ERR_INVALID_ARG;
+    LaunchEvents lev;
+    return fwd_impl(q, k, v, out, B, heads, T, H, W, d, factorisation, tile_h, tile_w, dtype, stream, lev,
+                    stride_b, stride_h, stride_n);
 }
 
 int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void *out, int B, int heads,

@@ -99,3 +99,19 @@ def test_product_package_does_not_import_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "monarch_oracle" not in text, f
+
+
+def _strided(lib, sb, sh, sn, B=1, heads=2, T=2, H=4, W=4, d=128, fact=0, th=0, tw=0, dtype=1):
+    big = 1 << 40
+    return lib.monarch_attn_fwd_strided(16, big, 2 * big, 3 * big, B, heads, T, H, W, d, fact, th, tw,
+                                        dtype, sb, sh, sn, None)
+
+
+def test_strided_validation_without_cuda(lib):
+    N, d, heads = 32, 128, 2
+    assert _strided(lib, 0, N * d, d) == 1                   # stride below 1
+    assert _strided(lib, heads * N * d, N * d, d - 8) == 1   # token rows overlap
+    assert _strided(lib, heads * N * d, d, d) == 1           # heads and tokens overlap
+    assert _strided(lib, heads * N * d, N * d + 4, d) == 1   # not a 16-byte multiple (bf16)
+    # the tiled factorisation keeps the contiguous layout
+    assert _strided(lib, N * heads * d, d, heads * d, fact=1, th=2, tw=2) == 2

@@ -239,3 +239,48 @@ def test_timeout_machinery_reports_and_context_survives():
     assert binding.selftest_timeout(2_000_000) == 4  # MONARCH_ERR_TIMEOUT
     assert binding.last_device_error() == 0          # the self-test cleared the word
     test_tiny_fp32_full()                             # the context is still usable
+
+
+# ------------------------------------------------------------------ strided layouts
+
+STRIDED_CASES = [
+    # B, heads, T, H, W, d
+    (2, 3, 3, 12, 20, 128),
+    (1, 2, 5, 9, 17, 64),
+]
+
+
+@pytest.mark.parametrize("B,heads,T,H,W,d", STRIDED_CASES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32], ids=["bf16", "f16", "f32"])
+def test_bnhd_layout_matches_contiguous_bitwise(B, heads, T, H, W, d, dtype):
+    """[B, N, heads, d] tensors through the strided entry point give exactly the
+    contiguous call's result (same arithmetic, different addressing)."""
+    dev = _dev()
+    q, k, v = workloads.random_inputs(B, heads, T, H, W, d, dtype=dtype, seed=B * 100 + T,
+                                      scale=d ** -0.25 if dtype == torch.float32 else 1.0)
+    q, k, v = (x.to(dev) for x in (q, k, v))
+    ref = torch.full_like(q, float("nan"))
+    binding.monarch_attn_fwd(q, k, v, T, H, W, out=ref)
+    # BNHD storage, viewed as [B, heads, N, d]
+    qs, ks, vs = (x.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3) for x in (q, k, v))
+    out_s = torch.full((B, T * H * W, heads, d), float("nan"), dtype=dtype, device=dev).permute(0, 2, 1, 3)
+    binding.monarch_attn_fwd_strided(qs, ks, vs, out_s, T, H, W)
+    torch.cuda.synchronize()
+    assert binding.last_device_error() == 0
+    assert torch.equal(out_s.contiguous(), ref)
+
+
+def test_strided_entry_with_contiguous_strides_and_tiles():
+    dev = _dev()
+    B, heads, T, H, W, d, th, tw = 1, 2, 3, 20, 26, 128, 10, 13
+    q, k, v = (x.to(dev) for x in workloads.random_inputs(B, heads, T, H, W, d, seed=3))
+    ref = torch.empty_like(q)
+    binding.monarch_attn_fwd(q, k, v, T, H, W, 1, th, tw, out=ref)
+    out = torch.full_like(q, float("nan"))
+    binding.monarch_attn_fwd_strided(q, k, v, out, T, H, W, 1, th, tw)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    # tiles need the contiguous layout
+    qs = q.permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    with pytest.raises(binding.MonarchError):
+        binding.monarch_attn_fwd_strided(qs, qs, qs, torch.empty_like(qs), T, H, W, 1, th, tw)
