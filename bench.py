@@ -25,6 +25,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -103,13 +104,18 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, log_dir: str | None = None):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.keep = bool(log_dir)
+        if log_dir:  # keep the raw samples
+            self.path = os.path.join(log_dir, f"clocks_rank{index}.csv")
+        else:
+            fd, self.path = tempfile.mkstemp(prefix=f"clocks_rank{index}_", suffix=".csv")
+            os.close(fd)
 
     def start(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        os.makedirs(os.path.dirname(self.path) or ".", exist_ok=True)
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -129,7 +135,11 @@ class ClockSampler:
             self.proc.kill()
         self.fh.close()
         rows = []
-        for line in open(self.path):
+        with open(self.path) as fh:
+            lines = fh.readlines()
+        if not self.keep:
+            os.unlink(self.path)
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -288,7 +298,7 @@ def run_ours(args):
     torch.cuda.synchronize(device)
 
     # clocks under load: sample during a short soak of the same calls, then the timed region
-    sampler = ClockSampler(device.index)
+    sampler = ClockSampler(device.index, args.clock_log)
     sampler.start()
     t_soak = time.perf_counter()
     i = 0
@@ -421,6 +431,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="directory for the raw nvidia-smi clock samples (default: a temporary file)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture "

@@ -35,7 +35,7 @@ extern "C" {
 typedef enum {
     MONARCH_OK = 0,
     MONARCH_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment, aliasing or enum; nothing launched */
-    MONARCH_ERR_UNSUPPORTED = 2, /* valid but outside this build's limits (see below); nothing launched */
+    MONARCH_ERR_UNSUPPORTED = 2, /* valid but outside the library's limits (see below); nothing launched */
     MONARCH_ERR_LAUNCH = 3,      /* a kernel launch failed (cudaGetLastError after launch) */
     MONARCH_ERR_TIMEOUT = 4,     /* a device-side wait gave up (reported by monarch_attn_device_status) */
     MONARCH_ERR_CUDA = 5         /* a CUDA runtime/driver call other than a launch failed */
@@ -75,7 +75,7 @@ typedef enum {
  *   dtype     MONARCH_DTYPE_BF16, MONARCH_DTYPE_F16 or MONARCH_DTYPE_F32.
  *   stream    cudaStream_t (NULL = legacy default stream) the work is queued on.
  *
- * Limits of this build (MONARCH_ERR_UNSUPPORTED otherwise): T <= 128;
+ * Limits of this library version (MONARCH_ERR_UNSUPPORTED otherwise): T <= 128;
  * tile_w <= 128 for MONARCH_FACT_TILED; N <= 2^31; a device of compute
  * capability 10.0 (B200).  Pointers must be 16-byte aligned
  * (MONARCH_ERR_INVALID_ARG otherwise).

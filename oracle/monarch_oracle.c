@@ -35,7 +35,7 @@
  * group.  Indices stay in the original token order throughout, so no final
  * permutation is applied.
  *
- * Readings where the pages say nothing (each also listed in the design doc):
+ * Readings where the pages say nothing:
  *   - scale d^-1/2 inside every softmax; no mask; no KV cache;
  *   - stage 2 reuses Q and K; its values are stage-1 outputs;
  *   - B1 acts first, then B2;
