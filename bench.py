@@ -127,6 +127,8 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
+            if not self.keep and os.path.exists(self.path):
+                os.unlink(self.path)
             return None
         self.proc.terminate()
         try:
