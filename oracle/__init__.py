@@ -55,9 +55,10 @@ def _configure(lib):
     lib.oracle_monarch_stage2.argtypes = [dp, dp, dp, dp] + [i] * 6
     lib.oracle_monarch_fwd_groups.argtypes = (
         [dp, dp, dp] + [i] * 9 + [ctypes.POINTER(ctypes.c_long), i, dp])
+    lib.oracle_monarch_bwd.argtypes = [dp] * 7 + [i] * 9
     for f in (lib.oracle_monarch_fwd, lib.oracle_monarch_stage1,
               lib.oracle_monarch_stage2, lib.oracle_monarch_fwd_groups,
-              lib.oracle_num_threads):
+              lib.oracle_monarch_bwd, lib.oracle_num_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -124,6 +125,19 @@ def monarch_fwd(q, k, v, T, H, W, fact=FACT_FRAME, tile_h=0, tile_w=0) -> np.nda
     _check(_load().oracle_monarch_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                       B, heads, T, H, W, d, fact, tile_h, tile_w), "fwd")
     return out
+
+
+def monarch_bwd(q, k, v, dout, T, H, W, fact=FACT_FRAME, tile_h=0, tile_w=0):
+    """Gradients (dq, dk, dv) of out = P^T B2 P B1 V for an upstream gradient
+    dout, all [B, heads, T*H*W, d], in float64."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, heads, d = _dims(q, T, H, W)
+    if dout.shape != q.shape:
+        raise ValueError("dout must be shaped like q")
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    _check(_load().oracle_monarch_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), B, heads, T, H, W, d, fact, tile_h, tile_w), "bwd")
+    return dq, dk, dv
 
 
 def monarch_stage1(q, k, v, T, H, W, fact=FACT_FRAME, tile_h=0, tile_w=0) -> np.ndarray:

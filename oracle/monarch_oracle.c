@@ -1,5 +1,6 @@
 /*
- * monarch_oracle.c -- fp64 CPU oracle for the Monarch attention forward.
+ * monarch_oracle.c -- fp64 CPU oracle for the Monarch attention forward and
+ * its gradients.
  *
  * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously correct
  * definition that the CUDA path is checked against.  Only the tests, the
@@ -301,5 +302,137 @@ int oracle_monarch_fwd_groups(const double *q, const double *k, const double *v,
         }
         free(kr); free(vr); free(logit); free(y1); free(yr);
     }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ gradients
+ *
+ * The pages state that their custom kernels run the backward pass as well
+ * (gist.science/nl/paper/2602.12271, section "Methodologie";
+ * gist.science/zh/paper/2602.12271, section 2.2).  The
+ * gradient of the forward above follows from the chain rule alone, so it
+ * needs no reading of the pages beyond the forward's.  For one dense block
+ * with logits l_j = s <q_x, k_j>, weights p = softmax(l) and output
+ * y_x = sum_j p_j val_j, an upstream gradient dy_x gives
+ *     dp_j  = <dy_x, val_j>
+ *     dl_j  = p_j (dp_j - sum_i p_i dp_i)          (softmax Jacobian)
+ *     dq_x += s sum_j dl_j k_j,   dk_j += s dl_j q_x,   dval_j += p_j dy_x.
+ * For out = A2(Q, K) Y1 with Y1 = A1(Q, K) V: stage 2's backward takes dy =
+ * dout and yields dY1 (its value gradient) and stage-2 parts of dQ and dK;
+ * stage 1's backward takes dy = dY1 and yields dV and the stage-1 parts. */
+
+/* Backward of one query of one block: accumulates into dq (the query's row),
+ * dkrows[j] and dvrows[j].  logit and dp are scratch of len doubles. */
+static void attend_one_bwd(const double *q, const double *const *krows,
+                           const double *const *vrows, long len, int d, double scale,
+                           const double *dy, double *logit, double *dp, double *dq,
+                           double *const *dkrows, double *const *dvrows) {
+    double mx = -INFINITY;
+    for (long j = 0; j < len; ++j) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += q[c] * krows[j][c];
+        logit[j] = scale * acc;
+        if (logit[j] > mx) mx = logit[j];
+    }
+    double z = 0.0;
+    for (long j = 0; j < len; ++j) {
+        logit[j] = exp(logit[j] - mx);
+        z += logit[j];
+    }
+    double pdp = 0.0;
+    for (long j = 0; j < len; ++j) {
+        logit[j] /= z; /* now p_j */
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += dy[c] * vrows[j][c];
+        dp[j] = acc;
+        pdp += logit[j] * acc;
+    }
+    for (long j = 0; j < len; ++j) {
+        double dl = logit[j] * (dp[j] - pdp);
+        for (int c = 0; c < d; ++c) {
+            dq[c] += scale * dl * krows[j][c];
+            dkrows[j][c] += scale * dl * q[c];
+            dvrows[j][c] += logit[j] * dy[c];
+        }
+    }
+}
+
+/* Gradients of out = P^T B2 P B1 V with respect to q, k and v for an upstream
+ * gradient dout.  All arrays [B*heads][N][d]; dq, dk, dv are overwritten and
+ * must not alias the inputs or each other. */
+int oracle_monarch_bwd(const double *q, const double *k, const double *v, const double *dout,
+                       double *dq, double *dk, double *dv,
+                       int B, int heads, int T, int H, int W, int d,
+                       int fact, int tile_h, int tile_w) {
+    int st = check_shape(B, heads, T, H, W, d, fact, tile_h, tile_w);
+    if (st) return st;
+    long HW = (long)H * W, N = (long)T * HW;
+    size_t n = (size_t)B * heads * N * d;
+    double *y1 = (double *)malloc(sizeof(double) * n);
+    double *dy1 = (double *)calloc(n, sizeof(double));
+    if (!y1 || !dy1) { free(y1); free(dy1); return ORACLE_ERR_NOMEM; }
+    memset(dq, 0, sizeof(double) * n);
+    memset(dk, 0, sizeof(double) * n);
+    memset(dv, 0, sizeof(double) * n);
+    st = oracle_monarch_stage1(q, k, v, y1, B, heads, T, H, W, d, fact, tile_h, tile_w);
+    if (st) { free(y1); free(dy1); return st; }
+    double scale = 1.0 / sqrt((double)d);
+    int failed = 0;
+    long nblocks, len;
+    stage1_geometry(T, H, W, fact, tile_h, tile_w, &nblocks, &len);
+    long maxlen = len > T ? len : T;
+#pragma omp parallel
+    {
+        const double **kr = (const double **)malloc(sizeof(double *) * maxlen);
+        const double **vr = (const double **)malloc(sizeof(double *) * maxlen);
+        double **dkr = (double **)malloc(sizeof(double *) * maxlen);
+        double **dvr = (double **)malloc(sizeof(double *) * maxlen);
+        double *logit = (double *)malloc(sizeof(double) * maxlen);
+        double *dp = (double *)malloc(sizeof(double) * maxlen);
+        if (!kr || !vr || !dkr || !dvr || !logit || !dp) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            /* stage 2: groups of T tokens sharing a position; values Y1 */
+#pragma omp for schedule(dynamic, 16)
+            for (long w = 0; w < (long)B * heads * HW; ++w) {
+                long bh = w / HW, pos = w % HW;
+                long off = bh * N * d;
+                for (int t = 0; t < T; ++t) {
+                    long row = off + (t * HW + pos) * d;
+                    kr[t] = k + row;
+                    vr[t] = y1 + row;
+                    dkr[t] = dk + row;
+                    dvr[t] = dy1 + row;
+                }
+                for (int t = 0; t < T; ++t) {
+                    long row = off + (t * HW + pos) * d;
+                    attend_one_bwd(q + row, kr, vr, T, d, scale, dout + row, logit, dp, dq + row,
+                                   dkr, dvr);
+                }
+            }
+            /* stage 1: blocks; upstream gradient dY1, values V */
+#pragma omp for schedule(dynamic, 1)
+            for (long w = 0; w < (long)B * heads * nblocks; ++w) {
+                long bh = w / nblocks, b = w % nblocks;
+                long off = bh * N * d;
+                for (long j = 0; j < len; ++j) {
+                    long row = off + stage1_token(b, j, T, H, W, fact, tile_h, tile_w) * d;
+                    kr[j] = k + row;
+                    vr[j] = v + row;
+                    dkr[j] = dk + row;
+                    dvr[j] = dv + row;
+                }
+                for (long i = 0; i < len; ++i) {
+                    long row = off + stage1_token(b, i, T, H, W, fact, tile_h, tile_w) * d;
+                    attend_one_bwd(q + row, kr, vr, len, d, scale, dy1 + row, logit, dp, dq + row,
+                                   dkr, dvr);
+                }
+            }
+        }
+        free(kr); free(vr); free(dkr); free(dvr); free(logit); free(dp);
+    }
+    free(y1);
+    free(dy1);
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }

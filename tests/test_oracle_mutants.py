@@ -87,3 +87,49 @@ def test_pins_catch_mutant(tmp_path, name, old, new):
     finally:
         oracle.restore_library(prev)
     assert caught, f"no pin rejects the planted mistake '{name}'"
+
+
+# ---------------------------------------------------------------- gradients
+
+import test_oracle_bwd as bwd_pins
+
+BWD_MUTANTS = [
+    ("bwd_no_jacobian_mean", "double dl = logit[j] * (dp[j] - pdp);", "double dl = logit[j] * dp[j];"),
+    ("bwd_dk_unscaled", "dkrows[j][c] += scale * dl * q[c];", "dkrows[j][c] += dl * q[c];"),
+    ("bwd_dq_uses_values", "dq[c] += scale * dl * krows[j][c];", "dq[c] += scale * dl * vrows[j][c];"),
+    ("bwd_stage1_upstream_is_dout", "attend_one_bwd(q + row, kr, vr, len, d, scale, dy1 + row,",
+     "attend_one_bwd(q + row, kr, vr, len, d, scale, dout + row,"),
+    ("bwd_stage2_values_are_v", "vr[t] = y1 + row;", "vr[t] = v + row;"),
+    ("bwd_dv_unweighted", "dvrows[j][c] += logit[j] * dy[c];", "dvrows[j][c] += dy[c];"),
+    ("bwd_stage2_dk_misplaced", "dkr[t] = dk + row;", "dkr[t] = dv + row;"),
+]
+
+BWD_PROBES = [
+    ("bwd_value_frame", lambda: bwd_pins.test_value_gradient_is_monarch_transpose(*pins.BRUTE_SHAPES[0])),
+    ("bwd_value_tiled", lambda: bwd_pins.test_value_gradient_is_monarch_transpose(*pins.BRUTE_SHAPES[2])),
+    ("bwd_fd_frame", lambda: bwd_pins.test_finite_differences(*bwd_pins.FD_SHAPES[0])),
+    ("bwd_fd_tiled", lambda: bwd_pins.test_finite_differences(*bwd_pins.FD_SHAPES[1])),
+    ("bwd_single_frame", lambda: bwd_pins.test_single_frame_gradients_are_dense_attention_gradients(3, 5, 8)),
+    ("bwd_single_position", lambda: bwd_pins.test_single_position_gradients_are_dense_attention_gradients(5, 8)),
+]
+
+
+def test_unmutated_passes_every_gradient_probe():
+    for label, fn in BWD_PROBES:
+        fn()
+
+
+@pytest.mark.parametrize("name,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
+def test_gradient_pins_catch_mutant(tmp_path, name, old, new):
+    so = _build_mutant(tmp_path, name, old, new)
+    prev = oracle.use_library(so)
+    caught = []
+    try:
+        for label, fn in BWD_PROBES:
+            try:
+                fn()
+            except (AssertionError, ValueError, FloatingPointError):
+                caught.append(label)
+    finally:
+        oracle.restore_library(prev)
+    assert caught, f"no gradient pin rejects the planted mistake '{name}'"
