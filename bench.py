@@ -227,15 +227,18 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ our arm
 
+# The files the tensor-core kernel and its launch are built from.
+KERNEL_SOURCES = ("attn_tc.cuh", "monarch_attn.cu", "sm100.cuh")
+
+
 def kernel_sources_sha256() -> str:
     """Hash of the CUDA sources the dominant kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "structured_attention_video_monarch_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            h.update(name.encode())
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in KERNEL_SOURCES:
+        h.update(name.encode())
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 

@@ -27,6 +27,8 @@
 #ifndef MONARCH_ATTN_H
 #define MONARCH_ATTN_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -182,6 +184,34 @@ int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void 
 int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *out,
                              int B, int heads, int T, int H, int W, int d,
                              int factorisation, int tile_h, int tile_w, void *stream);
+
+/*
+ * monarch_attn_bwd -- gradients of out = P^T B2 P B1 V (as monarch_attn_fwd)
+ * with respect to q, k and v for an upstream gradient dout.  The pages state
+ * that their kernels run the backward pass too (gist.science/nl/paper/
+ * 2602.12271, "Methodologie"; gist.science/zh/paper/2602.12271, section 2.2);
+ * the gradient itself follows from the forward by the chain rule.
+ *
+ * This build provides the fp32 path on CUDA cores (dtype MONARCH_DTYPE_F32;
+ * bf16 and fp16 return MONARCH_ERR_UNSUPPORTED).  Layout [B][heads][N][d]
+ * contiguous, as monarch_attn_fwd.  q, k, v, dout are read; dq, dk, dv are
+ * written (previous contents ignored).  workspace: caller-owned device memory
+ * of at least monarch_attn_bwd_workspace_size(...) bytes, holding the
+ * recomputed stage-1 output and its gradient; its contents on entry do not
+ * matter.  No output or the workspace may overlap an input or another
+ * output.  Limits: T <= 128, and for the stage-1 blocks 8*m floats of shared
+ * memory (m <= 6400 tokens per block).  Asynchronous on `stream`; dk and dv
+ * are accumulated with atomic adds, so repeated calls can differ in the last
+ * bits.  Returns MONARCH_ERR_INVALID_ARG for bad pointers, sizes, alignment
+ * (16 bytes), overlap or a too-small workspace.
+ */
+int monarch_attn_bwd(const void *q, const void *k, const void *v, const void *dout,
+                     void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                     int B, int heads, int T, int H, int W, int d,
+                     int factorisation, int tile_h, int tile_w, int dtype, void *stream);
+
+/* Workspace bytes monarch_attn_bwd needs for these sizes (0 if unsupported). */
+size_t monarch_attn_bwd_workspace_size(int B, int heads, int T, int H, int W, int d, int dtype);
 
 /* Human-readable text of a status code; never NULL, owned by the library. */
 const char *monarch_attn_strerror(int status);

@@ -60,6 +60,11 @@ def load_library(path: str | None = None):
     lib.monarch_attn_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.monarch_attn_selftest_timeout.restype = i
     ll = ctypes.c_longlong
+    sz = ctypes.c_size_t
+    lib.monarch_attn_bwd.argtypes = [vp] * 8 + [sz] + [i] * 10 + [vp]
+    lib.monarch_attn_bwd.restype = i
+    lib.monarch_attn_bwd_workspace_size.argtypes = [i] * 7
+    lib.monarch_attn_bwd_workspace_size.restype = sz
     lib.monarch_attn_fwd_strided.argtypes = [vp, vp, vp, vp] + [i] * 10 + [ll, ll, ll, vp]
     lib.monarch_attn_fwd_strided.restype = i
     lib.monarch_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp] + [i] * 9 + [vp]
@@ -146,6 +151,33 @@ def monarch_attn_fwd_strided(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
     if st != 0:
         raise MonarchError(st, "monarch_attn_fwd_strided")
     return out
+
+
+def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int = FACT_FRAME,
+                     tile_h: int = 0, tile_w: int = 0, stream=None):
+    """Gradients (dq, dk, dv) of monarch_attn_fwd for an upstream gradient dout;
+    fp32 [B, heads, N, d] contiguous CUDA tensors.  Outputs and the workspace are
+    allocated here with PyTorch; every step runs in the library's kernels.
+    """
+    ts = (q, k, v, dout)
+    if not all(t.is_cuda and t.is_contiguous() for t in ts):
+        raise ValueError("q, k, v, dout must be contiguous CUDA tensors")
+    if q.dim() != 4 or any(t.shape != q.shape or t.dtype != q.dtype for t in ts):
+        raise ValueError("q, k, v, dout must share one [B, heads, N, d] shape and dtype")
+    B, heads, N, d = q.shape
+    if N != T * H * W:
+        raise ValueError(f"N={N} does not equal T*H*W={T * H * W}")
+    lib = load_library()
+    code = _dtype_code(q)
+    need = lib.monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, code)
+    ws = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    st = lib.monarch_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                              dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), B, heads, T, H, W,
+                              d, int(factorisation), int(tile_h), int(tile_w), code, _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_bwd")
+    return dq, dk, dv
 
 
 def monarch_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -16,6 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libmonarch_attn.so")
 MAIN = os.path.join(CSRC, "monarch_attn.cu")
+BWD = os.path.join(CSRC, "monarch_bwd.cu")
 
 
 def nvcc_path() -> str:
@@ -40,7 +41,7 @@ def up_to_date() -> bool:
 def nvcc_command(out: str, verbose: bool = False) -> list[str]:
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
-           "-o", out, MAIN]
+           "-o", out, MAIN, BWD]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     return cmd

@@ -115,3 +115,33 @@ def test_strided_validation_without_cuda(lib):
     assert _strided(lib, heads * N * d, N * d + 4, d) == 1   # not a 16-byte multiple (bf16)
     # the tiled factorisation keeps the contiguous layout
     assert _strided(lib, N * heads * d, d, heads * d, fact=1, th=2, tw=2) == 2
+
+
+def test_bwd_workspace_size_and_validation_without_cuda(lib):
+    size = lib.monarch_attn_bwd_workspace_size
+    assert size(1, 2, 3, 4, 5, 64, 0) == 2 * 1 * 2 * 3 * 4 * 5 * 64 * 4
+    assert size(1, 2, 3, 4, 5, 64, 1) == 0   # bf16 backward not built
+    assert size(1, 2, 3, 4, 5, 96, 0) == 0   # unsupported head width
+    big = 1 << 40
+    ptrs = [16 + i * big for i in range(8)]
+    ws = 2 * 1 * 1 * 2 * 4 * 4 * 128 * 4
+
+    def call(**kw):
+        a = dict(B=1, heads=1, T=2, H=4, W=4, d=128, fact=0, th=0, tw=0, dtype=0, ws=ws, p=ptrs)
+        a.update(kw)
+        p = a["p"]
+        return lib.monarch_attn_bwd(*p, a["ws"], a["B"], a["heads"], a["T"], a["H"], a["W"], a["d"],
+                                    a["fact"], a["th"], a["tw"], a["dtype"], None)
+
+    assert call(dtype=1) == 2                     # bf16: not built
+    assert call(ws=ws - 16) == 1                  # workspace too small
+    assert call(p=[0] + ptrs[1:]) == 1            # null pointer
+    assert call(p=ptrs[:4] + [ptrs[0]] + ptrs[5:]) == 1  # dq aliases q
+    assert call(d=96) == 1
+    assert call(T=129) == 2
+    # a workspace that runs into the buffer before it is refused before any
+    # CUDA call (back-to-back buffers that do not overlap are accepted: the
+    # GPU tests allocate them that way)
+    n = ws // 2
+    packed = [16 + i * n for i in range(7)]
+    assert call(p=packed + [packed[6] + 16]) == 1
