@@ -26,6 +26,7 @@ import numpy as np
 
 FACT_FRAME = 0
 FACT_TILED = 1
+FACT_ROW = 2  # the (f*h, w) split: stage-1 blocks are the W tokens of one (frame, row)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "monarch_oracle.c")

@@ -56,6 +56,7 @@
 
 #define ORACLE_FACT_FRAME 0
 #define ORACLE_FACT_TILED 1
+#define ORACLE_FACT_ROW 2
 
 enum { ORACLE_OK = 0, ORACLE_ERR_ARG = 1, ORACLE_ERR_NOMEM = 2 };
 
@@ -72,10 +73,18 @@ static int check_shape(int B, int heads, int T, int H, int W, int d,
     if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1 || d < 1) return ORACLE_ERR_ARG;
     if (fact == ORACLE_FACT_TILED) {
         if (tile_h < 1 || tile_w < 1 || H % tile_h != 0 || W % tile_w != 0) return ORACLE_ERR_ARG;
-    } else if (fact != ORACLE_FACT_FRAME) {
+    } else if (fact != ORACLE_FACT_FRAME && fact != ORACLE_FACT_ROW) {
         return ORACLE_ERR_ARG;
     }
     return ORACLE_OK;
+}
+
+/* Stage-2 groups: the tokens n = i * stride + g, i = 0 .. len-1, of group g
+ * = 0 .. stride-1.  FRAME and TILED: stride H*W (one group per spatial
+ * position, across the T frames).  ROW, the (f*h, w) split: stride W (one
+ * group per column w, across all T*H frame rows). */
+static long stage2_stride(int H, int W, int fact) {
+    return fact == ORACLE_FACT_ROW ? (long)W : (long)H * W;
 }
 
 /* Number of stage-1 blocks per (batch, head) and tokens per block. */
@@ -84,6 +93,9 @@ static void stage1_geometry(int T, int H, int W, int fact, int tile_h, int tile_
     if (fact == ORACLE_FACT_TILED) {
         *nblocks = (long)T * (H / tile_h) * (W / tile_w);
         *blocklen = (long)tile_h * tile_w;
+    } else if (fact == ORACLE_FACT_ROW) {
+        *nblocks = (long)T * H;
+        *blocklen = W;
     } else {
         *nblocks = T;
         *blocklen = (long)H * W;
@@ -104,6 +116,7 @@ static long stage1_token(long b, long i, int T, int H, int W, int fact,
         long h = ti * tile_h + hl, w = tj * tile_w + wl;
         return (t * H + h) * (long)W + w;
     }
+    if (fact == ORACLE_FACT_ROW) return b * (long)W + i;
     return b * (long)H * W + i;
 }
 
@@ -177,45 +190,53 @@ int oracle_monarch_stage1(const double *q, const double *k, const double *v, dou
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
 
-/* Stage 2, out = P^T B2 P y1: every token attends, with its own Q and K,
- * within the group of tokens at the same spatial position across frames;
- * the values are the stage-1 outputs. */
-int oracle_monarch_stage2(const double *q, const double *k, const double *y1, double *out,
-                          int B, int heads, int T, int H, int W, int d) {
-    int st = check_shape(B, heads, T, H, W, d, ORACLE_FACT_FRAME, 0, 0);
-    if (st) return st;
-    long HW = (long)H * W, N = (long)T * HW;
+/* Stage 2 over the groups of stride `gs` (see stage2_stride): every token
+ * attends, with its own Q and K, within its group; the values are the
+ * stage-1 outputs. */
+static int stage2_groups(const double *q, const double *k, const double *y1, double *out,
+                         int B, int heads, long N, long gs, int d) {
+    long gl = N / gs;
     double scale = 1.0 / sqrt((double)d);
-    long nwork = (long)B * heads * HW;
+    long nwork = (long)B * heads * gs;
     int failed = 0;
 #pragma omp parallel
     {
-        const double **kr = (const double **)malloc(sizeof(double *) * T);
-        const double **vr = (const double **)malloc(sizeof(double *) * T);
-        double *logit = (double *)malloc(sizeof(double) * T);
+        const double **kr = (const double **)malloc(sizeof(double *) * gl);
+        const double **vr = (const double **)malloc(sizeof(double *) * gl);
+        double *logit = (double *)malloc(sizeof(double) * gl);
         if (!kr || !vr || !logit) {
 #pragma omp atomic write
             failed = 1;
         } else {
 #pragma omp for schedule(dynamic, 16)
             for (long w = 0; w < nwork; ++w) {
-                long bh = w / HW, pos = w % HW;
+                long bh = w / gs, g = w % gs;
                 const double *qb = q + bh * N * d;
                 const double *kb = k + bh * N * d;
                 const double *yb = y1 + bh * N * d;
                 double *ob = out + bh * N * d;
-                for (int t = 0; t < T; ++t) {
-                    kr[t] = kb + (t * HW + pos) * d;
-                    vr[t] = yb + (t * HW + pos) * d;
+                for (long i = 0; i < gl; ++i) {
+                    kr[i] = kb + (i * gs + g) * d;
+                    vr[i] = yb + (i * gs + g) * d;
                 }
-                for (int t = 0; t < T; ++t)
-                    attend_one(qb + (t * HW + pos) * d, kr, vr, T, d, scale, logit,
-                               ob + (t * HW + pos) * d);
+                for (long i = 0; i < gl; ++i)
+                    attend_one(qb + (i * gs + g) * d, kr, vr, gl, d, scale, logit, ob + (i * gs + g) * d);
             }
         }
         free(kr); free(vr); free(logit);
     }
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* Stage 2, out = P^T B2 P y1, for the frame and tiled splits: every token
+ * attends, with its own Q and K, within the group of tokens at the same
+ * spatial position across frames; the values are the stage-1 outputs. */
+int oracle_monarch_stage2(const double *q, const double *k, const double *y1, double *out,
+                          int B, int heads, int T, int H, int W, int d) {
+    int st = check_shape(B, heads, T, H, W, d, ORACLE_FACT_FRAME, 0, 0);
+    if (st) return st;
+    long N = (long)T * H * W;
+    return stage2_groups(q, k, y1, out, B, heads, N, stage2_stride(H, W, ORACLE_FACT_FRAME), d);
 }
 
 /* Full forward: out = P^T B2 P B1 V.  out must not alias q, k or v. */
@@ -228,7 +249,7 @@ int oracle_monarch_fwd(const double *q, const double *k, const double *v, double
     double *y1 = (double *)malloc(sizeof(double) * n);
     if (!y1) return ORACLE_ERR_NOMEM;
     st = oracle_monarch_stage1(q, k, v, y1, B, heads, T, H, W, d, fact, tile_h, tile_w);
-    if (!st) st = oracle_monarch_stage2(q, k, y1, out, B, heads, T, H, W, d);
+    if (!st) st = stage2_groups(q, k, y1, out, B, heads, (long)T * H * W, stage2_stride(H, W, fact), d);
     free(y1);
     return st;
 }
@@ -244,6 +265,7 @@ int oracle_monarch_fwd_groups(const double *q, const double *k, const double *v,
                               const long *groups, int ngroups, double *out_rows) {
     int st = check_shape(B, heads, T, H, W, d, fact, tile_h, tile_w);
     if (st) return st;
+    if (fact == ORACLE_FACT_ROW) return ORACLE_ERR_ARG; /* groups here are spatial positions */
     long HW = (long)H * W, N = (long)T * HW;
     long nblocks, len;
     stage1_geometry(T, H, W, fact, tile_h, tile_w, &nblocks, &len);
@@ -380,7 +402,8 @@ int oracle_monarch_bwd(const double *q, const double *k, const double *v, const 
     int failed = 0;
     long nblocks, len;
     stage1_geometry(T, H, W, fact, tile_h, tile_w, &nblocks, &len);
-    long maxlen = len > T ? len : T;
+    long gs = stage2_stride(H, W, fact), gl = N / gs;
+    long maxlen = len > gl ? len : gl;
 #pragma omp parallel
     {
         const double **kr = (const double **)malloc(sizeof(double *) * maxlen);
@@ -393,21 +416,21 @@ int oracle_monarch_bwd(const double *q, const double *k, const double *v, const 
 #pragma omp atomic write
             failed = 1;
         } else {
-            /* stage 2: groups of T tokens sharing a position; values Y1 */
+            /* stage 2: the groups of stride gs (gl tokens each); values Y1 */
 #pragma omp for schedule(dynamic, 16)
-            for (long w = 0; w < (long)B * heads * HW; ++w) {
-                long bh = w / HW, pos = w % HW;
+            for (long w = 0; w < (long)B * heads * gs; ++w) {
+                long bh = w / gs, g = w % gs;
                 long off = bh * N * d;
-                for (int t = 0; t < T; ++t) {
-                    long row = off + (t * HW + pos) * d;
-                    kr[t] = k + row;
-                    vr[t] = y1 + row;
-                    dkr[t] = dk + row;
-                    dvr[t] = dy1 + row;
+                for (long i = 0; i < gl; ++i) {
+                    long row = off + (i * gs + g) * d;
+                    kr[i] = k + row;
+                    vr[i] = y1 + row;
+                    dkr[i] = dk + row;
+                    dvr[i] = dy1 + row;
                 }
-                for (int t = 0; t < T; ++t) {
-                    long row = off + (t * HW + pos) * d;
-                    attend_one_bwd(q + row, kr, vr, T, d, scale, dout + row, logit, dp, dq + row,
+                for (long i = 0; i < gl; ++i) {
+                    long row = off + (i * gs + g) * d;
+                    attend_one_bwd(q + row, kr, vr, gl, d, scale, dout + row, logit, dp, dq + row,
                                    dkr, dvr);
                 }
             }

@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_oracle_row as row_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "monarch_oracle.c")
 
@@ -24,21 +25,27 @@ MUTANTS = [
     ("dropped_feature", "for (int c = 0; c < d; ++c) acc += q[c] * krows[j][c];",
      "for (int c = 1; c < d; ++c) acc += q[c] * krows[j][c];"),
     ("shifted_value_column", "y[c] += p * vrows[j][c];", "y[c] += p * vrows[j][(c + 1) % d];"),
-    ("stage2_values_are_v", "st = oracle_monarch_stage2(q, k, y1, out,",
-     "st = oracle_monarch_stage2(q, k, v, out,"),
+    ("stage2_values_are_v", "if (!st) st = stage2_groups(q, k, y1, out,",
+     "if (!st) st = stage2_groups(q, k, v, out,"),
     ("stage1_blocks_position_major", "return b * (long)H * W + i;", "return i * (long)T + b;"),
-    ("stage2_keys_contiguous", "kr[t] = kb + (t * HW + pos) * d;", "kr[t] = kb + (pos * T + t) * d;"),
-    ("stage2_query_is_key", "attend_one(qb + (t * HW + pos) * d, kr, vr, T,",
-     "attend_one(kb + (t * HW + pos) * d, kr, vr, T,"),
+    ("stage2_keys_contiguous", "kr[i] = kb + (i * gs + g) * d;", "kr[i] = kb + (g * gl + i) * d;"),
+    ("stage2_query_is_key", "attend_one(qb + (i * gs + g) * d, kr, vr, gl,",
+     "attend_one(kb + (i * gs + g) * d, kr, vr, gl,"),
     ("tile_rows_interleaved", "long h = ti * tile_h + hl, w = tj * tile_w + wl;",
      "long h = ti + hl * (H / tile_h), w = tj * tile_w + wl;"),
     ("tile_cols_interleaved", "long h = ti * tile_h + hl, w = tj * tile_w + wl;",
      "long h = ti * tile_h + hl, w = tj + wl * (W / tile_w);"),
     ("stage_order_swapped",
      "st = oracle_monarch_stage1(q, k, v, y1, B, heads, T, H, W, d, fact, tile_h, tile_w);\n"
-     "    if (!st) st = oracle_monarch_stage2(q, k, y1, out, B, heads, T, H, W, d);",
-     "st = oracle_monarch_stage2(q, k, v, y1, B, heads, T, H, W, d);\n"
+     "    if (!st) st = stage2_groups(q, k, y1, out, B, heads, (long)T * H * W, stage2_stride(H, W, fact), d);",
+     "st = stage2_groups(q, k, v, y1, B, heads, (long)T * H * W, stage2_stride(H, W, fact), d);\n"
      "    if (!st) st = oracle_monarch_stage1(q, k, y1, out, B, heads, T, H, W, d, fact, tile_h, tile_w);"),
+    # the (f*h, w) split
+    ("row_groups_are_positions", "return fact == ORACLE_FACT_ROW ? (long)W : (long)H * W;",
+     "return (long)H * W;"),
+    ("row_blocks_are_frames",
+     "} else if (fact == ORACLE_FACT_ROW) {\n        *nblocks = (long)T * H;\n        *blocklen = W;",
+     "} else if (fact == ORACLE_FACT_ROW) {\n        *nblocks = T;\n        *blocklen = (long)H * W;"),
 ]
 
 GOLDEN = json.load(open(pins.GOLDEN))["cases"]
@@ -53,6 +60,8 @@ PROBES = [(f"golden:{c['name']}", (lambda c=c: pins.test_hand_derived_golden(c))
     ("zero_qk_tiled", pins.test_zero_qk_tiled_gives_tile_mean),
     ("transpose", lambda: pins.test_transpose_h_w(1, 2, 3)),
     ("numpy", lambda: pins.test_numpy_restatement_small((1, 2, 6, 4, 6, 1, 2, 3))),
+    ("row_brute", lambda: row_pins.test_brute_force_effective_matrix(2, 3, 4, 4)),
+    ("row_single_column", row_pins.test_single_column_is_dense_attention),
 ]
 
 
@@ -99,9 +108,9 @@ BWD_MUTANTS = [
     ("bwd_dq_uses_values", "dq[c] += scale * dl * krows[j][c];", "dq[c] += scale * dl * vrows[j][c];"),
     ("bwd_stage1_upstream_is_dout", "attend_one_bwd(q + row, kr, vr, len, d, scale, dy1 + row,",
      "attend_one_bwd(q + row, kr, vr, len, d, scale, dout + row,"),
-    ("bwd_stage2_values_are_v", "vr[t] = y1 + row;", "vr[t] = v + row;"),
+    ("bwd_stage2_values_are_v", "vr[i] = y1 + row;", "vr[i] = v + row;"),
     ("bwd_dv_unweighted", "dvrows[j][c] += logit[j] * dy[c];", "dvrows[j][c] += dy[c];"),
-    ("bwd_stage2_dk_misplaced", "dkr[t] = dk + row;", "dkr[t] = dv + row;"),
+    ("bwd_stage2_dk_misplaced", "dkr[i] = dk + row;", "dkr[i] = dv + row;"),
 ]
 
 BWD_PROBES = [
