@@ -136,6 +136,26 @@ int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, voi
                           void *stream);
 
 /*
+ * monarch_attn_fwd_host_pipelined -- monarch_attn_fwd_host with the copies
+ * overlapped with the computation.  The B*heads (batch, head) problems are
+ * independent; the call splits them into `nchunks` chunks of consecutive
+ * batch-heads and pipelines them: chunk c+1 is uploaded while chunk c is
+ * computed (on `stream`, one monarch_attn_fwd call per chunk) and chunk c-1
+ * is downloaded.  Uploads and downloads run on two streams the call creates
+ * and destroys; the first upload waits for work already queued on `stream`.
+ * Results equal monarch_attn_fwd_host's bit for bit (each problem's
+ * arithmetic does not depend on the chunking).  Host buffers must be pinned
+ * for the copies to overlap.  nchunks >= 1 (capped at B*heads).  Arguments,
+ * buffer rules and status codes as monarch_attn_fwd_host; returns after h_out
+ * is written, or with the first error.
+ */
+int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k, const void *h_v, void *h_out,
+                                    void *d_q, void *d_k, void *d_v, void *d_out,
+                                    int B, int heads, int T, int H, int W, int d,
+                                    int factorisation, int tile_h, int tile_w, int dtype,
+                                    int nchunks, void *stream);
+
+/*
  * monarch_attn_fwd_profiled -- monarch_attn_fwd that also records CUDA events
  * on `stream` so a caller can time each kernel launch of the call:
  * events[0] before the first launch and events[i + 1] after launch i.

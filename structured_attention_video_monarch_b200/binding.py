@@ -52,6 +52,8 @@ def load_library(path: str | None = None):
                                               [vp, ctypes.POINTER(vp), i, ctypes.POINTER(i)])
     lib.monarch_attn_fwd_profiled.restype = i
     lib.monarch_attn_fwd_host.argtypes = [vp] * 8 + [i] * 10 + [vp]
+    lib.monarch_attn_fwd_host_pipelined.argtypes = [vp] * 8 + [i] * 11 + [vp]
+    lib.monarch_attn_fwd_host_pipelined.restype = i
     lib.monarch_attn_fwd_host.restype = i
     lib.monarch_attn_strerror.argtypes = [i]
     lib.monarch_attn_strerror.restype = ctypes.c_char_p
@@ -232,6 +234,20 @@ def monarch_attn_fwd_host(h_q, h_k, h_v, h_out, d_q, d_k, d_v, d_out, T, H, W,
     if st != 0:
         raise MonarchError(st, "monarch_attn_fwd_host")
     return h_out
+
+
+def monarch_attn_fwd_host_pipelined(h_q, h_k, h_v, h_out, d_q, d_k, d_v, d_out, T, H, W,
+                                    factorisation=FACT_FRAME, tile_h=0, tile_w=0, nchunks=4,
+                                    stream=None) -> None:
+    """monarch_attn_fwd_host with uploads, computation and downloads overlapped
+    over `nchunks` chunks of batch-heads (pinned host tensors for overlap)."""
+    B, heads, N, d = h_q.shape
+    st = load_library().monarch_attn_fwd_host_pipelined(
+        h_q.data_ptr(), h_k.data_ptr(), h_v.data_ptr(), h_out.data_ptr(), d_q.data_ptr(), d_k.data_ptr(),
+        d_v.data_ptr(), d_out.data_ptr(), B, heads, T, H, W, d, int(factorisation), int(tile_h),
+        int(tile_w), _dtype_code(h_q), int(nchunks), _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_host_pipelined")
 
 
 def last_device_error(reset: bool = True, stream=None) -> int:

@@ -17,6 +17,7 @@ LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libmonarch_attn.so")
 MAIN = os.path.join(CSRC, "monarch_attn.cu")
 BWD = os.path.join(CSRC, "monarch_bwd.cu")
+HOST = os.path.join(CSRC, "monarch_host.cu")
 
 
 def nvcc_path() -> str:
@@ -41,7 +42,7 @@ def up_to_date() -> bool:
 def nvcc_command(out: str, verbose: bool = False) -> list[str]:
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr",
-           "-o", out, MAIN, BWD]
+           "-o", out, MAIN, BWD, HOST]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     return cmd

@@ -1,0 +1,102 @@
+// monarch_host.cu -- monarch_attn_fwd_host_pipelined: the host-buffer entry
+// point with the copies overlapped with the computation (include/monarch_attn.h).
+//
+// The (batch, head) problems are independent, so the call splits them into
+// chunks of consecutive batch-heads ([B][heads][N][d] keeps each chunk
+// contiguous) and pipelines: the upload of chunk c+1 runs while chunk c is
+// computed and chunk c-1 is downloaded.  Uploads and downloads use two
+// streams of their own, so both copy directions run at once.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <initializer_list>
+#include <vector>
+
+#include "../../include/monarch_attn.h"
+
+namespace {
+
+struct Streams {
+    cudaStream_t up = nullptr, down = nullptr;
+    ~Streams() {
+        if (up) cudaStreamDestroy(up);
+        if (down) cudaStreamDestroy(down);
+    }
+};
+
+struct Events {
+    std::vector<cudaEvent_t> ev;
+    ~Events() {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+    }
+};
+
+}  // namespace
+
+extern "C" int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k, const void *h_v, void *h_out,
+                                               void *d_q, void *d_k, void *d_v, void *d_out, int B, int heads,
+                                               int T, int H, int W, int d, int factorisation, int tile_h,
+                                               int tile_w, int dtype, int nchunks, void *stream) {
+    if (!h_q || !h_k || !h_v || !h_out || !d_q || !d_k || !d_v || !d_out) return MONARCH_ERR_INVALID_ARG;
+    if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1 || nchunks < 1) return MONARCH_ERR_INVALID_ARG;
+    if (dtype != MONARCH_DTYPE_F32 && dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F16)
+        return MONARCH_ERR_INVALID_ARG;
+    const long long bh = static_cast<long long>(B) * heads;
+    const long long n = bh < nchunks ? bh : nchunks;
+    const size_t es = dtype == MONARCH_DTYPE_F32 ? 4 : 2;
+    const size_t per_bh = static_cast<size_t>(T) * H * W * d * es;
+    // each chunk's call validates its own slices; the whole output buffer may
+    // not overlap a whole input buffer either
+    const size_t total = static_cast<size_t>(bh) * per_bh;
+    const uintptr_t o = reinterpret_cast<uintptr_t>(d_out);
+    for (const void *in : {static_cast<const void *>(d_q), static_cast<const void *>(d_k),
+                           static_cast<const void *>(d_v)}) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(in);
+        if (x < o + total && o < x + total) return MONARCH_ERR_INVALID_ARG;
+    }
+    cudaStream_t compute = static_cast<cudaStream_t>(stream);
+    Streams s;
+    if (cudaStreamCreateWithFlags(&s.up, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&s.down, cudaStreamNonBlocking) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    Events e;
+    e.ev.assign(static_cast<size_t>(2 * n), nullptr);
+    for (cudaEvent_t &x : e.ev)
+        if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return MONARCH_ERR_CUDA;
+    // the computation must not start before earlier work on the caller's stream
+    // is done with the device buffers: uploads wait for it
+    cudaEvent_t start = nullptr;
+    if (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess) return MONARCH_ERR_CUDA;
+    e.ev.push_back(start);
+    if (cudaEventRecord(start, compute) != cudaSuccess || cudaStreamWaitEvent(s.up, start, 0) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    int st = MONARCH_OK;
+    for (long long c = 0; c < n && st == MONARCH_OK; ++c) {
+        const long long b0 = bh * c / n, b1 = bh * (c + 1) / n;
+        const size_t off = static_cast<size_t>(b0) * per_bh, bytes = static_cast<size_t>(b1 - b0) * per_bh;
+        auto dev = [&](void *p) { return static_cast<void *>(static_cast<uint8_t *>(p) + off); };
+        auto host = [&](const void *p) { return static_cast<const void *>(static_cast<const uint8_t *>(p) + off); };
+        cudaEvent_t in = e.ev[2 * c], out = e.ev[2 * c + 1];
+        if (cudaMemcpyAsync(dev(d_q), host(h_q), bytes, cudaMemcpyHostToDevice, s.up) != cudaSuccess ||
+            cudaMemcpyAsync(dev(d_k), host(h_k), bytes, cudaMemcpyHostToDevice, s.up) != cudaSuccess ||
+            cudaMemcpyAsync(dev(d_v), host(h_v), bytes, cudaMemcpyHostToDevice, s.up) != cudaSuccess ||
+            cudaEventRecord(in, s.up) != cudaSuccess || cudaStreamWaitEvent(compute, in, 0) != cudaSuccess) {
+            st = MONARCH_ERR_CUDA;
+            break;
+        }
+        // chunk c as its own call: batch 1, (b1 - b0) heads
+        st = monarch_attn_fwd(dev(d_q), dev(d_k), dev(d_v), dev(d_out), 1, static_cast<int>(b1 - b0), T, H, W, d,
+                              factorisation, tile_h, tile_w, dtype, compute);
+        if (st != MONARCH_OK) break;
+        if (cudaEventRecord(out, compute) != cudaSuccess || cudaStreamWaitEvent(s.down, out, 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<uint8_t *>(h_out) + off, dev(d_out), bytes, cudaMemcpyDeviceToHost,
+                            s.down) != cudaSuccess)
+            st = MONARCH_ERR_CUDA;
+    }
+    // the streams and events are released only after all queued work is done
+    const cudaError_t e1 = cudaStreamSynchronize(s.up), e2 = cudaStreamSynchronize(compute),
+                      e3 = cudaStreamSynchronize(s.down);
+    if (st == MONARCH_OK && (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)) st = MONARCH_ERR_CUDA;
+    return st;
+}

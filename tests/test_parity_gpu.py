@@ -211,6 +211,19 @@ def test_host_entry_point_matches_device_call():
     assert torch.equal(hout, ref)
 
 
+@pytest.mark.parametrize("nchunks", [1, 5, 12])
+def test_pipelined_host_entry_point_matches_device_call(nchunks):
+    wl = workloads.BY_NAME["chunk_bf16"]
+    q, k, v = workloads.generate(wl)
+    hq, hk, hv = (x.pin_memory() for x in (q, k, v))
+    hout = torch.full_like(hq, float("nan")).pin_memory()
+    dq, dk, dv, dout = (torch.empty_like(x, device=_dev()) for x in (q, k, v, q))
+    binding.monarch_attn_fwd_host_pipelined(hq, hk, hv, hout, dq, dk, dv, dout, wl.T, wl.H, wl.W,
+                                            nchunks=nchunks)
+    ref = binding.monarch_attn_fwd(q.to(_dev()), k.to(_dev()), v.to(_dev()), wl.T, wl.H, wl.W).cpu()
+    assert torch.equal(hout, ref)
+
+
 def test_invalid_arguments_are_rejected_without_launch():
     dev = _dev()
     x = torch.zeros(1, 1, 2 * 4 * 4, 128, dtype=torch.bfloat16, device=dev)
