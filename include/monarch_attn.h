@@ -141,8 +141,10 @@ int monarch_attn_fwd_host(const void *h_q, const void *h_k, const void *h_v, voi
  * independent; the call splits them into `nchunks` chunks of consecutive
  * batch-heads and pipelines them: chunk c+1 is uploaded while chunk c is
  * computed (on `stream`, one monarch_attn_fwd call per chunk) and chunk c-1
- * is downloaded.  Uploads and downloads run on two streams the call creates
- * and destroys; the first upload waits for work already queued on `stream`.
+ * is downloaded.  Uploads and downloads run on two streams the library
+ * creates on first use, one pair per device, and keeps (calls from several
+ * threads on one device share them); the first upload waits for work
+ * already queued on `stream`.
  * Results equal monarch_attn_fwd_host's bit for bit (each problem's
  * arithmetic does not depend on the chunking).  Host buffers must be pinned
  * for the copies to overlap.  nchunks >= 1 (capped at B*heads).  Arguments,

@@ -5,24 +5,46 @@
 // chunks of consecutive batch-heads ([B][heads][N][d] keeps each chunk
 // contiguous) and pipelines: the upload of chunk c+1 runs while chunk c is
 // computed and chunk c-1 is downloaded.  Uploads and downloads use two
-// streams of their own, so both copy directions run at once.
+// streams of their own (one pair per device, kept), so both copy directions
+// run at once.
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <initializer_list>
+#include <mutex>
 #include <vector>
 
 #include "../../include/monarch_attn.h"
 
 namespace {
 
-struct Streams {
+// Upload and download streams, created once per device and kept (creating
+// them costs about as much as a chunk's copy).  Calls from several host
+// threads on one device share them, which orders their copies but keeps
+// each call correct: every call waits only on its own events.
+struct CopyStreams {
     cudaStream_t up = nullptr, down = nullptr;
-    ~Streams() {
-        if (up) cudaStreamDestroy(up);
-        if (down) cudaStreamDestroy(down);
-    }
 };
+constexpr int kMaxDevices = 64;
+CopyStreams g_copy[kMaxDevices];
+std::mutex g_copy_mu;
+
+int copy_streams(CopyStreams *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_copy_mu);
+    CopyStreams &c = g_copy[dev];
+    if (!c.up && cudaStreamCreateWithFlags(&c.up, cudaStreamNonBlocking) != cudaSuccess) {
+        c.up = nullptr;
+        return MONARCH_ERR_CUDA;
+    }
+    if (!c.down && cudaStreamCreateWithFlags(&c.down, cudaStreamNonBlocking) != cudaSuccess) {
+        c.down = nullptr;
+        return MONARCH_ERR_CUDA;
+    }
+    *out = c;
+    return MONARCH_OK;
+}
 
 struct Events {
     std::vector<cudaEvent_t> ev;
@@ -56,10 +78,8 @@ extern "C" int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k,
         if (x < o + total && o < x + total) return MONARCH_ERR_INVALID_ARG;
     }
     cudaStream_t compute = static_cast<cudaStream_t>(stream);
-    Streams s;
-    if (cudaStreamCreateWithFlags(&s.up, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaStreamCreateWithFlags(&s.down, cudaStreamNonBlocking) != cudaSuccess)
-        return MONARCH_ERR_CUDA;
+    CopyStreams s;
+    if (copy_streams(&s) != MONARCH_OK) return MONARCH_ERR_CUDA;
     Events e;
     e.ev.assign(static_cast<size_t>(2 * n), nullptr);
     for (cudaEvent_t &x : e.ev)
@@ -94,7 +114,7 @@ extern "C" int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k,
                             s.down) != cudaSuccess)
             st = MONARCH_ERR_CUDA;
     }
-    // the streams and events are released only after all queued work is done
+    // the events are released only after all queued work is done
     const cudaError_t e1 = cudaStreamSynchronize(s.up), e2 = cudaStreamSynchronize(compute),
                       e3 = cudaStreamSynchronize(s.down);
     if (st == MONARCH_OK && (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)) st = MONARCH_ERR_CUDA;
