@@ -57,9 +57,10 @@ def _configure(lib):
     lib.oracle_monarch_fwd_groups.argtypes = (
         [dp, dp, dp] + [i] * 9 + [ctypes.POINTER(ctypes.c_long), i, dp])
     lib.oracle_monarch_bwd.argtypes = [dp] * 7 + [i] * 9
+    lib.oracle_monarch_fwd_chunk.argtypes = [dp] * 7 + [i] * 10
     for f in (lib.oracle_monarch_fwd, lib.oracle_monarch_stage1,
               lib.oracle_monarch_stage2, lib.oracle_monarch_fwd_groups,
-              lib.oracle_monarch_bwd, lib.oracle_num_threads):
+              lib.oracle_monarch_bwd, lib.oracle_monarch_fwd_chunk, lib.oracle_num_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -139,6 +140,27 @@ def monarch_bwd(q, k, v, dout, T, H, W, fact=FACT_FRAME, tile_h=0, tile_w=0):
     _check(_load().oracle_monarch_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
                                       _ptr(dv), B, heads, T, H, W, d, fact, tile_h, tile_w), "bwd")
     return dq, dk, dv
+
+
+def monarch_fwd_chunk(q, k, v, k_cache, y1_cache, T_old, T_new, H, W, fact=FACT_FRAME, tile_h=0,
+                      tile_w=0):
+    """Forward of a chunk of T_new new frames with T_old earlier frames as
+    context (their keys k_cache and stage-1 outputs y1_cache, [B, heads,
+    T_old*H*W, d]; None when T_old = 0).  Returns (out, y1_new) for the new
+    frames, float64."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, heads, d = _dims(q, T_new, H, W)
+    out, y1 = np.empty_like(q), np.empty_like(q)
+    if T_old > 0:
+        kc, yc = _as_f64(k_cache), _as_f64(y1_cache)
+        if kc.shape != (B, heads, T_old * H * W, d) or yc.shape != kc.shape:
+            raise ValueError("k_cache and y1_cache must be [B, heads, T_old*H*W, d]")
+        pk, py = _ptr(kc), _ptr(yc)
+    else:
+        pk = py = None
+    _check(_load().oracle_monarch_fwd_chunk(_ptr(q), _ptr(k), _ptr(v), pk, py, _ptr(out), _ptr(y1), B, heads,
+                                            T_old, T_new, H, W, d, fact, tile_h, tile_w), "fwd_chunk")
+    return out, y1
 
 
 def monarch_stage1(q, k, v, T, H, W, fact=FACT_FRAME, tile_h=0, tile_w=0) -> np.ndarray:

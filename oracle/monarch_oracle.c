@@ -459,3 +459,65 @@ int oracle_monarch_bwd(const double *q, const double *k, const double *v, const 
     free(dy1);
     return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------ autoregressive chunks
+ *
+ * The pages' main workload is an autoregressive few-step video model
+ * (gist.science/it/paper/2602.12271, problem statement: autoregressive
+ * generation), and their kernels process the query frames in chunks
+ * ("mini-sequence", gist.science/zh/paper/2602.12271, section 2.2).  Reading:
+ * a chunk of new frames is generated with the earlier frames as context.
+ * With the frame or tiled split, stage-1 blocks never cross frames, so the
+ * new chunk's stage 1 needs only its own frames; its stage 2 (the group of a
+ * spatial position) attends over the keys and stage-1 outputs of every frame
+ * so far.  So the context kept from earlier frames is their K and Y1 (their
+ * V is no longer needed).  For the last chunk this gives exactly the full
+ * forward's rows for those frames.
+ *
+ * q, k, v, out, y1_new: [B*heads][T_new*H*W][d] (the new frames);
+ * k_cache, y1_cache:    [B*heads][T_old*H*W][d] (may be NULL when T_old = 0). */
+int oracle_monarch_fwd_chunk(const double *q, const double *k, const double *v,
+                             const double *k_cache, const double *y1_cache,
+                             double *out, double *y1_new,
+                             int B, int heads, int T_old, int T_new, int H, int W, int d,
+                             int fact, int tile_h, int tile_w) {
+    if (fact == ORACLE_FACT_ROW || T_old < 0) return ORACLE_ERR_ARG; /* (f*h, w) groups are not per position */
+    int st = check_shape(B, heads, T_new, H, W, d, fact, tile_h, tile_w);
+    if (st) return st;
+    if (T_old > 0 && (!k_cache || !y1_cache)) return ORACLE_ERR_ARG;
+    st = oracle_monarch_stage1(q, k, v, y1_new, B, heads, T_new, H, W, d, fact, tile_h, tile_w);
+    if (st) return st;
+    long HW = (long)H * W, Nn = (long)T_new * HW, No = (long)T_old * HW;
+    long tot = (long)T_old + T_new;
+    double scale = 1.0 / sqrt((double)d);
+    int failed = 0;
+#pragma omp parallel
+    {
+        const double **kr = (const double **)malloc(sizeof(double *) * tot);
+        const double **vr = (const double **)malloc(sizeof(double *) * tot);
+        double *logit = (double *)malloc(sizeof(double) * tot);
+        if (!kr || !vr || !logit) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long w = 0; w < (long)B * heads * HW; ++w) {
+                long bh = w / HW, pos = w % HW;
+                for (long t = 0; t < T_old; ++t) {
+                    kr[t] = k_cache + (bh * No + t * HW + pos) * d;
+                    vr[t] = y1_cache + (bh * No + t * HW + pos) * d;
+                }
+                for (long t = 0; t < T_new; ++t) {
+                    kr[T_old + t] = k + (bh * Nn + t * HW + pos) * d;
+                    vr[T_old + t] = y1_new + (bh * Nn + t * HW + pos) * d;
+                }
+                for (long t = 0; t < T_new; ++t) {
+                    long row = (bh * Nn + t * HW + pos) * d;
+                    attend_one(q + row, kr, vr, tot, d, scale, logit, out + row);
+                }
+            }
+        }
+        free(kr); free(vr); free(logit);
+    }
+    return failed ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

@@ -142,3 +142,40 @@ def test_gradient_pins_catch_mutant(tmp_path, name, old, new):
     finally:
         oracle.restore_library(prev)
     assert caught, f"no gradient pin rejects the planted mistake '{name}'"
+
+
+# ---------------------------------------------------------------- autoregressive chunks
+
+import test_oracle_chunk as chunk_pins
+
+CHUNK_MUTANTS = [
+    ("chunk_cache_values_are_keys", "vr[t] = y1_cache + (bh * No + t * HW + pos) * d;",
+     "vr[t] = k_cache + (bh * No + t * HW + pos) * d;"),
+    ("chunk_new_values_are_v", "vr[T_old + t] = y1_new + (bh * Nn + t * HW + pos) * d;",
+     "vr[T_old + t] = v + (bh * Nn + t * HW + pos) * d;"),
+    ("chunk_context_dropped", "attend_one(q + row, kr, vr, tot, d, scale, logit, out + row);",
+     "attend_one(q + row, kr + T_old, vr + T_old, T_new, d, scale, logit, out + row);"),
+    ("chunk_cache_rows_frame_major_off_by_one", "kr[t] = k_cache + (bh * No + t * HW + pos) * d;",
+     "kr[t] = k_cache + (bh * No + ((t + 1) % T_old) * HW + pos) * d;"),
+]
+
+CHUNK_PROBES = [(f"chunk_case{i}", (lambda c=c: chunk_pins.test_last_chunk_equals_full_forward_rows(*c)))
+                for i, c in enumerate(chunk_pins.CASES)] + [
+    ("chunk_no_context", chunk_pins.test_no_context_is_the_plain_forward),
+]
+
+
+@pytest.mark.parametrize("name,old,new", CHUNK_MUTANTS, ids=[m[0] for m in CHUNK_MUTANTS])
+def test_chunk_pins_catch_mutant(tmp_path, name, old, new):
+    so = _build_mutant(tmp_path, name, old, new)
+    prev = oracle.use_library(so)
+    caught = []
+    try:
+        for label, fn in CHUNK_PROBES:
+            try:
+                fn()
+            except (AssertionError, ValueError, FloatingPointError):
+                caught.append(label)
+    finally:
+        oracle.restore_library(prev)
+    assert caught, f"no chunk pin rejects the planted mistake '{name}'"
