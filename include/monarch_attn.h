@@ -208,6 +208,39 @@ int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *
                              int factorisation, int tile_h, int tile_w, void *stream);
 
 /*
+ * monarch_attn_fwd_chunk -- one chunk of autoregressive generation: the
+ * forward of T_new new frames with the T_old frames before them as context.
+ * The pages' main model generates video autoregressively (gist.science/it/
+ * paper/2602.12271, problem statement) and their kernels split the query
+ * frames into chunks (gist.science/zh/paper/2602.12271, section 2.2); they
+ * define no cache.  Reading used here: stage 1 (frame or tiled blocks) never
+ * crosses frames, so it runs on the new frames alone; stage 2 of a new query
+ * at spatial position pos attends over the keys of all T_old + T_new frames
+ * at pos, with their stage-1 outputs as values.  So the context is the keys
+ * and stage-1 outputs of the earlier frames.  For the last chunk of a clip,
+ * with the context taken from a forward of the whole clip, `out` equals that
+ * forward's rows for those frames.
+ *
+ * q, k, v: the new frames, [B][heads][T_new*H*W][d] contiguous (as
+ * monarch_attn_fwd with T = T_new).  k_cache, y1_cache: keys and stage-1
+ * outputs of the context, [B][heads][T_old*H*W][d] contiguous, same dtype;
+ * ignored (may be NULL) when T_old = 0.  out: the chunk's output; y1_new:
+ * the stage-1 output of the new frames (to append to y1_cache for the next
+ * chunk, with k appended to k_cache); both [B][heads][T_new*H*W][d],
+ * written, previous contents ignored.  No output may overlap an input or the
+ * other output.  All pointers 16-byte aligned.  dtype, d, factorisation and
+ * tiles as monarch_attn_fwd (MONARCH_FACT_FRAME or _TILED); 1 <= T_new <=
+ * 128, T_old >= 0.  Two launches on `stream`: the forward's stage-1 kernel
+ * (tensor cores for bf16/fp16, CUDA cores for fp32), then a CUDA-core stage 2.
+ * Y1 is held in the input dtype.  Status codes as monarch_attn_fwd;
+ * MONARCH_ERR_INVALID_ARG also for T_old < 0 or missing context pointers.
+ */
+int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v,
+                           const void *k_cache, const void *y1_cache, void *out, void *y1_new,
+                           int B, int heads, int T_old, int T_new, int H, int W, int d,
+                           int factorisation, int tile_h, int tile_w, int dtype, void *stream);
+
+/*
  * monarch_attn_bwd -- gradients of out = P^T B2 P B1 V (as monarch_attn_fwd)
  * with respect to q, k and v for an upstream gradient dout.  The pages state
  * that their kernels run the backward pass too (gist.science/nl/paper/

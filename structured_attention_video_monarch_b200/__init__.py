@@ -13,7 +13,7 @@ used without loading the CUDA library.
 """
 
 __all__ = [
-    "monarch_attn_fwd", "monarch_attn_fwd_host", "MonarchError", "lib_path",
+    "monarch_attn_fwd", "monarch_attn_fwd_host", "monarch_attn_fwd_chunk", "MonarchError", "lib_path",
     "FACT_FRAME", "FACT_TILED", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16",
 ]
 
@@ -25,7 +25,7 @@ DTYPE_F16 = 2
 
 
 def __getattr__(name):
-    if name in ("monarch_attn_fwd", "monarch_attn_fwd_host", "MonarchError", "lib_path",
+    if name in ("monarch_attn_fwd", "monarch_attn_fwd_host", "monarch_attn_fwd_chunk", "MonarchError", "lib_path",
                 "load_library", "strerror", "last_device_error"):
         from . import binding
         return getattr(binding, name)

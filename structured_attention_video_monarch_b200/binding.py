@@ -71,6 +71,8 @@ def load_library(path: str | None = None):
     lib.monarch_attn_fwd_strided.restype = i
     lib.monarch_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp] + [i] * 9 + [vp]
     lib.monarch_attn_fwd_noalloc.restype = i
+    lib.monarch_attn_fwd_chunk.argtypes = [vp] * 7 + [i] * 11 + [vp]
+    lib.monarch_attn_fwd_chunk.restype = i
     lib.monarch_attn_version.argtypes = []
     lib.monarch_attn_version.restype = i
     if path == _build.LIB:
@@ -180,6 +182,41 @@ def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int =
     if st != 0:
         raise MonarchError(st, "monarch_attn_bwd")
     return dq, dk, dv
+
+
+def monarch_attn_fwd_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, k_cache, y1_cache,
+                           T_old: int, T_new: int, H: int, W: int, factorisation: int = FACT_FRAME,
+                           tile_h: int = 0, tile_w: int = 0, out=None, y1_new=None, stream=None):
+    """One autoregressive chunk: the forward of T_new new frames (q, k, v of shape
+    [B, heads, T_new*H*W, d]) with T_old context frames given by their keys and
+    stage-1 outputs (k_cache, y1_cache of shape [B, heads, T_old*H*W, d]; None
+    when T_old = 0).  Returns (out, y1_new); y1_new is the new frames' stage-1
+    output, to append to y1_cache for the next chunk.
+    """
+    ts = [q, k, v] + ([k_cache, y1_cache] if T_old > 0 else [])
+    if not all(t is not None and t.is_cuda and t.is_contiguous() for t in ts):
+        raise ValueError("q, k, v and the context must be contiguous CUDA tensors")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape or any(t.dtype != q.dtype for t in ts):
+        raise ValueError("q, k, v must share one [B, heads, N, d] shape and dtype")
+    B, heads, N, d = q.shape
+    if N != T_new * H * W:
+        raise ValueError(f"N={N} does not equal T_new*H*W={T_new * H * W}")
+    if T_old > 0 and (k_cache.shape != (B, heads, T_old * H * W, d) or y1_cache.shape != k_cache.shape):
+        raise ValueError("k_cache and y1_cache must be [B, heads, T_old*H*W, d]")
+    out = torch.empty_like(q) if out is None else out
+    y1_new = torch.empty_like(q) if y1_new is None else y1_new
+    for t in (out, y1_new):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("out and y1_new must be contiguous CUDA tensors shaped and typed like q")
+    kc = k_cache.data_ptr() if T_old > 0 else None
+    yc = y1_cache.data_ptr() if T_old > 0 else None
+    st = load_library().monarch_attn_fwd_chunk(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), kc, yc, out.data_ptr(), y1_new.data_ptr(), B, heads,
+        int(T_old), int(T_new), H, W, d, int(factorisation), int(tile_h), int(tile_w), _dtype_code(q),
+        _stream_ptr(stream))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_chunk")
+    return out, y1_new
 
 
 def monarch_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -1,0 +1,280 @@
+// attn_chunk.cuh -- stage 2 of an autoregressive chunk, on CUDA cores.
+//
+// A chunk of T_new new frames is computed with the T_old earlier frames as
+// context (MonarchRT: Efficient Attention for Real-Time Video Generation,
+// gist.science/it/paper/2602.12271, problem statement: autoregressive
+// generation; gist.science/zh/paper/2602.12271 section 2.2: query frames
+// processed in chunks).  Stage 1 of the new frames is the full forward's
+// stage 1 (its blocks never cross frames).  Stage 2 of a new query at spatial
+// position pos attends over the keys of all T_old + T_new frames at pos, with
+// their stage-1 outputs as values: frames [0, T_old) from k_cache / y1_cache,
+// the rest from k / y1_new.
+//
+// Per query this is a softmax over T_old + T_new keys: about 4 flops per
+// element of the 2 x d key/value elements it reads, so the kernel is bound by
+// HBM bandwidth and runs on CUDA cores.  One warp per (batch-head, position);
+// each lane owns C = d/32 consecutive features, so a row is one coalesced
+// 32-lane access; up to QG queries per pass share every key/value row loaded.
+// Accumulation, softmax and normalisation are fp32; exp2 of log2(e)-
+// prescaled logits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <cstring>
+#include <type_traits>
+
+namespace monarch {
+
+struct ChunkParams {
+    int HW;            // positions per frame
+    int T_old, T_new;  // context frames, new frames
+    long long n_old;   // context tokens per batch-head (T_old * HW)
+    long long n_new;   // new tokens per batch-head (T_new * HW)
+    long long groups;  // batch-heads x positions
+    float scale_log2;  // d^-1/2 * log2(e)
+};
+
+// Two 16-bit values packed in one word -> two floats.
+template <typename E>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+    if constexpr (std::is_same<E, __half>::value) {
+        __half2 h;
+        memcpy(&h, &w, 4);
+        return __half22float2(h);
+    } else {
+        __nv_bfloat162 h;
+        memcpy(&h, &w, 4);
+        return __bfloat1622float2(h);
+    }
+}
+
+template <typename E>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    uint32_t w;
+    if constexpr (std::is_same<E, __half>::value) {
+        const __half2 h = __floats2half2_rn(a, b);
+        memcpy(&w, &h, 4);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        memcpy(&w, &h, 4);
+    }
+    return w;
+}
+
+// Raw bytes of a lane's C consecutive elements of a row (4, 8 or 16 bytes),
+// loaded with one instruction and converted to fp32 only when used, so a
+// block's rows stay packed while their loads are in flight.
+template <int BYTES>
+struct RawOf;
+template <>
+struct RawOf<4> { using T = unsigned int; };
+template <>
+struct RawOf<8> { using T = uint2; };
+template <>
+struct RawOf<16> { using T = uint4; };
+template <typename E, int C>
+using RawRow = typename RawOf<C * static_cast<int>(sizeof(E))>::T;
+
+template <typename E, int C>
+__device__ __forceinline__ RawRow<E, C> raw_load(const E *p) {
+    return __ldg(reinterpret_cast<const RawRow<E, C> *>(p));
+}
+
+template <typename E, int C>
+__device__ __forceinline__ void raw_unpack(const RawRow<E, C> &r, float (&x)[C]) {
+    constexpr int NW = C * static_cast<int>(sizeof(E)) / 4;
+    uint32_t w[NW];
+    memcpy(w, &r, sizeof(w));
+    if constexpr (std::is_same<E, float>::value) {
+#pragma unroll
+        for (int i = 0; i < C; ++i) x[i] = __uint_as_float(w[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            const float2 f = unpack2<E>(w[i]);
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    }
+}
+
+template <typename E, int C>
+__device__ __forceinline__ void chunk_store(E *__restrict__ p, const float (&x)[C]) {
+    if constexpr (std::is_same<E, float>::value) {
+        if constexpr (C == 4)
+            *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+        else
+            *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    } else {
+        if constexpr (C == 4)
+            *reinterpret_cast<uint2 *>(p) = make_uint2(pack2<E>(x[0], x[1]), pack2<E>(x[2], x[3]));
+        else
+            *reinterpret_cast<unsigned int *>(p) = pack2<E>(x[0], x[1]);
+    }
+}
+
+// Sums NV (16 or 32) per-lane partial values over the warp so that lane l
+// ends with the full sum of value l % NV.  Each step exchanges only the half
+// of the values the partner keeps (a butterfly reduce-scatter): 31 shuffles
+// for 32 values instead of 5 per value.
+template <int NV>
+__device__ __forceinline__ void reduce_scatter(float (&v)[NV], int lane) {
+    static_assert(NV == 16 || NV == 32, "16 or 32 values");
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const int nb = NV < 2 * o ? NV : 2 * o;  // values still held
+        if (NV > o) {
+            const int h = nb / 2;
+            const bool up = (lane & o) != 0;  // keep the upper half
+#pragma unroll
+            for (int i = 0; i < h; ++i) {
+                const float send = up ? v[i] : v[i + h];
+                const float keep = up ? v[i + h] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < nb; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+        }
+    }
+}
+
+// All tensors [B*heads][tokens][D] contiguous: q, k, y1_new and out hold the
+// T_new new frames, k_cache and y1_cache the T_old context frames.
+//
+// Per pass of up to QG queries, keys go in blocks of KB: the block's key and
+// value rows are loaded first (2*KB loads in flight per lane), then its QG x
+// KB logits are reduced together, and the online softmax takes one step per
+// block (block maximum, one exp2 per lane, rescale once).
+template <int D, typename E>
+__global__ void __launch_bounds__(256, 2)
+monarch_chunk_stage2(const E *__restrict__ q, const E *__restrict__ k, const E *__restrict__ k_cache,
+                     const E *__restrict__ y1_cache, const E *__restrict__ y1_new, E *__restrict__ out,
+                     ChunkParams p) {
+    constexpr int C = D / 32, QG = 4;
+    constexpr int KB = sizeof(E) == 2 ? 8 : 4;  // keys per block
+    constexpr int NV = QG * KB;                 // logits per block
+    static_assert(C == 2 || C == 4, "d must be 64 or 128");
+    using Raw = RawRow<E, C>;
+    const long long g = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (g >= p.groups) return;  // whole warps leave together
+    const int lane = threadIdx.x & 31;
+    const long long bh = g / p.HW;
+    const int pos = static_cast<int>(g - bh * p.HW);
+    const long long fstride = static_cast<long long>(p.HW) * D;  // one frame
+    const long long base_new = (bh * p.n_new + pos) * D + lane * C;
+    const E *qb = q + base_new, *kn = k + base_new, *yn = y1_new + base_new;
+    E *ob = out + base_new;
+    // with no context the cache pointers are not used (and may be null)
+    const long long base_old = (bh * p.n_old + pos) * D + lane * C;
+    const E *kc = p.T_old ? k_cache + base_old : kn;
+    const E *yc = p.T_old ? y1_cache + base_old : yn;
+    const int T_tot = p.T_old + p.T_new;
+    // this lane's logit after the reduction: query ql, key ul of the block
+    const int ql = (lane % NV) / KB, ul = lane % KB;
+
+    for (int t0 = 0; t0 < p.T_new; t0 += QG) {
+        const int nq = p.T_new - t0 < QG ? p.T_new - t0 : QG;
+        float qx[QG][C], acc[QG][C], m[QG], l[QG];
+#pragma unroll
+        for (int qi = 0; qi < QG; ++qi) {
+            m[qi] = -INFINITY;
+            l[qi] = 0.f;
+#pragma unroll
+            for (int c = 0; c < C; ++c) acc[qi][c] = 0.f;
+            if (qi < nq) {
+                raw_unpack<E, C>(raw_load<E, C>(qb + (t0 + qi) * fstride), qx[qi]);
+#pragma unroll
+                for (int c = 0; c < C; ++c) qx[qi][c] *= p.scale_log2;
+            } else {
+#pragma unroll
+                for (int c = 0; c < C; ++c) qx[qi][c] = 0.f;
+            }
+        }
+        for (int j0 = 0; j0 < T_tot; j0 += KB) {
+            const int nk = T_tot - j0 < KB ? T_tot - j0 : KB;
+            Raw kr[KB], yr[KB];
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const int j = j0 + u;
+                if (u < nk) {
+                    const long long off = (j < p.T_old ? j : j - p.T_old) * fstride;
+                    kr[u] = raw_load<E, C>((j < p.T_old ? kc : kn) + off);
+                    yr[u] = raw_load<E, C>((j < p.T_old ? yc : yn) + off);
+                } else {
+                    kr[u] = Raw{};
+                    yr[u] = Raw{};
+                }
+            }
+            float v[NV];
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                float kx[C];
+                raw_unpack<E, C>(kr[u], kx);
+#pragma unroll
+                for (int qi = 0; qi < QG; ++qi) {
+                    float sacc = 0.f;
+#pragma unroll
+                    for (int c = 0; c < C; ++c) sacc = fmaf(qx[qi][c], kx[c], sacc);
+                    v[qi * KB + u] = sacc;
+                }
+            }
+            reduce_scatter<NV>(v, lane);
+            // padding queries get a finite logit (their results are dropped),
+            // padding keys weight 0
+            float s = v[0];
+            if (ql >= nq) s = 0.f;
+            else if (ul >= nk) s = -INFINITY;
+            float m_old = m[0];
+#pragma unroll
+            for (int qi = 1; qi < QG; ++qi)
+                if (ql == qi) m_old = m[qi];
+            float bm = s;
+#pragma unroll
+            for (int o = 1; o < KB; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const float mn = fmaxf(m_old, bm);
+            const float pe = exp2f(s - mn);
+            float bs = pe;
+#pragma unroll
+            for (int o = 1; o < KB; o <<= 1) bs += __shfl_xor_sync(0xffffffffu, bs, o);
+#pragma unroll
+            for (int qi = 0; qi < QG; ++qi) {
+                if (qi >= nq) break;  // the same for every lane
+                const float mq = __shfl_sync(0xffffffffu, mn, qi * KB);
+                const float sq = __shfl_sync(0xffffffffu, bs, qi * KB);
+                const float corr = exp2f(m[qi] - mq);
+                l[qi] = fmaf(l[qi], corr, sq);
+                m[qi] = mq;
+#pragma unroll
+                for (int c = 0; c < C; ++c) acc[qi][c] *= corr;
+            }
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                if (u >= nk) break;
+                float yx[C];
+                raw_unpack<E, C>(yr[u], yx);
+#pragma unroll
+                for (int qi = 0; qi < QG; ++qi) {
+                    if (qi >= nq) break;
+                    const float pq = __shfl_sync(0xffffffffu, pe, qi * KB + u);
+#pragma unroll
+                    for (int c = 0; c < C; ++c) acc[qi][c] = fmaf(pq, yx[c], acc[qi][c]);
+                }
+            }
+        }
+#pragma unroll
+        for (int qi = 0; qi < QG; ++qi) {
+            if (qi >= nq) break;
+            const float inv = 1.f / l[qi];
+            float o[C];
+#pragma unroll
+            for (int c = 0; c < C; ++c) o[c] = acc[qi][c] * inv;
+            chunk_store<E, C>(ob + (t0 + qi) * fstride, o);
+        }
+    }
+}
+
+}  // namespace monarch

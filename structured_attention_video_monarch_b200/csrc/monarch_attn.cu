@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "../../include/monarch_attn.h"
+#include "attn_chunk.cuh"
 #include "attn_f32.cuh"
 #include "attn_tc.cuh"
 
@@ -266,7 +267,8 @@ struct LaunchEvents {
 
 template <int D, bool F16>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
-              cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr) {
+              cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr,
+              bool stage1_only = false) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
@@ -311,6 +313,8 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     // stage-1 units per batch-head: blocks in pairs, each pair = the shared
     // query-tile pairs of both blocks plus one unit joining their odd tiles
     p.u1_bh = (p.nblk_bh / 2) * p.upg + (p.nblk_bh % 2) * (p.ns + p.odd);
+    // stage 1 alone (Y1 into `out`): no stage-2 units
+    if (stage1_only) p.s2_pairs = 0;
     const long long units = bh * (p.u1_bh + p.s2_pairs);
     if (units >= (1ll << 31) - 1) return MONARCH_ERR_UNSUPPORTED;
     p.units = static_cast<int>(units);
@@ -321,7 +325,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
         const long long wave = di->sms;
         long long lag = (2 * wave + p.u1_bh - 1) / p.u1_bh;
         if (lag < 1) lag = 1;
-        if (lag > bh) lag = bh;
+        if (lag > bh || stage1_only) lag = bh;
         p.lag = static_cast<int>(lag);
     }
     p.fd_u1 = make_fastdiv(static_cast<uint32_t>(p.u1_bh));
@@ -370,7 +374,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
 
 template <int D>
 int launch_f32(const void *q, const void *k, const void *v, void *out, const Shape &s,
-               cudaStream_t stream, LaunchEvents &lev) {
+               cudaStream_t stream, LaunchEvents &lev, bool stage1_only = false) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
@@ -410,8 +414,33 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
     monarch_f32_stage1<D><<<static_cast<unsigned>(g1), 128, 0, stream>>>(fq, fk, fv, fo, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
     lev.record(++lev.launches, stream);
+    if (stage1_only) return MONARCH_OK;
     const int threads2 = ((2 * s.T + 31) / 32) * 32;
     monarch_f32_stage2<D><<<static_cast<unsigned>(g2), threads2, smem2, stream>>>(fq, fk, fo, p);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    lev.record(++lev.launches, stream);
+    return MONARCH_OK;
+}
+
+// Stage 2 of an autoregressive chunk (attn_chunk.cuh): one warp per
+// (batch-head, position), 8 warps per block.
+template <int D, typename E>
+int launch_chunk_stage2(const void *q, const void *k, const void *k_cache, const void *y1_cache,
+                        const void *y1_new, void *out, const Shape &s, int T_old, cudaStream_t stream,
+                        LaunchEvents &lev) {
+    ChunkParams p{};
+    p.HW = s.H * s.W;
+    p.T_old = T_old;
+    p.T_new = s.T;
+    p.n_old = static_cast<long long>(T_old) * p.HW;
+    p.n_new = s.N;
+    p.groups = static_cast<long long>(s.B) * s.heads * p.HW;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    const long long blocks = (p.groups + 7) / 8;
+    if (blocks >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+    monarch_chunk_stage2<D, E><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const E *>(q), static_cast<const E *>(k), static_cast<const E *>(k_cache),
+        static_cast<const E *>(y1_cache), static_cast<const E *>(y1_new), static_cast<E *>(out), p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
     lev.record(++lev.launches, stream);
     return MONARCH_OK;
@@ -545,6 +574,62 @@ int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *
     LaunchEvents lev;
     st = d == 128 ? launch_tc<128, false>(q, k, v, out, s, cs, lev, counters)
                   : launch_tc<64, false>(q, k, v, out, s, cs, lev, counters);
+    if (st) return st;
+    if (env_debug()) return read_status(cs, 0);
+    return MONARCH_OK;
+}
+
+// One chunk of T_new new frames with T_old context frames: stage 1 of the new
+// frames into y1_new (the forward's kernels, stage 1 alone), then stage 2 of
+// the new queries over [k_cache; k] with values [y1_cache; y1_new].
+int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v, const void *k_cache,
+                           const void *y1_cache, void *out, void *y1_new, int B, int heads, int T_old,
+                           int T_new, int H, int W, int d, int factorisation, int tile_h, int tile_w,
+                           int dtype, void *stream) {
+    if (!out || T_old < 0) return MONARCH_ERR_INVALID_ARG;
+    if (T_old > 0 && (!k_cache || !y1_cache)) return MONARCH_ERR_INVALID_ARG;
+    Shape s{B, heads, T_new, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
+    int st = validate(q, k, v, y1_new, s);
+    if (st) return st;
+    const size_t es = dtype == MONARCH_DTYPE_F32 ? 4 : 2;
+    const long long n_old = static_cast<long long>(T_old) * H * W;
+    if (n_old > (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+    const size_t new_bytes = static_cast<size_t>(s.elems) * es;
+    const size_t old_bytes = static_cast<size_t>(B) * heads * n_old * d * es;
+    if (reinterpret_cast<uintptr_t>(out) % 16 != 0) return MONARCH_ERR_INVALID_ARG;
+    if (T_old > 0) {
+        for (const void *c : {k_cache, y1_cache})
+            if (reinterpret_cast<uintptr_t>(c) % 16 != 0) return MONARCH_ERR_INVALID_ARG;
+        // the outputs may not overlap the context
+        for (const void *o : {static_cast<const void *>(out), static_cast<const void *>(y1_new)})
+            for (const void *c : {k_cache, y1_cache}) {
+                const uintptr_t x = reinterpret_cast<uintptr_t>(o), y = reinterpret_cast<uintptr_t>(c);
+                if (x < y + old_bytes && y < x + new_bytes) return MONARCH_ERR_INVALID_ARG;
+            }
+    }
+    for (const void *x : {q, k, v, static_cast<const void *>(y1_new)})
+        if (overlaps(out, x, new_bytes)) return MONARCH_ERR_INVALID_ARG;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    LaunchEvents lev;
+    if (dtype == MONARCH_DTYPE_BF16) {
+        st = d == 128 ? launch_tc<128, false>(q, k, v, y1_new, s, cs, lev, nullptr, true)
+                      : launch_tc<64, false>(q, k, v, y1_new, s, cs, lev, nullptr, true);
+        if (!st)
+            st = d == 128 ? launch_chunk_stage2<128, __nv_bfloat16>(q, k, k_cache, y1_cache, y1_new, out, s, T_old, cs, lev)
+                          : launch_chunk_stage2<64, __nv_bfloat16>(q, k, k_cache, y1_cache, y1_new, out, s, T_old, cs, lev);
+    } else if (dtype == MONARCH_DTYPE_F16) {
+        st = d == 128 ? launch_tc<128, true>(q, k, v, y1_new, s, cs, lev, nullptr, true)
+                      : launch_tc<64, true>(q, k, v, y1_new, s, cs, lev, nullptr, true);
+        if (!st)
+            st = d == 128 ? launch_chunk_stage2<128, __half>(q, k, k_cache, y1_cache, y1_new, out, s, T_old, cs, lev)
+                          : launch_chunk_stage2<64, __half>(q, k, k_cache, y1_cache, y1_new, out, s, T_old, cs, lev);
+    } else {
+        st = d == 128 ? launch_f32<128>(q, k, v, y1_new, s, cs, lev, true)
+                      : launch_f32<64>(q, k, v, y1_new, s, cs, lev, true);
+        if (!st)
+            st = d == 128 ? launch_chunk_stage2<128, float>(q, k, k_cache, y1_cache, y1_new, out, s, T_old, cs, lev)
+                          : launch_chunk_stage2<64, float>(q, k, k_cache, y1_cache, y1_new, out, s, T_old, cs, lev);
+    }
     if (st) return st;
     if (env_debug()) return read_status(cs, 0);
     return MONARCH_OK;

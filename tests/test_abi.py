@@ -145,3 +145,31 @@ def test_bwd_workspace_size_and_validation_without_cuda(lib):
     n = ws // 2
     packed = [16 + i * n for i in range(7)]
     assert call(p=packed + [packed[6] + 16]) == 1
+
+
+def test_chunk_validation_without_cuda(lib):
+    big = 1 << 40
+    # q, k, v, k_cache, y1_cache, out, y1_new at disjoint fake addresses
+    ptrs = [16 + i * big for i in range(7)]
+
+    def call(p=ptrs, B=1, heads=1, T_old=2, T_new=2, H=4, W=4, d=128, fact=0, th=0, tw=0, dtype=1):
+        return lib.monarch_attn_fwd_chunk(*p, B, heads, T_old, T_new, H, W, d, fact, th, tw, dtype, None)
+
+    def swap(i, val):
+        p = list(ptrs)
+        p[i] = val
+        return p
+
+    assert call(T_old=-1) == 1                      # negative context length
+    assert call(p=swap(3, 0)) == 1                  # context keys missing
+    assert call(p=swap(4, 0)) == 1                  # context stage-1 outputs missing
+    assert call(p=swap(5, 0)) == 1                  # no out
+    assert call(p=swap(5, ptrs[5] + 8)) == 1        # out misaligned
+    assert call(p=swap(3, ptrs[3] + 8)) == 1        # context misaligned
+    assert call(p=swap(5, ptrs[6] + 16)) == 1       # out overlaps y1_new
+    assert call(p=swap(6, ptrs[4] + 64)) == 1       # y1_new overlaps the context
+    assert call(p=swap(5, ptrs[0] + 32)) == 1       # out overlaps q
+    assert call(fact=2) == 1                        # the (f*h, w) split has no chunk form
+    assert call(dtype=3) == 1
+    assert call(T_new=0) == 1
+    assert call(T_new=129) == 2                     # stage-1 launch limit
