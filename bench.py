@@ -52,7 +52,8 @@ def workload_config(wl, extra=None):
     cfg = {
         "workload": (f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} T={wl.T} H={wl.H} W={wl.W} "
                      f"(N={wl.N}), {'tiled ' + str(wl.tile_h) + 'x' + str(wl.tile_w) if wl.fact else 'frame'}"
-                     f" split m={wl.m} b={wl.b}"),
+                     f" split m={wl.m} b={wl.b}"
+                     + (f"; chunk of {wl.T} new frames after {wl.T_ctx} context frames" if wl.T_ctx else "")),
         "global_batch": wl.B,
         "seq_len": wl.N,
         "heads": wl.heads,
@@ -184,6 +185,31 @@ def oracle_sample(wl, seconds: float, seed: int = 1234):
     return q, k, v, groups, flops_per_group
 
 
+def oracle_chunk_sample(wl, seconds: float):
+    """Time the fp64 oracle's chunk form on whole heads of a chunk workload:
+    as many heads (one call each) as fit in about `seconds`.  Returns
+    (TFLOP/s, seconds, heads)."""
+    import oracle
+    from structured_attention_video_monarch_b200 import workloads
+    q, k, v = workloads.generate(wl, heads=1)
+    kc, yc = workloads.generate_context(wl, heads=1)
+    args = [x.double().numpy() for x in (q, k, v, kc, yc)]
+
+    def one():
+        oracle.monarch_fwd_chunk(*args, wl.T_ctx, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w)
+
+    t0 = time.perf_counter()
+    one()
+    dt1 = time.perf_counter() - t0
+    reps = max(1, min(wl.heads * wl.B, int(seconds / max(dt1, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        one()
+    dt = time.perf_counter() - t0
+    per_head = wl.flops / (wl.B * wl.heads)
+    return reps * per_head / dt / 1e12, dt, reps
+
+
 def time_oracle(wl, q, k, v, groups, flops_per_group):
     import oracle
     t0 = time.perf_counter()
@@ -201,6 +227,8 @@ def run_reference(args):
         return 0
     oracle.build()
     budget = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    if wl.T_ctx:
+        return run_reference_chunk(args, wl, budget)
     q, k, v, groups, fpg = oracle_sample(wl, budget)
     for _ in range(args.warmup):
         time_oracle(wl, q, k, v, groups, fpg)
@@ -225,27 +253,58 @@ def run_reference(args):
     return 0
 
 
+def run_reference_chunk(args, wl, budget):
+    import oracle
+    for _ in range(args.warmup):
+        oracle_chunk_sample(wl, budget)
+    total, flops, heads = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        val, dt, reps = oracle_chunk_sample(wl, budget)
+        total += dt
+        flops += val * dt * 1e12
+        heads = reps
+    value = flops / total / 1e12
+    sample = (f"{heads} head(s) of the chunk per step (exact stage 1 of the new frames and stage 2 "
+              f"over {wl.T_ctx}+{wl.T} frames)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, {"parallelism": "host cores (OpenMP)"}),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ our arm
 
-# The files the tensor-core kernel and its launch are built from.
-KERNEL_SOURCES = ("attn_tc.cuh", "monarch_attn.cu", "sm100.cuh")
+# The files each profiled kernel and its launch are built from.
+KERNEL_SOURCES = {
+    "monarch_tc_kernel": ("attn_tc.cuh", "monarch_attn.cu", "sm100.cuh"),
+    "monarch_chunk_stage2": ("attn_chunk.cuh", "monarch_attn.cu"),
+}
 
 
-def kernel_sources_sha256() -> str:
-    """Hash of the CUDA sources the dominant kernel is built from."""
+def kernel_sources_sha256(kernel: str = "monarch_tc_kernel") -> str:
+    """Hash of the CUDA sources a kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "structured_attention_video_monarch_b200", "csrc")
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         h.update(name.encode())
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def captured_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload,
-    or None when there is none or the kernel sources changed since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"monarch_tc_kernel_{workload}.md")
+def captured_traffic(workload: str, kernel: str = "monarch_tc_kernel"):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary of this
+    workload, or None when there is none or the kernel's sources changed since
+    it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -254,7 +313,7 @@ def captured_traffic(workload: str):
             key, sep, val = line.strip().partition(":")
             if sep and key in ("kernel_sources_sha256", "traffic_bytes_per_launch"):
                 fields[key] = val.strip()
-    if fields.get("kernel_sources_sha256") != kernel_sources_sha256():
+    if fields.get("kernel_sources_sha256") != kernel_sources_sha256(kernel):
         return None
     try:
         return float(fields["traffic_bytes_per_launch"])
@@ -279,6 +338,7 @@ def run_ours(args):
     wl = workloads.BY_NAME[args.workload]
     peaks, peak_src = load_peaks()
 
+    chunk = wl.T_ctx > 0  # autoregressive chunk: new frames plus a resident context
     q0, k0, v0 = workloads.generate(wl)
     nsets = 3
     sets = []
@@ -287,11 +347,23 @@ def run_ours(args):
             q, k, v = q0, k0, v0
         else:  # same distribution, different seed: distinct buffers so L2 holds none of them
             q, k, v = workloads.generate(wl, seed=wl.index + 100 * sidx)
-        sets.append(tuple(x.to(device) for x in (q, k, v)) + (torch.empty_like(q0, device=device),))
+        bufs = tuple(x.to(device) for x in (q, k, v)) + (torch.empty_like(q0, device=device),)
+        if chunk:
+            ctx = workloads.generate_context(wl, seed=1000 + wl.index + 100 * sidx)
+            bufs += tuple(x.to(device) for x in ctx) + (torch.empty_like(q0, device=device),)
+        sets.append(bufs)
     stream = torch.cuda.current_stream(device)
 
     def call(i, events=None):
-        q, k, v, o = sets[i % nsets]
+        if chunk:
+            q, k, v, o, kc, yc, y1 = sets[i % nsets]
+            if events is None:
+                binding.monarch_attn_fwd_chunk(q, k, v, kc, yc, wl.T_ctx, wl.T, wl.H, wl.W, wl.fact,
+                                               wl.tile_h, wl.tile_w, out=o, y1_new=y1)
+                return 2
+            return binding.monarch_attn_fwd_chunk_profiled(q, k, v, kc, yc, o, y1, wl.T_ctx, wl.T, wl.H,
+                                                           wl.W, events, wl.fact, wl.tile_h, wl.tile_w)
+        q, k, v, o = sets[i % nsets][:4]
         if events is None:
             binding.monarch_attn_fwd(q, k, v, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w, out=o)
             return 1
@@ -337,48 +409,100 @@ def run_ours(args):
     max_s = max_over_ranks(elapsed_s, device)
     value, ms = aggregate(world, wl.flops, args.steps, max_s)
 
-    # roofline of the dominant kernel: the bf16 call is one persistent kernel
-    # running both stages; its algorithmic work is the metric's 4*N*(m+b)*d
-    # FLOPs per (batch, head), timed per launch with events on this stream
-    kern_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    k_avg = statistics.mean(kern_ms) / 1e3
-    k_tflops = wl.flops / k_avg / 1e12
+    # roofline of the dominant kernel, timed per launch with events on this
+    # stream.  The forward is one persistent kernel running both stages; its
+    # algorithmic work is the metric's 4*N*(m+b)*d FLOPs per (batch, head).  A
+    # chunk is two launches: stage 1 of the new frames (tensor cores) and the
+    # stage 2 over context plus new frames (CUDA cores); each is rated
+    # against its own work and the slower one is reported as dominant.
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    io_bytes = wl.io_bytes
-    k_gbs = io_bytes / k_avg / 1e9
-    # the bound follows the workload's arithmetic intensity against the ridge
-    # point of the measured peaks (about 247 FLOP/B): the frame split is far
-    # above it (tensor cores), small tiles fall below it (HBM)
+    # the bound follows the arithmetic intensity against the ridge point of
+    # the measured peaks (about 247 FLOP/B): the frame split is far above it
+    # (tensor cores), small tiles and the chunk's stage 2 fall below it (HBM)
     ridge = peak * 1e12 / (hbm_peak * 1e9)
-    tensor_bound = wl.flops / io_bytes >= ridge
-    roofline = {
-        "bound": "tensor" if tensor_bound else "hbm",
-        "achieved": k_tflops if tensor_bound else k_gbs,
-        "peak": peak if tensor_bound else hbm_peak,
-        "unit": "TFLOP/s" if tensor_bound else "GB/s",
-        "frac": k_tflops / peak if tensor_bound else k_gbs / hbm_peak,
-        "traffic": args.traffic if args.traffic is not None else captured_traffic(wl.name),
-        "kernel": f"monarch_tc_kernel<{wl.d}> (both stages, one persistent launch)",
-        "peak_source": f"{peak_src} " + ("bf16_tflops (burst)" if tensor_bound else "hbm_gbs (copy)"),
-        "arithmetic_intensity_flop_per_byte": wl.flops / io_bytes,
-        "ridge_flop_per_byte": ridge,
-        "tflops": k_tflops,
-        "tensor_frac": k_tflops / peak,
-        "frac_of_sustained": k_tflops / peak_sus,
-        "algorithmic_flops_per_launch": wl.flops,
-        "launch_ms": k_avg * 1e3,
-        "algorithmic_bytes_per_launch": io_bytes,
-        "hbm_gbs_at_algorithmic_bytes": k_gbs,
-        "hbm_frac": k_gbs / hbm_peak,
-        "launches_per_call": per_call[0] if per_call else None,
-    }
+
+    def rate(kernel, label, launch_idx, flops, io_bytes):
+        k_avg = statistics.mean(ev[i][launch_idx].elapsed_time(ev[i][launch_idx + 1])
+                                for i in range(args.steps)) / 1e3
+        k_tflops = flops / k_avg / 1e12
+        k_gbs = io_bytes / k_avg / 1e9
+        tensor_bound = flops / io_bytes >= ridge
+        traffic = captured_traffic(wl.name, kernel)
+        if args.traffic is not None and launch_idx == 0 and not chunk:
+            traffic = args.traffic
+        return {
+            "bound": "tensor" if tensor_bound else "hbm",
+            "achieved": k_tflops if tensor_bound else k_gbs,
+            "peak": peak if tensor_bound else hbm_peak,
+            "unit": "TFLOP/s" if tensor_bound else "GB/s",
+            "frac": k_tflops / peak if tensor_bound else k_gbs / hbm_peak,
+            "traffic": traffic,
+            "kernel": label,
+            "peak_source": f"{peak_src} " + ("bf16_tflops (burst)" if tensor_bound else "hbm_gbs (copy)"),
+            "arithmetic_intensity_flop_per_byte": flops / io_bytes,
+            "ridge_flop_per_byte": ridge,
+            "tflops": k_tflops,
+            "tensor_frac": k_tflops / peak,
+            "frac_of_sustained": k_tflops / peak_sus,
+            "algorithmic_flops_per_launch": flops,
+            "launch_ms": k_avg * 1e3,
+            "algorithmic_bytes_per_launch": io_bytes,
+            "hbm_gbs_at_algorithmic_bytes": k_gbs,
+            "hbm_frac": k_gbs / hbm_peak,
+            "launches_per_call": per_call[0] if per_call else None,
+        }
+
+    if chunk:
+        es, bhd = 2, wl.B * wl.heads * wl.d
+        s1 = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (stage 1 of the {wl.T} new frames)", 0,
+                  4.0 * wl.N * wl.m * bhd, 4 * wl.N * bhd * es)
+        s2 = rate("monarch_chunk_stage2", f"monarch_chunk_stage2<{wl.d}> (stage 2 over {wl.T_ctx}+{wl.T} frames)",
+                  1, 4.0 * wl.N * wl.b * bhd, (4 * wl.N + 2 * wl.N_ctx) * bhd * es)
+        roofline, other = (s1, s2) if s1["launch_ms"] >= s2["launch_ms"] else (s2, s1)
+        roofline = dict(roofline, other_kernel=other)
+    else:
+        roofline = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (both stages, one persistent launch)",
+                        0, wl.flops, wl.io_bytes)
 
     # end to end through the host-buffer entry point: H2D of Q, K, V, the call, D2H of out,
     # with the copies overlapped with the computation over chunks of batch-heads
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and chunk:
+        # per chunk the host sends the new frames' Q, K, V and reads the output
+        # back; the context and y1_new stay on the device (the cache of an
+        # autoregressive loop lives in HBM)
+        hq, hk, hv = (x.pin_memory() for x in (q0, k0, v0))
+        hout = torch.empty_like(q0).pin_memory()
+        dq, dk, dv, dout, kc, yc, y1 = sets[0]
+
+        def e2e_call():
+            for h, d_ in ((hq, dq), (hk, dk), (hv, dv)):
+                d_.copy_(h, non_blocking=True)
+            binding.monarch_attn_fwd_chunk(dq, dk, dv, kc, yc, wl.T_ctx, wl.T, wl.H, wl.W, wl.fact,
+                                           wl.tile_h, wl.tile_w, out=dout, y1_new=y1)
+            hout.copy_(dout, non_blocking=True)
+
+        for _ in range(2):
+            e2e_call()
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_call()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
+        e2e_val, e2e_ms = aggregate(world, wl.flops, e2e_steps, e2e_s)
+        nbytes = q0.numel() * q0.element_size()
+        e2e = {"value": e2e_val, "unit": "TFLOP/s", "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "api": "monarch_attn_fwd_chunk with pinned host copies of Q, K, V in and out back "
+                      "(context resident on the device)"}
+    elif not args.no_e2e:
         hq, hk, hv = (x.pin_memory() for x in (q0, k0, v0))
         hout = torch.empty_like(q0).pin_memory()
         dq, dk, dv, dout = sets[0]
@@ -409,11 +533,16 @@ def run_ours(args):
         try:
             import oracle
             oracle.build()
-            qs, ks, vs, groups, fpg = oracle_sample(wl, args.cpu_seconds)
-            val, dt = time_oracle(wl, qs, ks, vs, groups, fpg)
+            if chunk:
+                val, dt, reps = oracle_chunk_sample(wl, args.cpu_seconds)
+                sample = f"{reps} head(s) of the chunk ({dt:.1f} s)"
+            else:
+                qs, ks, vs, groups, fpg = oracle_sample(wl, args.cpu_seconds)
+                val, dt = time_oracle(wl, qs, ks, vs, groups, fpg)
+                sample = (f"{len(groups)} stage-2 groups x {wl.T} rows of one head "
+                          f"({len(groups) * fpg / 1e9:.2f} GFLOP, {dt:.1f} s)")
             cpu = {"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-                   "sample": (f"{len(groups)} stage-2 groups x {wl.T} rows of one head "
-                              f"({len(groups) * fpg / 1e9:.2f} GFLOP, {dt:.1f} s)")}
+                   "sample": sample}
         except Exception as exc:  # the CPU baseline is a report, not the product
             cpu = {"value": None, "unit": "TFLOP/s", "cores": None, "kind": "oracle",
                    "sample": f"failed: {exc}"}
@@ -426,7 +555,9 @@ def run_ours(args):
             "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wl, {
                 "parallelism": f"replicas x{world} (independent (batch, head) problems; no collective)",
-                "l2": "inputs larger than L2: 3 rotating buffer sets of Q, K, V, out (1.2 GB)"}),
+                "l2": ("inputs larger than L2: 3 rotating buffer sets of Q, K, V, out, context K and Y1, "
+                       "y1_new" if chunk else
+                       "inputs larger than L2: 3 rotating buffer sets of Q, K, V, out (1.2 GB)")}),
             "pct_of_bf16_peak": {"measured_burst": value / world / peak,
                                  "measured_sustained": value / world / peak_sus,
                                  "datasheet_2250": value / world / 2250.0},

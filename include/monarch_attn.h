@@ -241,6 +241,20 @@ int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v,
                            int factorisation, int tile_h, int tile_w, int dtype, void *stream);
 
 /*
+ * monarch_attn_fwd_chunk_profiled -- monarch_attn_fwd_chunk recording CUDA
+ * events around its launches as monarch_attn_fwd_profiled does: events[0]
+ * before the first launch, events[i + 1] after launch i; *nlaunch receives 2
+ * (stage 1, then stage 2).  Same arguments, rules and status codes as
+ * monarch_attn_fwd_chunk otherwise.
+ */
+int monarch_attn_fwd_chunk_profiled(const void *q, const void *k, const void *v,
+                                    const void *k_cache, const void *y1_cache, void *out,
+                                    void *y1_new, int B, int heads, int T_old, int T_new, int H,
+                                    int W, int d, int factorisation, int tile_h, int tile_w,
+                                    int dtype, void *stream, void **events, int nevents,
+                                    int *nlaunch);
+
+/*
  * monarch_attn_bwd -- gradients of out = P^T B2 P B1 V (as monarch_attn_fwd)
  * with respect to q, k and v for an upstream gradient dout.  The pages state
  * that their kernels run the backward pass too (gist.science/nl/paper/

@@ -73,6 +73,9 @@ def load_library(path: str | None = None):
     lib.monarch_attn_fwd_noalloc.restype = i
     lib.monarch_attn_fwd_chunk.argtypes = [vp] * 7 + [i] * 11 + [vp]
     lib.monarch_attn_fwd_chunk.restype = i
+    lib.monarch_attn_fwd_chunk_profiled.argtypes = ([vp] * 7 + [i] * 11 +
+                                                    [vp, ctypes.POINTER(vp), i, ctypes.POINTER(i)])
+    lib.monarch_attn_fwd_chunk_profiled.restype = i
     lib.monarch_attn_version.argtypes = []
     lib.monarch_attn_version.restype = i
     if path == _build.LIB:
@@ -217,6 +220,25 @@ def monarch_attn_fwd_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, k_
     if st != 0:
         raise MonarchError(st, "monarch_attn_fwd_chunk")
     return out, y1_new
+
+
+def monarch_attn_fwd_chunk_profiled(q, k, v, k_cache, y1_cache, out, y1_new, T_old, T_new, H, W, events,
+                                    factorisation=FACT_FRAME, tile_h=0, tile_w=0, stream=None) -> int:
+    """monarch_attn_fwd_chunk into given ``out`` / ``y1_new``, recording ``events``
+    (torch.cuda.Event list) around each kernel launch.  Returns the number of
+    kernel launches queued."""
+    B, heads, N, d = q.shape
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    n = ctypes.c_int(0)
+    kc = k_cache.data_ptr() if T_old > 0 else None
+    yc = y1_cache.data_ptr() if T_old > 0 else None
+    st = load_library().monarch_attn_fwd_chunk_profiled(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), kc, yc, out.data_ptr(), y1_new.data_ptr(), B, heads,
+        int(T_old), int(T_new), H, W, d, int(factorisation), int(tile_h), int(tile_w), _dtype_code(q),
+        _stream_ptr(stream), arr, len(events), ctypes.byref(n))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_fwd_chunk_profiled")
+    return n.value
 
 
 def monarch_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -582,10 +582,9 @@ int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *
 // One chunk of T_new new frames with T_old context frames: stage 1 of the new
 // frames into y1_new (the forward's kernels, stage 1 alone), then stage 2 of
 // the new queries over [k_cache; k] with values [y1_cache; y1_new].
-int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v, const void *k_cache,
-                           const void *y1_cache, void *out, void *y1_new, int B, int heads, int T_old,
-                           int T_new, int H, int W, int d, int factorisation, int tile_h, int tile_w,
-                           int dtype, void *stream) {
+static int chunk_impl(const void *q, const void *k, const void *v, const void *k_cache, const void *y1_cache,
+                      void *out, void *y1_new, int B, int heads, int T_old, int T_new, int H, int W, int d,
+                      int factorisation, int tile_h, int tile_w, int dtype, void *stream, LaunchEvents &lev) {
     if (!out || T_old < 0) return MONARCH_ERR_INVALID_ARG;
     if (T_old > 0 && (!k_cache || !y1_cache)) return MONARCH_ERR_INVALID_ARG;
     Shape s{B, heads, T_new, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
@@ -610,7 +609,6 @@ int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v, const vo
     for (const void *x : {q, k, v, static_cast<const void *>(y1_new)})
         if (overlaps(out, x, new_bytes)) return MONARCH_ERR_INVALID_ARG;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    LaunchEvents lev;
     if (dtype == MONARCH_DTYPE_BF16) {
         st = d == 128 ? launch_tc<128, false>(q, k, v, y1_new, s, cs, lev, nullptr, true)
                       : launch_tc<64, false>(q, k, v, y1_new, s, cs, lev, nullptr, true);
@@ -633,6 +631,29 @@ int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v, const vo
     if (st) return st;
     if (env_debug()) return read_status(cs, 0);
     return MONARCH_OK;
+}
+
+int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v, const void *k_cache,
+                           const void *y1_cache, void *out, void *y1_new, int B, int heads, int T_old,
+                           int T_new, int H, int W, int d, int factorisation, int tile_h, int tile_w,
+                           int dtype, void *stream) {
+    LaunchEvents lev;
+    return chunk_impl(q, k, v, k_cache, y1_cache, out, y1_new, B, heads, T_old, T_new, H, W, d, factorisation,
+                      tile_h, tile_w, dtype, stream, lev);
+}
+
+int monarch_attn_fwd_chunk_profiled(const void *q, const void *k, const void *v, const void *k_cache,
+                                    const void *y1_cache, void *out, void *y1_new, int B, int heads,
+                                    int T_old, int T_new, int H, int W, int d, int factorisation,
+                                    int tile_h, int tile_w, int dtype, void *stream, void **events,
+                                    int nevents, int *nlaunch) {
+    LaunchEvents lev;
+    lev.ev = events;
+    lev.n = events ? nevents : 0;
+    const int st = chunk_impl(q, k, v, k_cache, y1_cache, out, y1_new, B, heads, T_old, T_new, H, W, d,
+                              factorisation, tile_h, tile_w, dtype, stream, lev);
+    if (nlaunch) *nlaunch = lev.launches;
+    return st;
 }
 
 const char *monarch_attn_strerror(int status) {

@@ -25,6 +25,11 @@ index, fp32 draws in the order Q, K, V, then extras, then cast):
   4 large_bf16    Q, K, V iid N(0,1); then randperm(N)[:5% of N] picks key
                   rows that are multiplied by 4 in every batch and head
                   (a stand-in for the sparse semantic outliers).
+  5 chunk_ar_bf16 the last chunk of a 21-frame clip generated
+                  autoregressively: Q, K, V of the 3 new frames iid N(0,1);
+                  the 18 context frames' keys and stage-1 outputs iid N(0,1),
+                  drawn by generate_context from a generator seeded
+                  1000 + index.
 """
 from __future__ import annotations
 
@@ -52,6 +57,7 @@ class Workload:
     tile_h: int = 0
     tile_w: int = 0
     extra: str = ""  # "scaled", "positional", "outliers" or ""
+    T_ctx: int = 0   # context frames before the chunk (autoregressive chunk workloads)
 
     @property
     def N(self) -> int:
@@ -65,9 +71,13 @@ class Workload:
         return self.H * self.W
 
     @property
+    def N_ctx(self) -> int:
+        return self.T_ctx * self.H * self.W
+
+    @property
     def b(self) -> int:
-        """Tokens per stage-2 group (one spatial position across frames)."""
-        return self.T
+        """Keys per stage-2 group (one spatial position across frames, context included)."""
+        return self.T + self.T_ctx
 
     @property
     def flops(self) -> float:
@@ -76,9 +86,11 @@ class Workload:
 
     @property
     def io_bytes(self) -> int:
-        """Minimum HBM bytes: read Q, K, V once, write O once."""
+        """Minimum HBM bytes: read Q, K, V once, write O once; a chunk also
+        reads the context's K and Y1 and writes the new frames' Y1."""
         es = 4 if self.dtype == "f32" else 2
-        return 4 * self.B * self.heads * self.N * self.d * es
+        rows = 4 * self.N + (self.N + 2 * self.N_ctx if self.T_ctx else 0)
+        return rows * self.B * self.heads * self.d * es
 
     def torch_dtype(self):
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
@@ -90,6 +102,7 @@ WORKLOADS = [
     Workload(2, "fullclip_bf16", 1, 12, 128, 21, 30, 52, "bf16", extra="positional"),
     Workload(3, "tiled_bf16", 1, 12, 128, 21, 30, 52, "bf16", FACT_TILED, 10, 13),
     Workload(4, "large_bf16", 2, 12, 128, 21, 45, 80, "bf16", extra="outliers"),
+    Workload(5, "chunk_ar_bf16", 1, 12, 128, 3, 30, 52, "bf16", T_ctx=18),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -149,3 +162,19 @@ def random_inputs(B, heads, T, H, W, d, dtype=torch.bfloat16, seed=0, scale=1.0)
         x = torch.randn(shape, generator=g, dtype=torch.float32) * scale
         out.append(x.to(dtype))
     return tuple(out)
+
+
+def generate_context(wl: Workload, seed: int | None = None, B: int | None = None,
+                     heads: int | None = None):
+    """Seeded context (K_ctx, Y1_ctx) of a chunk workload on the CPU, shape
+    [B, heads, T_ctx*H*W, d], workload dtype."""
+    seed = 1000 + wl.index if seed is None else seed
+    B = wl.B if B is None else B
+    heads = wl.heads if heads is None else heads
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    shape = (B, heads, wl.N_ctx, wl.d)
+    kc = torch.randn(shape, generator=g, dtype=torch.float32)
+    yc = torch.randn(shape, generator=g, dtype=torch.float32)
+    dt = wl.torch_dtype()
+    return kc.to(dt), yc.to(dt)

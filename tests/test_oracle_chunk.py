@@ -55,3 +55,17 @@ def test_rejects_the_row_split_and_bad_context():
         oracle.monarch_fwd_chunk(q, q, q, None, None, 0, 2, 2, 3, oracle.FACT_ROW)
     with pytest.raises(ValueError):
         oracle.monarch_fwd_chunk(q, q, q, q[:, :, :6], q, 1, 2, 2, 3)
+
+
+def test_chunk_workload_context_and_counts():
+    from structured_attention_video_monarch_b200 import workloads
+    wl = workloads.BY_NAME["chunk_ar_bf16"]
+    assert (wl.T, wl.T_ctx, wl.H, wl.W, wl.heads, wl.d) == (3, 18, 30, 52, 12, 128)
+    kc, yc = workloads.generate_context(wl, heads=1)
+    assert kc.shape == yc.shape == (1, 1, 18 * 30 * 52, 128)
+    kc2, _ = workloads.generate_context(wl, heads=1)
+    assert (kc.float() == kc2.float()).all()  # seeded
+    # per query: m stage-1 keys and T_ctx + T stage-2 keys, 4*d flops each
+    assert wl.flops == 4.0 * wl.N * (wl.H * wl.W + 21) * wl.d * wl.heads
+    # read Q, K, V and the context's K and Y1; write out and the new Y1
+    assert wl.io_bytes == (5 * wl.N + 2 * 18 * 30 * 52) * wl.heads * wl.d * 2
