@@ -422,8 +422,7 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
     return MONARCH_OK;
 }
 
-// Stage 2 of an autoregressive chunk (attn_chunk.cuh): one warp per
-// (batch-head, position), 8 warps per block.
+// Stage 2 of an autoregressive chunk (attn_chunk.cuh).
 template <int D, typename E>
 int launch_chunk_stage2(const void *q, const void *k, const void *k_cache, const void *y1_cache,
                         const void *y1_new, void *out, const Shape &s, int T_old, cudaStream_t stream,
@@ -436,12 +435,11 @@ int launch_chunk_stage2(const void *q, const void *k, const void *k_cache, const
     p.n_new = s.N;
     p.groups = static_cast<long long>(s.B) * s.heads * p.HW;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-    const long long blocks = (p.groups + 7) / 8;
-    if (blocks >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
-    monarch_chunk_stage2<D, E><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const E *>(q), static_cast<const E *>(k), static_cast<const E *>(k_cache),
-        static_cast<const E *>(y1_cache), static_cast<const E *>(y1_new), static_cast<E *>(out), p);
-    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    if (p.groups / ChunkCfg<D, E>::WARPS >= (1ll << 31) - 1) return MONARCH_ERR_UNSUPPORTED;
+    if (chunk_stage2_launch<D, E>(static_cast<const E *>(q), static_cast<const E *>(k),
+                                  static_cast<const E *>(k_cache), static_cast<const E *>(y1_cache),
+                                  static_cast<const E *>(y1_new), static_cast<E *>(out), p, stream) != cudaSuccess)
+        return MONARCH_ERR_LAUNCH;
     lev.record(++lev.launches, stream);
     return MONARCH_OK;
 }
