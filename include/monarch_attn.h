@@ -54,7 +54,9 @@ typedef enum {
  * block dimension). */
 typedef enum {
     MONARCH_FACT_FRAME = 0, /* block = one frame, m = H*W tokens, b = T blocks */
-    MONARCH_FACT_TILED = 1  /* block = one tile_h x tile_w spatial tile of one frame */
+    MONARCH_FACT_TILED = 1, /* block = one tile_h x tile_w spatial tile of one frame */
+    MONARCH_FACT_ROW = 2    /* the (f*h, w) split: block = one frame row (W tokens),
+                               group = one column (the T*H tokens sharing w) */
 } monarch_fact_t;
 
 /*
@@ -71,14 +73,23 @@ typedef enum {
  *   B, heads  batch size and head count, >= 1.
  *   T, H, W   frames, height and width of the token grid, >= 1.
  *   d         head width: 64 or 128.
- *   factorisation  MONARCH_FACT_FRAME or MONARCH_FACT_TILED.
+ *   factorisation  MONARCH_FACT_FRAME, MONARCH_FACT_TILED or MONARCH_FACT_ROW.
  *   tile_h, tile_w tile size for MONARCH_FACT_TILED; must divide H and W
- *             respectively.  Ignored for MONARCH_FACT_FRAME.
+ *             respectively.  Ignored otherwise.
+ *
+ * MONARCH_FACT_ROW is the (f*h, w) block alignment (gist.science/pt/paper/
+ * 2602.12271, "Alinhamento de Blocos"; gist.science/zh/paper/2602.12271,
+ * section 2.2): the tokens form a (T*H) x W grid, stage-1 blocks are its rows
+ * and stage-2 groups its columns.  It runs as two stage-1 passes of the
+ * forward's kernels and keeps the stage-1 result in a scratch buffer the
+ * library allocates per (device, stream) on first use (N*d elements per
+ * batch-head; a larger call drains the stream and reallocates), so `out` is
+ * written only by the second pass.
  *   dtype     MONARCH_DTYPE_BF16, MONARCH_DTYPE_F16 or MONARCH_DTYPE_F32.
  *   stream    cudaStream_t (NULL = legacy default stream) the work is queued on.
  *
- * Limits of this library version (MONARCH_ERR_UNSUPPORTED otherwise): T <= 128;
- * tile_w <= 128 for MONARCH_FACT_TILED; N <= 2^31; a device of compute
+ * Limits of this library version (MONARCH_ERR_UNSUPPORTED otherwise): T <= 128
+ * (except MONARCH_FACT_ROW); tile_w <= 128 for MONARCH_FACT_TILED; N <= 2^31; a device of compute
  * capability 10.0 (B200).  Pointers must be 16-byte aligned
  * (MONARCH_ERR_INVALID_ARG otherwise).
  *
@@ -111,7 +122,7 @@ int monarch_attn_fwd(const void *q, const void *k, const void *v, void *out,
  * stride must be at least the next smaller stride times its extent, and the
  * smallest at least d), or, for 16-bit dtypes, if a stride is not a multiple
  * of 8 elements (16 bytes); MONARCH_ERR_UNSUPPORTED for MONARCH_FACT_TILED
- * with strides other than the contiguous ones.
+ * and MONARCH_FACT_ROW with strides other than the contiguous ones.
  */
 int monarch_attn_fwd_strided(const void *q, const void *k, const void *v, void *out,
                              int B, int heads, int T, int H, int W, int d,

@@ -14,11 +14,12 @@ used without loading the CUDA library.
 
 __all__ = [
     "monarch_attn_fwd", "monarch_attn_fwd_host", "monarch_attn_fwd_chunk", "MonarchError", "lib_path",
-    "FACT_FRAME", "FACT_TILED", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16",
+    "FACT_FRAME", "FACT_TILED", "FACT_ROW", "DTYPE_F32", "DTYPE_BF16", "DTYPE_F16",
 ]
 
 FACT_FRAME = 0
 FACT_TILED = 1
+FACT_ROW = 2
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 DTYPE_F16 = 2

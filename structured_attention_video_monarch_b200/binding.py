@@ -16,6 +16,7 @@ from . import build as _build
 
 FACT_FRAME = 0
 FACT_TILED = 1
+FACT_ROW = 2
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 DTYPE_F16 = 2

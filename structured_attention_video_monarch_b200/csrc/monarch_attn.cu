@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -83,6 +84,42 @@ int device_info(DeviceInfo **out) {
 // Counter buffer of at least n elements for (current device, stream),
 // allocated on first use; when a call needs more, the stream is drained and
 // the buffer replaced.
+// Per (device, stream) scratch for the (f*h, w) split's stage-1 output,
+// allocated on first use and replaced (after draining the stream) when a call
+// needs more.
+struct ScratchBuf {
+    int dev;
+    cudaStream_t stream;
+    void *ptr;
+    size_t cap;
+};
+std::vector<ScratchBuf> g_scratch;
+
+int scratch_for(cudaStream_t stream, size_t bytes, void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    ScratchBuf *sb = nullptr;
+    for (auto &c : g_scratch)
+        if (c.dev == dev && c.stream == stream) sb = &c;
+    if (!sb) {
+        g_scratch.push_back(ScratchBuf{dev, stream, nullptr, 0});
+        sb = &g_scratch.back();
+    }
+    if (sb->cap < bytes) {
+        if (sb->ptr) {
+            if (cudaStreamSynchronize(stream) != cudaSuccess) return MONARCH_ERR_CUDA;
+            cudaFree(sb->ptr);
+            sb->ptr = nullptr;
+            sb->cap = 0;
+        }
+        if (cudaMalloc(&sb->ptr, bytes) != cudaSuccess) return MONARCH_ERR_CUDA;
+        sb->cap = bytes;
+    }
+    *out = sb->ptr;
+    return MONARCH_OK;
+}
+
 int counters_for(cudaStream_t stream, size_t n, unsigned **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MONARCH_ERR_CUDA;
@@ -162,7 +199,8 @@ int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
     if (s.d != 64 && s.d != 128) return MONARCH_ERR_INVALID_ARG;
     if (s.dtype != MONARCH_DTYPE_F32 && s.dtype != MONARCH_DTYPE_BF16 && s.dtype != MONARCH_DTYPE_F16)
         return MONARCH_ERR_INVALID_ARG;
-    if (s.fact != MONARCH_FACT_FRAME && s.fact != MONARCH_FACT_TILED) return MONARCH_ERR_INVALID_ARG;
+    if (s.fact != MONARCH_FACT_FRAME && s.fact != MONARCH_FACT_TILED && s.fact != MONARCH_FACT_ROW)
+        return MONARCH_ERR_INVALID_ARG;
     if (s.fact == MONARCH_FACT_TILED) {
         if (s.tile_h < 1 || s.tile_w < 1 || s.H % s.tile_h != 0 || s.W % s.tile_w != 0)
             return MONARCH_ERR_INVALID_ARG;
@@ -190,15 +228,16 @@ int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
         }
         // 16-bit paths read through TMA: strides must be 16-byte multiples
         if (s.dtype != MONARCH_DTYPE_F32 && (s.sB % 8 || s.sH % 8 || s.sN % 8)) return MONARCH_ERR_INVALID_ARG;
-        // the tiled factorisation's tensor map needs the contiguous layout
-        if (s.fact == MONARCH_FACT_TILED && (s.sB != cB || s.sH != cH || s.sN != cN))
+        // the tiled factorisation's tensor map (also used by the row split's
+        // column pass) needs the contiguous layout
+        if (s.fact != MONARCH_FACT_FRAME && (s.sB != cB || s.sH != cH || s.sN != cN))
             return MONARCH_ERR_UNSUPPORTED;
     }
     const long long span = (s.B - 1) * s.sB + (s.heads - 1) * s.sH + (s.N - 1) * s.sN + s.d;
     const size_t bytes = static_cast<size_t>(span) * (s.dtype == MONARCH_DTYPE_F32 ? 4 : 2);
     if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
         return MONARCH_ERR_INVALID_ARG;
-    if (s.T > 128) return MONARCH_ERR_UNSUPPORTED;
+    if (s.T > 128 && s.fact != MONARCH_FACT_ROW) return MONARCH_ERR_UNSUPPORTED;
     if (s.fact == MONARCH_FACT_TILED && s.tile_w > 128) return MONARCH_ERR_UNSUPPORTED;
     if (static_cast<long long>(s.B) * s.heads > (1ll << 30)) return MONARCH_ERR_UNSUPPORTED;
     return MONARCH_OK;
@@ -307,7 +346,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.ns = p.nqt / 2;
     p.odd = p.nqt % 2;
     p.upg = 2 * p.ns + p.odd;
-    p.npos = 128 / s.T;
+    p.npos = stage1_only ? 1 : 128 / s.T;  // stage 1 alone may run on more than 128 frames
     p.s2_chunks = (p.HW + p.npos - 1) / p.npos;
     p.s2_pairs = (p.s2_chunks + 1) / 2;
     // stage-1 units per batch-head: blocks in pairs, each pair = the shared
@@ -350,10 +389,14 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.status = status;
 
     CUtensorMap mq1, mk1, mv1, mq2, mk2, my2;
-    if ((st = stage1_map(&mq1, q, s, p)) || (st = stage1_map(&mk1, k, s, p)) ||
-        (st = stage1_map(&mv1, v, s, p)) || (st = stage2_map(&mq2, q, s, p)) ||
-        (st = stage2_map(&mk2, k, s, p)) || (st = stage2_map(&my2, out, s, p)))
+    if ((st = stage1_map(&mq1, q, s, p)) || (st = stage1_map(&mk1, k, s, p)) || (st = stage1_map(&mv1, v, s, p)))
         return st;
+    if (stage1_only) {  // no stage-2 units read them
+        mq2 = mq1; mk2 = mk1; my2 = mv1;
+    } else if ((st = stage2_map(&mq2, q, s, p)) || (st = stage2_map(&mk2, k, s, p)) ||
+               (st = stage2_map(&my2, out, s, p))) {
+        return st;
+    }
 
     // One persistent launch runs both stages: stage-1 units write Y1 = B1 V
     // into out; stage-2 units overwrite it in place with P^T B2 P Y1 once the
@@ -420,6 +463,33 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
     lev.record(++lev.launches, stream);
     return MONARCH_OK;
+}
+
+// The (f*h, w) split: tokens form a (T*H) x W grid; stage-1 blocks are its
+// rows (the W tokens of one frame row), stage-2 groups its columns (the T*H
+// tokens sharing w).  Both are stage-1 passes of the forward's kernels over
+// virtual shapes of the same [B][heads][N][d] tensors (token n = r*W + w):
+//   rows:    T*H frames of 1 x W, frame split          -> Y1 into the scratch
+//   columns: one frame of (T*H) x W, tiles (T*H) x 1   -> out, values = Y1
+template <int D, typename E>
+int launch_row(const void *q, const void *k, const void *v, void *out, const Shape &s, cudaStream_t stream,
+               LaunchEvents &lev) {
+    void *y1 = nullptr;
+    int st = scratch_for(stream, static_cast<size_t>(s.elems) * sizeof(E), &y1);
+    if (st) return st;
+    Shape rows = s;
+    rows.T = s.T * s.H; rows.H = 1; rows.fact = MONARCH_FACT_FRAME; rows.tile_h = rows.tile_w = 0;
+    Shape cols = s;
+    cols.T = 1; cols.H = s.T * s.H; cols.fact = MONARCH_FACT_TILED; cols.tile_h = s.T * s.H; cols.tile_w = 1;
+    constexpr bool tc = !std::is_same<E, float>::value;
+    if constexpr (tc) {
+        constexpr bool f16 = std::is_same<E, __half>::value;
+        if ((st = launch_tc<D, f16>(q, k, v, y1, rows, stream, lev, nullptr, true))) return st;
+        return launch_tc<D, f16>(q, k, y1, out, cols, stream, lev, nullptr, true);
+    } else {
+        if ((st = launch_f32<D>(q, k, v, y1, rows, stream, lev, true))) return st;
+        return launch_f32<D>(q, k, y1, out, cols, stream, lev, true);
+    }
 }
 
 // Stage 2 of an autoregressive chunk (attn_chunk.cuh).
@@ -489,7 +559,17 @@ static int fwd_impl(const void *q, const void *k, const void *v, void *out, int 
     int st = validate(q, k, v, out, s);
     if (st) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (dtype == MONARCH_DTYPE_BF16)
+    if (factorisation == MONARCH_FACT_ROW) {
+        if (dtype == MONARCH_DTYPE_BF16)
+            st = d == 128 ? launch_row<128, __nv_bfloat16>(q, k, v, out, s, cs, lev)
+                          : launch_row<64, __nv_bfloat16>(q, k, v, out, s, cs, lev);
+        else if (dtype == MONARCH_DTYPE_F16)
+            st = d == 128 ? launch_row<128, __half>(q, k, v, out, s, cs, lev)
+                          : launch_row<64, __half>(q, k, v, out, s, cs, lev);
+        else
+            st = d == 128 ? launch_row<128, float>(q, k, v, out, s, cs, lev)
+                          : launch_row<64, float>(q, k, v, out, s, cs, lev);
+    } else if (dtype == MONARCH_DTYPE_BF16)
         st = d == 128 ? launch_tc<128, false>(q, k, v, out, s, cs, lev) : launch_tc<64, false>(q, k, v, out, s, cs, lev);
     else if (dtype == MONARCH_DTYPE_F16)
         st = d == 128 ? launch_tc<128, true>(q, k, v, out, s, cs, lev) : launch_tc<64, true>(q, k, v, out, s, cs, lev);
@@ -566,6 +646,7 @@ int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *
     int st = validate(q, k, v, out, s);
     if (st) return st;
     if (static_cast<long long>(B) * heads > MONARCH_NOALLOC_MAX_BH) return MONARCH_ERR_UNSUPPORTED;
+    if (factorisation == MONARCH_FACT_ROW) return MONARCH_ERR_UNSUPPORTED;  // needs the Y1 scratch
     unsigned *counters = nullptr;
     if ((st = noalloc_counters(&counters))) return st;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -584,6 +665,7 @@ static int chunk_impl(const void *q, const void *k, const void *v, const void *k
                       void *out, void *y1_new, int B, int heads, int T_old, int T_new, int H, int W, int d,
                       int factorisation, int tile_h, int tile_w, int dtype, void *stream, LaunchEvents &lev) {
     if (!out || T_old < 0) return MONARCH_ERR_INVALID_ARG;
+    if (factorisation == MONARCH_FACT_ROW) return MONARCH_ERR_INVALID_ARG;  // groups are not per position
     if (T_old > 0 && (!k_cache || !y1_cache)) return MONARCH_ERR_INVALID_ARG;
     Shape s{B, heads, T_new, H, W, d, factorisation, tile_h, tile_w, dtype, 0, 0};
     int st = validate(q, k, v, y1_new, s);

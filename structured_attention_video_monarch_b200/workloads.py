@@ -30,6 +30,8 @@ index, fp32 draws in the order Q, K, V, then extras, then cast):
                   the 18 context frames' keys and stage-1 outputs iid N(0,1),
                   drawn by generate_context from a generator seeded
                   1000 + index.
+  6 fullclip_row_bf16  the full-clip grid under the (f*h, w) split; Q, K, V
+                  iid N(0,1).
 """
 from __future__ import annotations
 
@@ -40,6 +42,7 @@ import torch
 
 FACT_FRAME = 0
 FACT_TILED = 1
+FACT_ROW = 2
 
 
 @dataclasses.dataclass(frozen=True)
@@ -68,6 +71,8 @@ class Workload:
         """Tokens per stage-1 block."""
         if self.fact == FACT_TILED:
             return self.tile_h * self.tile_w
+        if self.fact == FACT_ROW:
+            return self.W
         return self.H * self.W
 
     @property
@@ -76,7 +81,10 @@ class Workload:
 
     @property
     def b(self) -> int:
-        """Keys per stage-2 group (one spatial position across frames, context included)."""
+        """Keys per stage-2 group: one spatial position across frames (context
+        included), or for the (f*h, w) split one column across frames and rows."""
+        if self.fact == FACT_ROW:
+            return self.T * self.H
         return self.T + self.T_ctx
 
     @property
@@ -103,6 +111,7 @@ WORKLOADS = [
     Workload(3, "tiled_bf16", 1, 12, 128, 21, 30, 52, "bf16", FACT_TILED, 10, 13),
     Workload(4, "large_bf16", 2, 12, 128, 21, 45, 80, "bf16", extra="outliers"),
     Workload(5, "chunk_ar_bf16", 1, 12, 128, 3, 30, 52, "bf16", T_ctx=18),
+    Workload(6, "fullclip_row_bf16", 1, 12, 128, 21, 30, 52, "bf16", FACT_ROW),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 

@@ -61,7 +61,7 @@ def _call(lib, q=16, k=32, v=48, out=4096, B=1, heads=1, T=2, H=4, W=4, d=128, f
     dict(B=0), dict(heads=0), dict(T=0), dict(H=0), dict(W=-1),
     dict(d=96), dict(d=256),        # unsupported head width
     dict(dtype=3),                  # unknown dtype
-    dict(fact=2),                   # unknown factorisation
+    dict(fact=3),                   # unknown factorisation
     dict(fact=1, th=3, tw=2),       # tile does not divide H
     dict(fact=1, th=2, tw=0),
     dict(q=18),                     # misaligned (not 16-byte aligned)
@@ -113,8 +113,15 @@ def test_strided_validation_without_cuda(lib):
     assert _strided(lib, heads * N * d, N * d, d - 8) == 1   # token rows overlap
     assert _strided(lib, heads * N * d, d, d) == 1           # heads and tokens overlap
     assert _strided(lib, heads * N * d, N * d + 4, d) == 1   # not a 16-byte multiple (bf16)
-    # the tiled factorisation keeps the contiguous layout
+    # the tiled factorisation and the (f*h, w) split keep the contiguous layout
     assert _strided(lib, N * heads * d, d, heads * d, fact=1, th=2, tw=2) == 2
+    assert _strided(lib, N * heads * d, d, heads * d, fact=2) == 2
+
+
+def test_noalloc_refuses_the_row_split_without_cuda(lib):
+    big = 1 << 40
+    # the (f*h, w) split needs the library's Y1 scratch: refused before any CUDA call
+    assert lib.monarch_attn_fwd_noalloc(16, big, 2 * big, 3 * big, 1, 1, 2, 4, 4, 128, 2, 0, 0, None) == 2
 
 
 def test_bwd_workspace_size_and_validation_without_cuda(lib):
