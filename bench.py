@@ -51,7 +51,8 @@ def load_peaks():
 def workload_config(wl, extra=None):
     cfg = {
         "workload": (f"{wl.name}: B={wl.B} heads={wl.heads} d={wl.d} T={wl.T} H={wl.H} W={wl.W} "
-                     f"(N={wl.N}), {'tiled ' + str(wl.tile_h) + 'x' + str(wl.tile_w) if wl.fact else 'frame'}"
+                     f"(N={wl.N}), "
+                     f"{('frame', 'tiled ' + str(wl.tile_h) + 'x' + str(wl.tile_w), '(f*h, w)')[wl.fact]}"
                      f" split m={wl.m} b={wl.b}"
                      + (f"; chunk of {wl.T} new frames after {wl.T_ctx} context frames" if wl.T_ctx else "")),
         "global_batch": wl.B,
@@ -210,6 +211,30 @@ def oracle_chunk_sample(wl, seconds: float):
     return reps * per_head / dt / 1e12, dt, reps
 
 
+def oracle_head_sample(wl, seconds: float):
+    """Time the fp64 oracle's full forward on whole heads (for the (f*h, w)
+    split, whose column groups span every frame, so no exact sampled-group
+    form exists): as many heads (one call each) as fit in about `seconds`.
+    Returns (TFLOP/s, seconds, heads)."""
+    import oracle
+    from structured_attention_video_monarch_b200 import workloads
+    q, k, v = (x.double().numpy() for x in workloads.generate(wl, heads=1))
+
+    def one():
+        oracle.monarch_fwd(q, k, v, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w)
+
+    t0 = time.perf_counter()
+    one()
+    dt1 = time.perf_counter() - t0
+    reps = max(1, min(wl.heads * wl.B, int(seconds / max(dt1, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        one()
+    dt = time.perf_counter() - t0
+    per_head = wl.flops / (wl.B * wl.heads)
+    return reps * per_head / dt / 1e12, dt, reps
+
+
 def time_oracle(wl, q, k, v, groups, flops_per_group):
     import oracle
     t0 = time.perf_counter()
@@ -227,8 +252,8 @@ def run_reference(args):
         return 0
     oracle.build()
     budget = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
-    if wl.T_ctx:
-        return run_reference_chunk(args, wl, budget)
+    if wl.T_ctx or wl.fact == workloads.FACT_ROW:
+        return run_reference_heads(args, wl, budget)
     q, k, v, groups, fpg = oracle_sample(wl, budget)
     for _ in range(args.warmup):
         time_oracle(wl, q, k, v, groups, fpg)
@@ -253,19 +278,25 @@ def run_reference(args):
     return 0
 
 
-def run_reference_chunk(args, wl, budget):
+def run_reference_heads(args, wl, budget):
+    """Reference arm for workloads the oracle times by whole heads: an
+    autoregressive chunk, or the (f*h, w) split."""
     import oracle
+    sampler = oracle_chunk_sample if wl.T_ctx else oracle_head_sample
     for _ in range(args.warmup):
-        oracle_chunk_sample(wl, budget)
+        sampler(wl, budget)
     total, flops, heads = 0.0, 0.0, 0
     for _ in range(args.steps):
-        val, dt, reps = oracle_chunk_sample(wl, budget)
+        val, dt, reps = sampler(wl, budget)
         total += dt
         flops += val * dt * 1e12
         heads = reps
     value = flops / total / 1e12
-    sample = (f"{heads} head(s) of the chunk per step (exact stage 1 of the new frames and stage 2 "
-              f"over {wl.T_ctx}+{wl.T} frames)")
+    if wl.T_ctx:
+        sample = (f"{heads} head(s) of the chunk per step (exact stage 1 of the new frames and stage 2 "
+                  f"over {wl.T_ctx}+{wl.T} frames)")
+    else:
+        sample = f"{heads} head(s) of the full forward per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -282,21 +313,30 @@ def run_reference_chunk(args, wl, budget):
 
 # ------------------------------------------------------------------ our arm
 
-# The files each profiled kernel and its launch are built from.
+# The sources each profiled kernel and its launch are built from: whole files,
+# or "file#region" for the text between "// <region>" and "// </region>".
 KERNEL_SOURCES = {
-    "monarch_tc_kernel": ("attn_tc.cuh", "monarch_attn.cu", "sm100.cuh"),
-    "monarch_chunk_stage2": ("attn_chunk.cuh", "monarch_attn.cu"),
+    "monarch_tc_kernel": ("attn_tc.cuh", "sm100.cuh", "monarch_attn.cu#tc-launch"),
+    "monarch_chunk_stage2": ("attn_chunk.cuh", "monarch_attn.cu#chunk-launch"),
 }
 
 
 def kernel_sources_sha256(kernel: str = "monarch_tc_kernel") -> str:
-    """Hash of the CUDA sources a kernel is built from."""
+    """Hash of the CUDA sources a kernel and its launch are built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "structured_attention_video_monarch_b200", "csrc")
-    for name in KERNEL_SOURCES[kernel]:
-        h.update(name.encode())
+    for spec in KERNEL_SOURCES[kernel]:
+        name, _, region = spec.partition("#")
         with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+            text = f.read()
+        if region:
+            begin, end = f"// <{region}>".encode(), f"// </{region}>".encode()
+            i, j = text.find(begin), text.find(end)
+            if i < 0 or j < i:
+                raise ValueError(f"region {region} not found in {name}")
+            text = text[i:j]
+        h.update(spec.encode())
+        h.update(text)
     return h.hexdigest()
 
 
@@ -339,6 +379,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
 
     chunk = wl.T_ctx > 0  # autoregressive chunk: new frames plus a resident context
+    row = wl.fact == workloads.FACT_ROW  # (f*h, w) split: a rows pass, then a columns pass
     q0, k0, v0 = workloads.generate(wl)
     nsets = 3
     sets = []
@@ -454,7 +495,18 @@ def run_ours(args):
             "launches_per_call": per_call[0] if per_call else None,
         }
 
-    if chunk:
+    if row:
+        es, bhd = 2, wl.B * wl.heads * wl.d
+        r1 = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (rows pass: blocks of W={wl.W} tokens)", 0,
+                  4.0 * wl.N * wl.W * bhd, 4 * wl.N * bhd * es)
+        r2 = rate("monarch_tc_kernel",
+                  f"monarch_tc_kernel<{wl.d}> (columns pass: groups of T*H={wl.T * wl.H} tokens)", 1,
+                  4.0 * wl.N * wl.T * wl.H * bhd, 4 * wl.N * bhd * es)
+        # one kernel, two launches: a single ncu summary cannot give both traffics
+        r1["traffic"] = r2["traffic"] = None
+        roofline, other = (r1, r2) if r1["launch_ms"] >= r2["launch_ms"] else (r2, r1)
+        roofline = dict(roofline, other_kernel=other)
+    elif chunk:
         es, bhd = 2, wl.B * wl.heads * wl.d
         s1 = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (stage 1 of the {wl.T} new frames)", 0,
                   4.0 * wl.N * wl.m * bhd, 4 * wl.N * bhd * es)
@@ -533,9 +585,10 @@ def run_ours(args):
         try:
             import oracle
             oracle.build()
-            if chunk:
-                val, dt, reps = oracle_chunk_sample(wl, args.cpu_seconds)
-                sample = f"{reps} head(s) of the chunk ({dt:.1f} s)"
+            if chunk or row:
+                sampler = oracle_chunk_sample if chunk else oracle_head_sample
+                val, dt, reps = sampler(wl, args.cpu_seconds)
+                sample = f"{reps} head(s) of the {'chunk' if chunk else 'full forward'} ({dt:.1f} s)"
             else:
                 qs, ks, vs, groups, fpg = oracle_sample(wl, args.cpu_seconds)
                 val, dt = time_oracle(wl, qs, ks, vs, groups, fpg)

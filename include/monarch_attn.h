@@ -176,7 +176,8 @@ int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k, const void
  * (entries beyond what the call needs are left untouched; NULL entries are
  * skipped).  *nlaunch (if not NULL) receives the number of kernel launches
  * the call queued: 1 for bf16 and fp16 (both stages in one persistent
- * kernel), 2 for fp32 (stage 1, then stage 2).  Same arguments, rules and status codes as
+ * kernel), 2 for fp32 (stage 1, then stage 2), and 2 for MONARCH_FACT_ROW in
+ * every dtype (the rows pass, then the columns pass).  Same arguments, rules and status codes as
  * monarch_attn_fwd otherwise.
  */
 int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void *out,

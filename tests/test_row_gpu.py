@@ -83,3 +83,16 @@ def test_row_split_repeat_and_second_stream():
     s.synchronize()
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_row_split_profiled_events_bracket_each_pass():
+    # events[0] before the rows pass, events[1] between the passes, events[2] after
+    q, k, v = (x.cuda() for x in _inputs((1, 2, 3 * 4 * 20, 128), torch.bfloat16, seed=10))
+    out = torch.empty_like(q)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for e in ev:
+        e.record()
+    n = binding.monarch_attn_fwd_profiled(q, k, v, out, 3, 4, 20, ev, ROW)
+    torch.cuda.synchronize()
+    assert n == 2
+    assert ev[0].elapsed_time(ev[1]) > 0 and ev[1].elapsed_time(ev[2]) > 0
