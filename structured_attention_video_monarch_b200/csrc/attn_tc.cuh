@@ -192,13 +192,10 @@ template <int NP>
 __device__ __forceinline__ void s1_load(const TcParams &p, const CUtensorMap *map, uint32_t dst,
                                         uint32_t bar, int blk, int tile) {
     if (p.fact == 0) {
-#pragma unroll
-        {
-            // map (d, m, T, heads, B): block blk = bh * T + t
-            const int bh = static_cast<int>(fdiv(blk, p.fd_nblk_bh)), t = blk - bh * p.nblk_bh;
-            const int b = static_cast<int>(fdiv(bh, p.fd_heads)), hd = bh - b * p.heads;
-            for (int pn = 0; pn < NP; ++pn) tma_load_5d(dst + pn * 16384, map, bar, pn * 64, tile * 128, t, hd, b);
-        }
+        // map (d, m, T, heads, B): block blk = bh * T + t
+        const int bh = static_cast<int>(fdiv(blk, p.fd_nblk_bh)), t = blk - bh * p.nblk_bh;
+        const int b = static_cast<int>(fdiv(bh, p.fd_heads)), hd = bh - b * p.heads;
+        for (int pn = 0; pn < NP; ++pn) tma_load_5d(dst + pn * 16384, map, bar, pn * 64, tile * 128, t, hd, b);
     } else {
         const int frame = static_cast<int>(fdiv(blk, p.fd_tpf));
         const int tif = blk - frame * p.tiles_h * p.tiles_w;
