@@ -485,8 +485,12 @@ def run_ours(args):
     ridge = peak * 1e12 / (hbm_peak * 1e9)
 
     def rate(kernel, label, launch_idx, flops, io_bytes):
-        k_avg = statistics.mean(ev[i][launch_idx].elapsed_time(ev[i][launch_idx + 1])
-                                for i in range(args.steps)) / 1e3
+        per = sorted(ev[i][launch_idx].elapsed_time(ev[i][launch_idx + 1]) for i in range(args.steps))
+        k_avg = statistics.mean(per) / 1e3
+
+        def pct(f):  # nearest-rank percentile of the per-launch times, ms
+            return per[min(len(per) - 1, max(0, int(round(f * (len(per) - 1)))))]
+
         k_tflops = flops / k_avg / 1e12
         k_gbs = io_bytes / k_avg / 1e9
         tensor_bound = flops / io_bytes >= ridge
@@ -509,6 +513,7 @@ def run_ours(args):
             "frac_of_sustained": k_tflops / peak_sus,
             "algorithmic_flops_per_launch": flops,
             "launch_ms": k_avg * 1e3,
+            "launch_ms_p10_p50_p90": [pct(0.1), pct(0.5), pct(0.9)],
             "algorithmic_bytes_per_launch": io_bytes,
             "hbm_gbs_at_algorithmic_bytes": k_gbs,
             "hbm_frac": k_gbs / hbm_peak,
