@@ -3,8 +3,11 @@
     out = P^T B2 P B1 V
 
 over a video token grid N = T*H*W: stage 1 is softmax attention inside each
-frame (or spatial tile of a frame), stage 2 is softmax attention across frames
-at each spatial position, applied to stage 1's output.  Every step runs in
+frame (or spatial tile of a frame, or frame row for the (f*h, w) split),
+stage 2 is softmax attention across frames at each spatial position (or down
+each column), applied to stage 1's output.  Also: one autoregressive chunk of
+new frames against cached keys and stage-1 outputs (``monarch_attn_fwd_chunk``)
+and fp32 gradients (``binding.monarch_attn_bwd``).  Every step runs in
 hand-written sm_100a CUDA kernels behind a C ABI (``include/monarch_attn.h``);
 this package is the thin ctypes binding over it.
 
