@@ -484,7 +484,11 @@ def run_ours(args):
     # (tensor cores), small tiles and the chunk's stage 2 fall below it (HBM)
     ridge = peak * 1e12 / (hbm_peak * 1e9)
 
-    def rate(kernel, label, launch_idx, flops, io_bytes):
+    # FP32 FMA peak from unit counts and the boost clock: 148 SMs x 128 lanes x 2 FLOP
+    # x 1.965 GHz (nothing measured applies to CUDA-core FFMA work)
+    alu_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+
+    def rate(kernel, label, launch_idx, flops, io_bytes, alu=False):
         per = sorted(ev[i][launch_idx].elapsed_time(ev[i][launch_idx + 1]) for i in range(args.steps))
         k_avg = statistics.mean(per) / 1e3
 
@@ -497,15 +501,24 @@ def run_ours(args):
         traffic = captured_traffic(wl.name, kernel)
         if args.traffic is not None and launch_idx == 0 and not chunk:
             traffic = args.traffic
+        if alu:
+            bound, achieved, pk, unit = "alu", k_tflops, alu_peak, "TFLOP/s"
+            src = "derived FP32 FMA peak (148 SMs x 128 lanes x 2 x max SM clock)"
+        elif tensor_bound:
+            bound, achieved, pk, unit = "tensor", k_tflops, peak, "TFLOP/s"
+            src = f"{peak_src} bf16_tflops (burst)"
+        else:
+            bound, achieved, pk, unit = "hbm", k_gbs, hbm_peak, "GB/s"
+            src = f"{peak_src} hbm_gbs (copy)"
         return {
-            "bound": "tensor" if tensor_bound else "hbm",
-            "achieved": k_tflops if tensor_bound else k_gbs,
-            "peak": peak if tensor_bound else hbm_peak,
-            "unit": "TFLOP/s" if tensor_bound else "GB/s",
-            "frac": k_tflops / peak if tensor_bound else k_gbs / hbm_peak,
+            "bound": bound,
+            "achieved": achieved,
+            "peak": pk,
+            "unit": unit,
+            "frac": achieved / pk,
             "traffic": traffic,
             "kernel": label,
-            "peak_source": f"{peak_src} " + ("bf16_tflops (burst)" if tensor_bound else "hbm_gbs (copy)"),
+            "peak_source": src,
             "arithmetic_intensity_flop_per_byte": flops / io_bytes,
             "ridge_flop_per_byte": ridge,
             "tflops": k_tflops,
@@ -538,6 +551,15 @@ def run_ours(args):
         s2 = rate("monarch_chunk_stage2", f"monarch_chunk_stage2<{wl.d}> (stage 2 over {wl.T_ctx}+{wl.T} frames)",
                   1, 4.0 * wl.N * wl.b * bhd, (4 * wl.N + 2 * wl.N_ctx) * bhd * es)
         roofline, other = (s1, s2) if s1["launch_ms"] >= s2["launch_ms"] else (s2, s1)
+        roofline = dict(roofline, other_kernel=other)
+    elif wl.dtype == "f32":
+        # the exact path: stage 1 and stage 2 are separate CUDA-core launches
+        es, bhd = 4, wl.B * wl.heads * wl.d
+        f1 = rate("monarch_f32_stage1", f"monarch_f32_stage1<{wl.d}> (stage 1, CUDA cores)", 0,
+                  4.0 * wl.N * wl.m * bhd, 4 * wl.N * bhd * es, alu=True)
+        f2 = rate("monarch_f32_stage2", f"monarch_f32_stage2<{wl.d}> (stage 2, CUDA cores)", 1,
+                  4.0 * wl.N * wl.b * bhd, 4 * wl.N * bhd * es, alu=True)
+        roofline, other = (f1, f2) if f1["launch_ms"] >= f2["launch_ms"] else (f2, f1)
         roofline = dict(roofline, other_kernel=other)
     else:
         roofline = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (both stages, one persistent launch)",
@@ -630,7 +652,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic",
+            "dtype": wl.dtype, "data": "synthetic",
             "config": workload_config(wl, {
                 "parallelism": f"replicas x{world} (independent (batch, head) problems; no collective)",
                 "l2": ("inputs larger than L2: 3 rotating buffer sets of Q, K, V, out, context K and Y1, "
