@@ -340,6 +340,17 @@ def kernel_sources_sha256(kernel: str = "monarch_tc_kernel") -> str:
     return h.hexdigest()
 
 
+def traffic_source(workload: str, kernel: str = "monarch_tc_kernel") -> str:
+    """Where roofline.traffic comes from, or why it is null."""
+    rel = os.path.join("profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(os.path.join(ROOT, rel)):
+        return "none: no ncu summary for this kernel and workload"
+    if captured_traffic(workload, kernel) is None:
+        return (f"none: {rel} was taken on earlier sources (its kernel_sources_sha256 does not match "
+                "the current ones), so its DRAM counters are not reported")
+    return f"{rel} (dram__bytes_read.sum + dram__bytes_write.sum of one launch)"
+
+
 def captured_traffic(workload: str, kernel: str = "monarch_tc_kernel"):
     """DRAM bytes per launch of `kernel` from the committed ncu summary of this
     workload, or None when there is none or the kernel's sources changed since
@@ -499,8 +510,9 @@ def run_ours(args):
         k_gbs = io_bytes / k_avg / 1e9
         tensor_bound = flops / io_bytes >= ridge
         traffic = captured_traffic(wl.name, kernel)
+        t_src = traffic_source(wl.name, kernel)
         if args.traffic is not None and launch_idx == 0 and not chunk:
-            traffic = args.traffic
+            traffic, t_src = args.traffic, "--traffic argument"
         if alu:
             bound, achieved, pk, unit = "alu", k_tflops, alu_peak, "TFLOP/s"
             src = "derived FP32 FMA peak (148 SMs x 128 lanes x 2 x max SM clock)"
@@ -517,6 +529,7 @@ def run_ours(args):
             "unit": unit,
             "frac": achieved / pk,
             "traffic": traffic,
+            "traffic_source": t_src,
             "kernel": label,
             "peak_source": src,
             "arithmetic_intensity_flop_per_byte": flops / io_bytes,
@@ -542,6 +555,7 @@ def run_ours(args):
                   4.0 * wl.N * wl.T * wl.H * bhd, 4 * wl.N * bhd * es)
         # one kernel, two launches: a single ncu summary cannot give both traffics
         r1["traffic"] = r2["traffic"] = None
+        r1["traffic_source"] = r2["traffic_source"] = "none: no per-pass ncu summary for this split"
         roofline, other = (r1, r2) if r1["launch_ms"] >= r2["launch_ms"] else (r2, r1)
         roofline = dict(roofline, other_kernel=other)
     elif chunk:

@@ -86,3 +86,19 @@ def test_reference_arm_line_for_the_chunk_workload():
     assert line["cpu_baseline"]["kind"] == "oracle" and "head(s) of the chunk" in line["cpu_baseline"]["sample"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert "context frames" in line["config"]["workload"]
+
+
+def test_traffic_source_explains_a_null_traffic(tmp_path, monkeypatch):
+    csrc = tmp_path / "structured_attention_video_monarch_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    (csrc / "k.cuh").write_text("kernel\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setitem(bench.KERNEL_SOURCES, "kern", ("k.cuh",))
+    assert bench.traffic_source("wl", "kern").startswith("none: no ncu summary")
+    h = bench.kernel_sources_sha256("kern")
+    (tmp_path / "profiles" / "kern_wl.md").write_text(
+        f"    kernel_sources_sha256: {h}\n    traffic_bytes_per_launch: 5\n")
+    assert bench.traffic_source("wl", "kern").startswith("profiles/kern_wl.md")
+    (csrc / "k.cuh").write_text("kernel changed\n")
+    assert "earlier sources" in bench.traffic_source("wl", "kern")
