@@ -180,3 +180,18 @@ def test_chunk_validation_without_cuda(lib):
     assert call(dtype=3) == 1
     assert call(T_new=0) == 1
     assert call(T_new=129) == 2                     # stage-1 launch limit
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: the header must compile as strict C99 (and as C++)
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "monarch_attn.h"\nint main(void) { return monarch_attn_version() > 0 ? 0 : 1; }\n')
+    inc = os.path.dirname(HEADER)
+    for cmd in ([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-I", inc, str(src)],
+                [gcc, "-x", "c++", "-std=c++11", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, str(src)]):
+        out = subprocess.run(cmd, capture_output=True, text=True)
+        assert out.returncode == 0, out.stderr
