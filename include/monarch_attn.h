@@ -202,7 +202,8 @@ int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void 
  * monarch_attn_fwd with dtype = MONARCH_DTYPE_BF16.  Scratch: the per-batch-
  * head completion counters live in one static device array per device of
  * MONARCH_NOALLOC_MAX_BH words; B*heads above that returns
- * MONARCH_ERR_UNSUPPORTED before anything is queued.  Those counters must be
+ * MONARCH_ERR_UNSUPPORTED before anything is queued, and so does
+ * MONARCH_FACT_ROW (its stage-1 result needs the library's scratch buffer).  Those counters must be
  * zero when the kernel starts; every call zeroes them with a cudaMemsetAsync
  * on `stream` ahead of its launch.  The first call on each device does a
  * one-time set-up on the host (the array's address, the kernel's shared-
