@@ -135,3 +135,17 @@ def test_sampled_group_mode_refuses_the_row_split():
     q = _rand((1, 1, 12, 4), 1)
     with pytest.raises(ValueError):
         oracle.monarch_fwd_groups(q, q, q, 2, 2, 3, [(0, 0)], ROW)
+
+
+@pytest.mark.parametrize("T,H,W", [(2, 3, 5), (3, 4, 2), (1, 6, 7)])
+def test_row_split_is_the_frame_split_of_the_row_grid(T, H, W):
+    # the (f*h, w) split of a T x H x W grid is the frame split of a (T*H) x 1 x W
+    # grid: its blocks (frame rows) are those frames, its groups (columns) those positions
+    d = 6
+    q, k, v = (_rand((1, 2, T * H * W, d), s) for s in (91, 92, 93))
+    np.testing.assert_allclose(oracle.monarch_fwd(q, k, v, T, H, W, oracle.FACT_ROW),
+                               oracle.monarch_fwd(q, k, v, T * H, 1, W, oracle.FACT_FRAME), rtol=0, atol=1e-14)
+    g = _rand((1, 2, T * H * W, d), 94)
+    for a, b in zip(oracle.monarch_bwd(q, k, v, g, T, H, W, oracle.FACT_ROW),
+                    oracle.monarch_bwd(q, k, v, g, T * H, 1, W, oracle.FACT_FRAME)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
