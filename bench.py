@@ -235,6 +235,30 @@ def oracle_head_sample(wl, seconds: float):
     return reps * per_head / dt / 1e12, dt, reps
 
 
+def oracle_bwd_sample(wl, seconds: float):
+    """Time the fp64 gradient oracle on whole heads of a gradient workload:
+    as many heads (one call each) as fit in about `seconds`.  Returns
+    (TFLOP/s, seconds, heads)."""
+    import oracle
+    from structured_attention_video_monarch_b200 import workloads
+    q, k, v = (x.double().numpy() for x in workloads.generate(wl, heads=1))
+    do = workloads.generate_upstream(wl, heads=1).double().numpy()
+
+    def one():
+        oracle.monarch_bwd(q, k, v, do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w)
+
+    t0 = time.perf_counter()
+    one()
+    dt1 = time.perf_counter() - t0
+    reps = max(1, min(wl.heads * wl.B, int(seconds / max(dt1, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        one()
+    dt = time.perf_counter() - t0
+    per_head = wl.flops / (wl.B * wl.heads)
+    return reps * per_head / dt / 1e12, dt, reps
+
+
 def time_oracle(wl, q, k, v, groups, flops_per_group):
     import oracle
     t0 = time.perf_counter()
@@ -252,7 +276,7 @@ def run_reference(args):
         return 0
     oracle.build()
     budget = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
-    if wl.T_ctx or wl.fact == workloads.FACT_ROW:
+    if wl.T_ctx or wl.grad or wl.fact == workloads.FACT_ROW:
         return run_reference_heads(args, wl, budget)
     q, k, v, groups, fpg = oracle_sample(wl, budget)
     for _ in range(args.warmup):
@@ -282,7 +306,7 @@ def run_reference_heads(args, wl, budget):
     """Reference arm for workloads the oracle times by whole heads: an
     autoregressive chunk, or the (f*h, w) split."""
     import oracle
-    sampler = oracle_chunk_sample if wl.T_ctx else oracle_head_sample
+    sampler = oracle_chunk_sample if wl.T_ctx else (oracle_bwd_sample if wl.grad else oracle_head_sample)
     for _ in range(args.warmup):
         sampler(wl, budget)
     total, flops, heads = 0.0, 0.0, 0
@@ -295,6 +319,8 @@ def run_reference_heads(args, wl, budget):
     if wl.T_ctx:
         sample = (f"{heads} head(s) of the chunk per step (exact stage 1 of the new frames and stage 2 "
                   f"over {wl.T_ctx}+{wl.T} frames)")
+    elif wl.grad:
+        sample = f"{heads} head(s) of the fp64 gradients (dQ, dK, dV) per step"
     else:
         sample = f"{heads} head(s) of the full forward per step"
     line = {
@@ -389,6 +415,7 @@ def run_ours(args):
     wl = workloads.BY_NAME[args.workload]
     peaks, peak_src = load_peaks()
 
+    grad = wl.grad        # gradients: dQ, dK, dV of an upstream dO (fp32 path)
     chunk = wl.T_ctx > 0  # autoregressive chunk: new frames plus a resident context
     row = wl.fact == workloads.FACT_ROW  # (f*h, w) split: a rows pass, then a columns pass
     q0, k0, v0 = workloads.generate(wl)
@@ -403,10 +430,23 @@ def run_ours(args):
         if chunk:
             ctx = workloads.generate_context(wl, seed=1000 + wl.index + 100 * sidx)
             bufs += tuple(x.to(device) for x in ctx) + (torch.empty_like(q0, device=device),)
+        if grad:
+            do = workloads.generate_upstream(wl, seed=2000 + wl.index + 100 * sidx).to(device)
+            bufs += (do, torch.empty_like(q0, device=device), torch.empty_like(q0, device=device),
+                     binding.monarch_attn_bwd_workspace(bufs[0], wl.T, wl.H, wl.W))
         sets.append(bufs)
     stream = torch.cuda.current_stream(device)
 
     def call(i, events=None):
+        if grad:
+            q, k, v, dq, do, dk, dv, ws = sets[i % nsets]
+            if events is not None:
+                events[0].record(stream)
+            binding.monarch_attn_bwd(q, k, v, do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w,
+                                     out=(dq, dk, dv), workspace=ws)
+            if events is not None:
+                events[1].record(stream)
+            return 3  # stage-1 recompute, stage-2 backward, stage-1 backward
         if chunk:
             q, k, v, o, kc, yc, y1 = sets[i % nsets]
             if events is None:
@@ -546,7 +586,10 @@ def run_ours(args):
             "launches_per_call": per_call[0] if per_call else None,
         }
 
-    if row:
+    if grad:
+        roofline = rate("monarch_bwd_f32", f"monarch_attn_bwd fp32 (3 CUDA-core kernels, d={wl.d}; whole call)",
+                        0, wl.flops, wl.io_bytes, alu=True)
+    elif row:
         es, bhd = 2, wl.B * wl.heads * wl.d
         r1 = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (rows pass: blocks of W={wl.W} tokens)", 0,
                   4.0 * wl.N * wl.W * bhd, 4 * wl.N * bhd * es)
@@ -582,7 +625,40 @@ def run_ours(args):
     # end to end through the host-buffer entry point: H2D of Q, K, V, the call, D2H of out,
     # with the copies overlapped with the computation over chunks of batch-heads
     e2e = None
-    if not args.no_e2e and chunk:
+    if not args.no_e2e and grad:
+        # per call the host sends Q, K, V, dO and reads dQ, dK, dV back
+        d_q, d_k, d_v, d_do = (torch.empty_like(q0, device=device) for _ in range(4))
+        hq, hk, hv = (x.pin_memory() for x in (q0, k0, v0))
+        hdo = workloads.generate_upstream(wl).pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(q0).pin_memory() for _ in range(3))
+        dq_b, dk_b, dv_b = (torch.empty_like(q0, device=device) for _ in range(3))
+        ws_b = binding.monarch_attn_bwd_workspace(d_q, wl.T, wl.H, wl.W)
+
+        def e2e_call():
+            for h, d_ in ((hq, d_q), (hk, d_k), (hv, d_v), (hdo, d_do)):
+                d_.copy_(h, non_blocking=True)
+            binding.monarch_attn_bwd(d_q, d_k, d_v, d_do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w,
+                                     out=(dq_b, dk_b, dv_b), workspace=ws_b)
+            for d_, h in ((dq_b, hdq), (dk_b, hdk), (dv_b, hdv)):
+                h.copy_(d_, non_blocking=True)
+
+        e2e_call()
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_call()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, device)
+        e2e_val, e2e_ms = aggregate(world, wl.flops, e2e_steps, e2e_s)
+        nbytes = q0.numel() * q0.element_size()
+        e2e = {"value": e2e_val, "unit": "TFLOP/s", "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 3 * nbytes,
+               "api": "monarch_attn_bwd with pinned host copies of Q, K, V, dO in and dQ, dK, dV out"}
+    elif not args.no_e2e and chunk:
         # per chunk the host sends the new frames' Q, K, V and reads the output
         # back; the context and y1_new stay on the device (the cache of an
         # autoregressive loop lives in HBM)
@@ -646,10 +722,11 @@ def run_ours(args):
         try:
             import oracle
             oracle.build()
-            if chunk or row:
-                sampler = oracle_chunk_sample if chunk else oracle_head_sample
+            if chunk or row or grad:
+                sampler = oracle_chunk_sample if chunk else (oracle_bwd_sample if grad else oracle_head_sample)
                 val, dt, reps = sampler(wl, args.cpu_seconds)
-                sample = f"{reps} head(s) of the {'chunk' if chunk else 'full forward'} ({dt:.1f} s)"
+                what = "chunk" if chunk else ("fp64 gradients" if grad else "full forward")
+                sample = f"{reps} head(s) of the {what} ({dt:.1f} s)"
             else:
                 qs, ks, vs, groups, fpg = oracle_sample(wl, args.cpu_seconds)
                 val, dt = time_oracle(wl, qs, ks, vs, groups, fpg)

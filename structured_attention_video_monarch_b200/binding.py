@@ -161,11 +161,20 @@ def monarch_attn_fwd_strided(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
     return out
 
 
+def monarch_attn_bwd_workspace(q, T: int, H: int, W: int) -> torch.Tensor:
+    """A workspace for monarch_attn_bwd on tensors shaped and typed like q."""
+    B, heads, N, d = q.shape
+    need = load_library().monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, _dtype_code(q))
+    return torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+
+
 def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int = FACT_FRAME,
-                     tile_h: int = 0, tile_w: int = 0, stream=None):
+                     tile_h: int = 0, tile_w: int = 0, stream=None, out=None, workspace=None):
     """Gradients (dq, dk, dv) of monarch_attn_fwd for an upstream gradient dout;
-    fp32 [B, heads, N, d] contiguous CUDA tensors.  Outputs and the workspace are
-    allocated here with PyTorch; every step runs in the library's kernels.
+    fp32 [B, heads, N, d] contiguous CUDA tensors.  ``out`` = (dq, dk, dv) and
+    ``workspace`` (monarch_attn_bwd_workspace) may be given to reuse buffers;
+    otherwise they are allocated here with PyTorch.  Every step runs in the
+    library's kernels.
     """
     ts = (q, k, v, dout)
     if not all(t.is_cuda and t.is_contiguous() for t in ts):
@@ -177,9 +186,14 @@ def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int =
         raise ValueError(f"N={N} does not equal T*H*W={T * H * W}")
     lib = load_library()
     code = _dtype_code(q)
-    need = lib.monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, code)
-    ws = torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = monarch_attn_bwd_workspace(q, T, H, W) if workspace is None else workspace
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    else:
+        dq, dk, dv = out
+        if any(t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or not t.is_cuda
+               for t in (dq, dk, dv)):
+            raise ValueError("out must be three contiguous CUDA tensors shaped and typed like q")
     st = lib.monarch_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
                               dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), B, heads, T, H, W,
                               d, int(factorisation), int(tile_h), int(tile_w), code, _stream_ptr(stream))

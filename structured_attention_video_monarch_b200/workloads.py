@@ -32,6 +32,10 @@ index, fp32 draws in the order Q, K, V, then extras, then cast):
                   1000 + index.
   6 fullclip_row_bf16  the full-clip grid under the (f*h, w) split; Q, K, V
                   iid N(0,1).
+  7 bwd_chunk_f32 gradients on the chunk shape in fp32: Q, K, V iid
+                  N(0,1) * d^-1/4 (moderate logits for the exact path); dO the
+                  same, drawn by generate_upstream from a generator seeded
+                  2000 + index.
 """
 from __future__ import annotations
 
@@ -61,6 +65,7 @@ class Workload:
     tile_w: int = 0
     extra: str = ""  # "scaled", "positional", "outliers" or ""
     T_ctx: int = 0   # context frames before the chunk (autoregressive chunk workloads)
+    grad: bool = False  # gradient workload: dQ, dK, dV for an upstream gradient dO
 
     @property
     def N(self) -> int:
@@ -89,14 +94,18 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs: 4*N*(m+b)*d per (batch, head); no padding."""
-        return 4.0 * self.N * (self.m + self.b) * self.d * self.B * self.heads
+        """Algorithmic FLOPs: 4*N*(m+b)*d per (batch, head), no padding; a
+        gradient workload counts 10*d per (query, key) pair (S, dP, dQ, dK, dV)."""
+        per_pair = 10.0 if self.grad else 4.0
+        return per_pair * self.N * (self.m + self.b) * self.d * self.B * self.heads
 
     @property
     def io_bytes(self) -> int:
         """Minimum HBM bytes: read Q, K, V once, write O once; a chunk also
         reads the context's K and Y1 and writes the new frames' Y1."""
         es = 4 if self.dtype == "f32" else 2
+        if self.grad:  # read Q, K, V, dO; write dQ, dK, dV
+            return 7 * self.N * self.B * self.heads * self.d * es
         rows = 4 * self.N + (self.N + 2 * self.N_ctx if self.T_ctx else 0)
         return rows * self.B * self.heads * self.d * es
 
@@ -112,6 +121,7 @@ WORKLOADS = [
     Workload(4, "large_bf16", 2, 12, 128, 21, 45, 80, "bf16", extra="outliers"),
     Workload(5, "chunk_ar_bf16", 1, 12, 128, 3, 30, 52, "bf16", T_ctx=18),
     Workload(6, "fullclip_row_bf16", 1, 12, 128, 21, 30, 52, "bf16", FACT_ROW),
+    Workload(7, "bwd_chunk_f32", 1, 12, 128, 3, 30, 52, "f32", grad=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -153,6 +163,9 @@ def generate(wl: Workload, seed: int | None = None, B: int | None = None,
         R = torch.randn((8, wl.d), generator=g, dtype=torch.float32)
         pos = (0.5 * positional_features(wl.T, wl.H, wl.W).float() @ R)  # [N, d]
         q.add_(pos); k.add_(pos)
+    elif wl.grad:
+        s = wl.d ** -0.25
+        q.mul_(s); k.mul_(s); v.mul_(s)
     elif wl.extra == "outliers":
         n_out = (wl.N * 5) // 100
         rows = torch.randperm(wl.N, generator=g)[:n_out]
@@ -187,3 +200,13 @@ def generate_context(wl: Workload, seed: int | None = None, B: int | None = None
     yc = torch.randn(shape, generator=g, dtype=torch.float32)
     dt = wl.torch_dtype()
     return kc.to(dt), yc.to(dt)
+
+
+def generate_upstream(wl: Workload, seed: int | None = None, heads: int | None = None):
+    """Seeded upstream gradient dO of a gradient workload, shape [B, heads, N, d]."""
+    seed = 2000 + wl.index if seed is None else seed
+    heads = wl.heads if heads is None else heads
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    do = torch.randn((wl.B, heads, wl.N, wl.d), generator=g, dtype=torch.float32) * wl.d ** -0.25
+    return do.to(wl.torch_dtype())

@@ -66,8 +66,12 @@ def test_committed_profiles_name_their_hash_and_traffic():
 def test_workload_accounting(name):
     wl = workloads.BY_NAME[name]
     bhd = wl.B * wl.heads * wl.d
-    assert wl.flops == 4.0 * wl.N * (wl.m + wl.b) * bhd
     es = 4 if wl.dtype == "f32" else 2
+    if wl.grad:  # 10*d FLOPs per (query, key) pair; read Q, K, V, dO, write dQ, dK, dV
+        assert wl.flops == 10.0 * wl.N * (wl.m + wl.b) * bhd
+        assert wl.io_bytes == 7 * wl.N * bhd * es
+        return
+    assert wl.flops == 4.0 * wl.N * (wl.m + wl.b) * bhd
     extra = wl.N + 2 * wl.N_ctx if wl.T_ctx else 0
     assert wl.io_bytes == (4 * wl.N + extra) * bhd * es
     if wl.fact == workloads.FACT_ROW:
