@@ -25,6 +25,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <type_traits>
 
 namespace monarch {
@@ -331,16 +332,22 @@ template <int D, typename E>
 inline cudaError_t chunk_stage2_launch(const E *q, const E *k, const E *k_cache, const E *y1_cache,
                                        const E *y1_new, E *out, const ChunkParams &p, cudaStream_t stream) {
     using Cfg = ChunkCfg<D, E>;
+    // the attribute is per function and device; setting it again is harmless,
+    // so concurrent first calls need no more than the flag's own lock
+    static std::mutex mu;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
-        e = cudaFuncSetAttribute(monarch_chunk_stage2<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!attr_done[dev]) {
+            e = cudaFuncSetAttribute(monarch_chunk_stage2<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM);
+            if (e != cudaSuccess) return e;
+            attr_done[dev] = true;
+        }
     }
     const long long blocks = (p.groups + Cfg::WARPS - 1) / Cfg::WARPS;
     monarch_chunk_stage2<D, E><<<static_cast<unsigned>(blocks), 32 * Cfg::WARPS, Cfg::SMEM, stream>>>(

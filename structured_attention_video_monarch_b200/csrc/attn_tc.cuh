@@ -310,9 +310,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
-// Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
-// bf16 pairs, and accumulate P into two packed fp32 partial sums (even and
-// odd pairs, so the additions form two independent chains).
 // Packs two fp32 values into the kernel's 16-bit input format (fp16 or bf16).
 template <bool F16>
 __device__ __forceinline__ uint32_t pack_in(float lo, float hi) {
@@ -321,6 +318,29 @@ __device__ __forceinline__ uint32_t pack_in(float lo, float hi) {
     else
         return pack_bf16x2(lo, hi);
 }
+
+// The two 16-bit values of a packed pair, widened (exactly) to fp32 and
+// returned as one packed fp32 pair.  A bf16 value is the high half of its
+// fp32 value, so widening it is a shift or a mask.
+template <bool F16>
+__device__ __forceinline__ uint64_t unpack_in(uint32_t w) {
+    if constexpr (F16) {
+        float lo, hi;
+        asm("{\n\t.reg .b16 l, h;\n\t"
+            "mov.b32 {l, h}, %2;\n\t"
+            "cvt.f32.f16 %0, l;\n\t"
+            "cvt.f32.f16 %1, h;\n\t}"
+            : "=f"(lo), "=f"(hi)
+            : "r"(w));
+        return pack_f32x2(lo, hi);
+    } else {
+        return pack_f32x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
+}
+
+// Exponentiate and pack one 32-column chunk: x = s*sl2 - moff, P = 2^x as
+// 16-bit pairs, and accumulate P into two packed fp32 partial sums (even and
+// odd pairs, so the additions form two independent chains).
 
 template <int C, bool F16>
 __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t scale, uint64_t off,
@@ -334,8 +354,9 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t sca
         b = fast_exp2(x1);
         const uint32_t w = pack_in<F16>(a, b);
         pk[e] = w;
-        // the denominator sums the bf16-rounded weights the PV MMA uses
-        const uint64_t r = pack_f32x2(a, b);  // softmax denominator
+        // the denominator sums the rounded weights the PV MMA multiplies, so
+        // each row's effective weights add up to one
+        const uint64_t r = unpack_in<F16>(w);
         if (e & 1)
             acc1 = add_f32x2(acc1, r);
         else

@@ -3,9 +3,10 @@
 Tolerances: fp32 inputs max-abs <= 1e-5; bf16 inputs max-abs <= 2e-2 and
 relative L2 <= 1e-2; fp16 inputs max-abs <= 1e-2 and relative L2 <= 4e-3
 (derived beside the constants).  Outputs are poisoned with NaN before each call so an
-unwritten element fails.  Full-size workloads are checked on oracle rows of
-sampled stage-2 groups (exact for those rows) plus properties that hold at
-any size.
+unwritten element fails.  Full-size workloads are compared with the full
+oracle element by element (the large workload on whole batch-heads, which are
+independent problems), and additionally on oracle rows of sampled stage-2
+groups plus a property that holds at any size.
 """
 import numpy as np
 import pytest
@@ -73,22 +74,29 @@ def test_chunk_bf16_full_heads():
     wl = workloads.BY_NAME["chunk_bf16"]
     q, k, v = workloads.generate(wl)
     got = _run(q, k, v, wl.T, wl.H, wl.W)
-    hs = slice(0, 3)  # heads are independent: the oracle on a head slice is exact for it
-    ref = oracle.monarch_fwd(q[:, hs], k[:, hs], v[:, hs], wl.T, wl.H, wl.W)
-    _check(got[:, hs], ref, torch.bfloat16)
-    assert torch.isfinite(got.float()).all()
+    _check(got, oracle.monarch_fwd(q, k, v, wl.T, wl.H, wl.W), torch.bfloat16)
 
 
 @pytest.mark.parametrize("name,in_dtype", [("fullclip_bf16", torch.bfloat16), ("tiled_bf16", torch.bfloat16),
                                            ("large_bf16", torch.bfloat16), ("fullclip_bf16", torch.float16)],
                          ids=["fullclip", "tiled", "large", "fullclip-f16"])
-def test_full_size_sampled_groups(name, in_dtype):
+def test_full_size_against_oracle(name, in_dtype):
     wl = workloads.BY_NAME[name]
     # fp16 runs take the workload's bf16 values, which fp16 holds exactly
     q, k, v = (x.to(in_dtype) for x in workloads.generate(wl))
     got = _run(q, k, v, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w)
     g = got.float()
     assert torch.isfinite(g).all(), "non-finite output at full size"
+    # every output element against the full oracle; for the large workload on
+    # the first and last batch-heads (each (batch, head) is an independent
+    # problem, so the oracle on one of them is exact for it)
+    if wl.B * wl.heads * wl.T * wl.H * wl.W <= 400_000:
+        _check(got, oracle.monarch_fwd(q, k, v, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w), in_dtype)
+    else:
+        for b, hd in ((0, 0), (wl.B - 1, wl.heads - 1)):
+            sl = (slice(b, b + 1), slice(hd, hd + 1))
+            ref = oracle.monarch_fwd(q[sl], k[sl], v[sl], wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w)
+            _check(got[sl], ref, in_dtype)
     HW = wl.H * wl.W
     # include the first/last positions (ragged last query tile, last stage-2 chunk)
     must = [(0, 0), (wl.B * wl.heads - 1, HW - 1), (1, HW - 2), (2, 1535 % HW), (3, 1559 % HW)]
@@ -154,14 +162,9 @@ def test_tiled_edge_cases(B, heads, T, H, W, d, th, tw, dtype):
 
 
 def test_large_logits_rescale_path():
-    """Peaked softmax rows (large |q.k|) exercise the running-max rescale.
-
-    This input lies far outside the workloads (logit spread ~6x theirs), so it
-    is held to a bound derived from the arithmetic rather than the workloads'
-    2e-2: when one weight dominates a row, the bf16 rounding of that weight
-    (relative 2^-9) reaches the output once in each stage, and the bf16 output
-    rounding adds one more half-ulp: 3 * 2^-9 * max|V|.
-    """
+    """Peaked softmax rows (large |q.k|, logit spread ~6x the workloads')
+    exercise the running-max rescale, held to the same bf16 bounds as every
+    other input (max-abs <= 2e-2, relative L2 <= 1e-2)."""
     B, heads, T, H, W, d = 1, 2, 3, 30, 52, 128
     q, k, v = workloads.random_inputs(B, heads, T, H, W, d, seed=77)
     # make later key tiles of each frame dominate so the running max grows
@@ -169,12 +172,8 @@ def test_large_logits_rescale_path():
     k.view(B, heads, T, H * W, d)[:, :, :, 1000:] *= 3.0
     k = k.to(torch.bfloat16)
     q = (q.float() * 2.0).to(torch.bfloat16)
-    got = _run(q, k, v, T, H, W).double().numpy()
-    ref = oracle.monarch_fwd(q, k, v, T, H, W)
-    assert np.isfinite(got).all()
-    atol = 3 * 2.0 ** -9 * float(v.float().abs().max())
-    assert np.abs(got - ref).max() <= atol
-    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= BF16_RL2
+    got = _run(q, k, v, T, H, W)
+    _check(got, oracle.monarch_fwd(q, k, v, T, H, W), torch.bfloat16)
 
 
 def test_constant_values_and_zero_qk():
