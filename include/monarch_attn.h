@@ -19,10 +19,27 @@
  * with the stage-1 outputs as values.
  *
  * Every entry point is plain C: raw pointers, ints, and a cudaStream_t passed
- * as void*.  The bf16 / fp16 path keeps a small per-(device, stream) buffer of
- * completion counters (one 32-bit word per batch-head, at least 4 KB),
- * allocated with cudaMalloc by the first call on that stream and reused
- * afterwards; a call needing more drains the stream and reallocates it.
+ * as void*.
+ *
+ * Device memory the library holds itself.  The bf16 / fp16 path needs one
+ * 32-bit completion counter per batch-head for each call in flight; the
+ * (f*h, w) split also needs a stage-1 scratch of N*d elements per batch-head.
+ * Both come from per-device pools that the first call needing them allocates
+ * with cudaMalloc and that stay allocated while the library is loaded (never
+ * freed, so a pointer captured into a CUDA graph stays valid):
+ *   - counters: 64 slots of max(4096, B*heads) words (1 MB for up to 4096
+ *     batch-heads).  A larger call allocates a pool of twice the slot size and
+ *     retires the old one, so the total stays below twice the largest pool.
+ *     A stream keeps its slot while it is among the 64 most recently used;
+ *     a stream taking over a slot is ordered after the slot's previous user
+ *     with cudaStreamWaitEvent (no host synchronisation).  A stream under
+ *     capture pins its slot to itself.
+ *   - (f*h, w) scratch: one buffer per device, grown by doubling (outgrown
+ *     buffers retired the same way); calls on different streams are ordered
+ *     through its event, so such calls on two streams run one after the other.
+ * No call frees device memory or synchronises the host (outside
+ * MONARCH_ATTN_DEBUG=1).  Encoded TMA tensor maps are cached host-side (1024
+ * most recently used, keyed by address, shape, strides, box and type).
  */
 #ifndef MONARCH_ATTN_H
 #define MONARCH_ATTN_H
@@ -81,10 +98,9 @@ typedef enum {
  * 2602.12271, "Alinhamento de Blocos"; gist.science/zh/paper/2602.12271,
  * section 2.2): the tokens form a (T*H) x W grid, stage-1 blocks are its rows
  * and stage-2 groups its columns.  It runs as two stage-1 passes of the
- * forward's kernels and keeps the stage-1 result in a scratch buffer the
- * library allocates per (device, stream) on first use (N*d elements per
- * batch-head; a larger call drains the stream and reallocates), so `out` is
- * written only by the second pass.
+ * forward's kernels and keeps the stage-1 result in the device's scratch
+ * pool (see the top of this file), so `out` is written only by the second
+ * pass.
  *   dtype     MONARCH_DTYPE_BF16, MONARCH_DTYPE_F16 or MONARCH_DTYPE_F32.
  *   stream    cudaStream_t (NULL = legacy default stream) the work is queued on.
  *
@@ -97,7 +113,11 @@ typedef enum {
  *   The caller owns all four buffers.  Argument errors are reported before
  *   anything is queued.  The call is asynchronous: it returns after queueing
  *   the kernels on `stream`; device faults surface at the caller's next
- *   synchronisation, following CUDA convention.  Device-side waits are
+ *   synchronisation, following CUDA convention.  The bf16 / fp16 kernel is a
+ *   cooperative launch (its stage-2 work waits for stage-1 results of other
+ *   CTAs): if the device cannot make the whole grid resident at once (for
+ *   example under an MPS SM limit) the launch fails and the call returns
+ *   MONARCH_ERR_LAUNCH.  Device-side waits are
  *   bounded: a wait that gives up records MONARCH_ERR_TIMEOUT in a device
  *   status word that monarch_attn_device_status() returns.  With the
  *   environment variable MONARCH_ATTN_DEBUG=1 the call synchronises `stream`
@@ -193,10 +213,10 @@ int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void 
  * monarch_attn_fwd_noalloc -- monarch_attn_fwd for bf16 that allocates no
  * device memory.  No counterpart in the pages: it exists for callers that
  * cannot allocate once running (a real-time generation loop, where
- * monarch_attn_fwd's first call on a new stream would cudaMalloc its counter
- * buffer and growing it would drain the stream and cudaFree, which waits for
- * the whole device; or a host whose device memory is all held by its own
- * pool).
+ * monarch_attn_fwd's first call on a device, or its first call with more
+ * batch-heads than any before, would cudaMalloc its counter pool, which can
+ * stall behind other work on the device; or a host whose device memory is
+ * all held by its own pool).
  *
  * Arguments, layout, ownership and status codes are those of
  * monarch_attn_fwd with dtype = MONARCH_DTYPE_BF16.  Scratch: the per-batch-
@@ -244,8 +264,9 @@ int monarch_attn_fwd_noalloc(const void *q, const void *k, const void *v, void *
  * other output.  All pointers 16-byte aligned.  dtype, d, factorisation and
  * tiles as monarch_attn_fwd (MONARCH_FACT_FRAME or _TILED); 1 <= T_new <=
  * 128, T_old >= 0.  Two launches on `stream`: the forward's stage-1 kernel
- * (tensor cores for bf16/fp16, CUDA cores for fp32), then a CUDA-core stage 2.
- * Y1 is held in the input dtype.  Status codes as monarch_attn_fwd;
+ * (tcgen05 tensor cores for bf16/fp16, CUDA cores for fp32), then stage 2,
+ * one warp per (batch-head, position) (warp-level mma.sync tensor-core tiles
+ * for bf16/fp16, CUDA cores for fp32).  Y1 is held in the input dtype.  Status codes as monarch_attn_fwd;
  * MONARCH_ERR_INVALID_ARG also for T_old < 0 or missing context pointers.
  */
 int monarch_attn_fwd_chunk(const void *q, const void *k, const void *v,
@@ -274,18 +295,35 @@ int monarch_attn_fwd_chunk_profiled(const void *q, const void *k, const void *v,
  * 2602.12271, "Methodologie"; gist.science/zh/paper/2602.12271, section 2.2);
  * the gradient itself follows from the forward by the chain rule.
  *
- * This build provides the fp32 path on CUDA cores (dtype MONARCH_DTYPE_F32;
- * bf16 and fp16 return MONARCH_ERR_UNSUPPORTED).  Layout [B][heads][N][d]
- * contiguous, as monarch_attn_fwd.  q, k, v, dout are read; dq, dk, dv are
- * written (previous contents ignored).  workspace: caller-owned device memory
- * of at least monarch_attn_bwd_workspace_size(...) bytes, holding the
- * recomputed stage-1 output and its gradient; its contents on entry do not
- * matter.  No output or the workspace may overlap an input or another
- * output.  Limits: T <= 128, and for the stage-1 blocks 8*m floats of shared
- * memory (m <= 6400 tokens per block).  Asynchronous on `stream`; dk and dv
- * are accumulated with atomic adds, so repeated calls can differ in the last
- * bits.  Returns MONARCH_ERR_INVALID_ARG for bad pointers, sizes, alignment
- * (16 bytes), overlap or a too-small workspace.
+ * Each stage's backward is the attention backward of its diagonal blocks:
+ * with P = softmax(Q K^T / sqrt(d)), upstream dY, values Vals and output Y,
+ * dVals = P^T dY, dS = P * (dY Vals^T - rowsum(dY * Y)), dQ = dS K / sqrt(d),
+ * dK = dS^T Q / sqrt(d).  Stage 2 (values Y1, upstream dout) yields dY1;
+ * stage 1 (values V, upstream dY1) yields dV; dQ and dK sum both stages.
+ *
+ * Layout [B][heads][N][d] contiguous, as monarch_attn_fwd.  q, k, v, dout are
+ * read; dq, dk, dv are written (previous contents ignored), all of type
+ * `dtype`.  workspace: caller-owned device memory of at least
+ * monarch_attn_bwd_workspace_size(...) bytes; its contents on entry do not
+ * matter.  No output or the workspace may overlap an input or another output.
+ * Returns MONARCH_ERR_INVALID_ARG for bad pointers, sizes, alignment (16
+ * bytes), overlap or a too-small workspace.  Asynchronous on `stream`.
+ *
+ * dtype MONARCH_DTYPE_BF16 / MONARCH_DTYPE_F16 (tensor cores; every
+ * factorisation, including MONARCH_FACT_ROW): the workspace holds the
+ * recomputed Y1 and O and dY1 (16-bit), per-row LSE and rowsum terms (fp32)
+ * and fp32 gradient accumulators: N*(6d + 8 + 12d) bytes per batch-head.  The
+ * forward's kernel recomputes Y1 and O; then per stage a query-outer kernel
+ * (dQ) and a key-outer kernel (dK and dValues) run on tcgen05 with fp32
+ * accumulation and 16-bit P, dS and dY1; every gradient row has one owning
+ * CTA, so the result is deterministic.  Limits as monarch_attn_fwd.
+ *
+ * dtype MONARCH_DTYPE_F32 (CUDA cores, frame and tiled factorisations): the
+ * workspace holds the recomputed stage-1 output and its gradient (2*N*d
+ * floats per batch-head).  Limits: T <= 128, and for the stage-1 blocks 8*m
+ * floats of shared memory (m <= 6400 tokens per block).  dk and dv are
+ * accumulated with atomic adds, so repeated calls can differ in the last
+ * bits.
  */
 int monarch_attn_bwd(const void *q, const void *k, const void *v, const void *dout,
                      void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
@@ -294,6 +332,21 @@ int monarch_attn_bwd(const void *q, const void *k, const void *v, const void *do
 
 /* Workspace bytes monarch_attn_bwd needs for these sizes (0 if unsupported). */
 size_t monarch_attn_bwd_workspace_size(int B, int heads, int T, int H, int W, int d, int dtype);
+
+/*
+ * monarch_attn_bwd_profiled -- monarch_attn_bwd that also records CUDA events
+ * (cudaEvent_t passed as void*, created by the caller) on `stream`:
+ * events[0] before the first launch and events[i] after the i-th phase.
+ * Phases, 16-bit dtypes: 1 Y1 recomputation, 2 O recomputation, 3 stage-2
+ * backward (row sums, dQ kernel, dK/dV kernel), 4 stage-1 backward, 5 casts
+ * of the fp32 accumulators; fp32: 1 the whole backward.  *nlaunch receives
+ * the number of phases recorded.  Events beyond `nevents` are not recorded.
+ */
+int monarch_attn_bwd_profiled(const void *q, const void *k, const void *v, const void *dout,
+                              void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                              int B, int heads, int T, int H, int W, int d,
+                              int factorisation, int tile_h, int tile_w, int dtype, void *stream,
+                              void **events, int nevents, int *nlaunch);
 
 /* Human-readable text of a status code; never NULL, owned by the library. */
 const char *monarch_attn_strerror(int status);

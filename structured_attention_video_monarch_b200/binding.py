@@ -66,6 +66,9 @@ def load_library(path: str | None = None):
     sz = ctypes.c_size_t
     lib.monarch_attn_bwd.argtypes = [vp] * 8 + [sz] + [i] * 10 + [vp]
     lib.monarch_attn_bwd.restype = i
+    lib.monarch_attn_bwd_profiled.argtypes = ([vp] * 8 + [sz] + [i] * 10 + [vp] +
+                                              [ctypes.POINTER(vp), i, ctypes.POINTER(i)])
+    lib.monarch_attn_bwd_profiled.restype = i
     lib.monarch_attn_bwd_workspace_size.argtypes = [i] * 7
     lib.monarch_attn_bwd_workspace_size.restype = sz
     lib.monarch_attn_fwd_strided.argtypes = [vp, vp, vp, vp] + [i] * 10 + [ll, ll, ll, vp]
@@ -171,7 +174,8 @@ def monarch_attn_bwd_workspace(q, T: int, H: int, W: int) -> torch.Tensor:
 def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int = FACT_FRAME,
                      tile_h: int = 0, tile_w: int = 0, stream=None, out=None, workspace=None):
     """Gradients (dq, dk, dv) of monarch_attn_fwd for an upstream gradient dout;
-    fp32 [B, heads, N, d] contiguous CUDA tensors.  ``out`` = (dq, dk, dv) and
+    [B, heads, N, d] contiguous CUDA tensors of one dtype (bf16 and fp16 on
+    tensor cores, fp32 on CUDA cores).  ``out`` = (dq, dk, dv) and
     ``workspace`` (monarch_attn_bwd_workspace) may be given to reuse buffers;
     otherwise they are allocated here with PyTorch.  Every step runs in the
     library's kernels.
@@ -184,18 +188,26 @@ def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int =
     B, heads, N, d = q.shape
     if N != T * H * W:
         raise ValueError(f"N={N} does not equal T*H*W={T * H * W}")
+    if any(t.device != q.device for t in ts):
+        raise ValueError("q, k, v, dout must be on one device")
     lib = load_library()
     code = _dtype_code(q)
-    ws = monarch_attn_bwd_workspace(q, T, H, W) if workspace is None else workspace
+    if workspace is None:
+        ws = monarch_attn_bwd_workspace(q, T, H, W)
+    else:
+        ws = workspace
+        if not (ws.is_cuda and ws.device == q.device and ws.is_contiguous()):
+            raise ValueError("workspace must be a contiguous CUDA tensor on q's device")
     if out is None:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     else:
         dq, dk, dv = out
         if any(t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous() or not t.is_cuda
-               for t in (dq, dk, dv)):
-            raise ValueError("out must be three contiguous CUDA tensors shaped and typed like q")
+               or t.device != q.device for t in (dq, dk, dv)):
+            raise ValueError("out must be three contiguous CUDA tensors on q's device, shaped and typed like q")
+    ws_bytes = ws.numel() * ws.element_size()
     st = lib.monarch_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(),
-                              dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), B, heads, T, H, W,
+                              dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_bytes, B, heads, T, H, W,
                               d, int(factorisation), int(tile_h), int(tile_w), code, _stream_ptr(stream))
     if st != 0:
         raise MonarchError(st, "monarch_attn_bwd")
@@ -331,3 +343,21 @@ def last_device_error(reset: bool = True, stream=None) -> int:
 
 def selftest_timeout(limit_cycles: int, stream=None) -> int:
     return int(load_library().monarch_attn_selftest_timeout(int(limit_cycles), _stream_ptr(stream)))
+
+
+def monarch_attn_bwd_profiled(q, k, v, dout, dq, dk, dv, workspace, T, H, W, events,
+                              factorisation=FACT_FRAME, tile_h=0, tile_w=0, stream=None) -> int:
+    """monarch_attn_bwd into given buffers, recording ``events`` (torch.cuda.Event
+    list) around its phases (see include/monarch_attn.h).  Returns the number
+    of phases recorded."""
+    B, heads, N, d = q.shape
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    n = ctypes.c_int(0)
+    st = load_library().monarch_attn_bwd_profiled(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), B, heads, T, H, W, d,
+        int(factorisation), int(tile_h), int(tile_w), _dtype_code(q), _stream_ptr(stream), arr, len(events),
+        ctypes.byref(n))
+    if st != 0:
+        raise MonarchError(st, "monarch_attn_bwd_profiled")
+    return n.value

@@ -1,0 +1,599 @@
+// attn_bwd_tc.cuh -- bf16 / fp16 gradients of the Monarch attention on
+// tcgen05 tensor cores.
+//
+// The pages' kernels run the backward pass as well as the forward
+// (MonarchRT: Efficient Attention for Real-Time Video Generation,
+// gist.science/nl/paper/2602.12271 "Methodologie"; gist.science/zh/paper/
+// 2602.12271 section 2.2).  Every diagonal block of B1 and B2 is a softmax
+// attention, so each stage's backward is the block-local attention backward:
+// with P = softmax(S), S = Q K^T / sqrt(d), upstream dY and values Vals,
+//   dVals = P^T dY,  dP = dY Vals^T,  dS = P * (dP - rowsum(dY * Y)),
+//   dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d).
+// Stage 2 (values Y1, output O, upstream dO) gives dY1 and its parts of dQ
+// and dK; stage 1 (values V, output Y1, upstream dY1) gives dV and the rest.
+//
+// Two kernels per stage, over that stage's geometry (frame or tile blocks,
+// or the forward's stacked stage-2 tiles):
+//   dq kernel   (query-outer): pass 1 over key tiles -> row LSE; pass 2 -> P, dP, dS, dQ += dS K
+//   dkdv kernel (key-outer):   per query tile S^T, dP^T -> P^T, dS^T; dV += P^T dY, dK += dS^T Q
+// Only the two MMA forms of the forward are used: SS with both operands
+// K-major (the S = Q K^T form) and TS with A in tensor memory and B MN-major
+// (the O += P V form), so S and S^T are each computed directly, never
+// transposed.  The same 128-row SW128 tile is a K-major operand (rows x d)
+// and an MN-major B operand (K = rows, N = d).  Every output row has one
+// owning CTA: no atomics.
+//
+// Roles (256 threads): warp 0 lane 0 controls loads and MMAs; warp 1
+// allocates TMEM; warps 4-7 (TMEM lanes 0-127, thread = row) do the
+// elementwise work.  Single-buffered: load, MMA, elementwise, MMA per tile.
+// Every wait is a bounded mbarrier wait.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace monarch {
+
+enum : int { BWD_GEOM_FRAME = 0, BWD_GEOM_STAGE2 = 1, BWD_GEOM_TILED = 2 };
+
+struct BwdParams {
+    int B, heads, T, H, W, HW;
+    long long N;          // tokens per batch-head
+    int m;                // frame: tokens per block (H*W); tiled: tile_h * tile_w
+    int nblk_bh;          // frame: frames per batch-head; tiled: T * tiles_h * tiles_w
+    int ntile;            // 128-row tiles per block (frame, tiled); stage 2: 1
+    int tile_h, tile_w, tiles_h, tiles_w, rows_per_tile;  // tiled: block = one tile of one frame
+    int npos;             // stage 2: positions per stacked tile
+    int s2_chunks;        // stage 2: stacked tiles per batch-head
+    float scale_log2;     // d^-1/2 * log2(e)
+    float scale;          // d^-1/2
+    const float *D;       // per row: rowsum(dY * Y) of this stage, [BH][N]
+    float *lse;           // per row: log2-sum-exp of the scaled logits, [BH][N] (dq writes, dkdv reads)
+    float *dq;            // fp32 [BH][N][d]; accumulate (add_dq) or write
+    float *dk;            // fp32 [BH][N][d]; accumulate (add_dk) or write
+    float *dv;            // fp32 [BH][N][d] (written), or null
+    void *dv16;           // 16-bit copy of dv [BH][N][d] (written), or null
+    int add_dq, add_dk;
+    long long timeout_cycles;
+    unsigned *status;
+};
+
+template <int D>
+struct BwdLayout {
+    static constexpr int NP = D / 64;
+    static constexpr int TILE = NP * 16384;            // 128 rows x D bf16, SW128 panels
+    static constexpr int OFF_A = 0;                    // dq: Q      dkdv: K
+    static constexpr int OFF_B = OFF_A + TILE;         // dq: dY     dkdv: Vals
+    static constexpr int OFF_C = OFF_B + TILE;         // dq: K_j    dkdv: Q_i
+    static constexpr int OFF_E = OFF_C + TILE;         // dq: Vals_j dkdv: dY_i
+    static constexpr int OFF_BAR = OFF_E + TILE;
+    static constexpr int NBAR = 6;                     // ld_full, mma_done, ew_done, mm2_done, fin, spare
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+    static constexpr int BYTES = OFF_MISC + 16;
+    static constexpr int SLACK = 1024;
+    // Every CTA allocates all 512 TMEM columns, so a second CTA on the same SM
+    // could only block in tcgen05.alloc until the first one exits.  Asking for
+    // more than half of the SM's shared memory keeps the CTAs one per SM.
+    static constexpr int ONE_PER_SM = 116 * 1024;
+    static constexpr int ALLOC = BYTES + SLACK > ONE_PER_SM ? BYTES + SLACK : ONE_PER_SM;
+    static_assert(ALLOC <= 232448, "too much shared memory");
+    static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+};
+
+// Problem geometry: which tokens a 128-row tile holds and which (row, col)
+// pairs of a tile pair are inside one attention block.
+struct BwdGeom {
+    int kind;
+    // frame: problem = (bh, t); tiles are 128-row slabs of the frame
+    // stage 2: problem = (bh, chunk); one stacked tile npos positions x T frames
+    __device__ static long long token(const BwdParams &p, int kind, int prob_local, int tile, int row) {
+        if (kind == BWD_GEOM_TILED) {
+            const int tpf = p.tiles_h * p.tiles_w;
+            const int t = prob_local / tpf, tif = prob_local - t * tpf;
+            const int ti = tif / p.tiles_w, tj = tif - ti * p.tiles_w;
+            const int rr = row / p.tile_w, wl = row - rr * p.tile_w;
+            const int hl = tile * p.rows_per_tile + rr;
+            if (rr >= p.rows_per_tile || hl >= p.tile_h) return -1;
+            return static_cast<long long>(t) * p.HW + static_cast<long long>(ti * p.tile_h + hl) * p.W +
+                   tj * p.tile_w + wl;
+        }
+        if (kind == BWD_GEOM_FRAME) {
+            const int i = tile * 128 + row;
+            if (i >= p.m) return -1;
+            return static_cast<long long>(prob_local) * p.HW + i;
+        }
+        const int t = row / p.npos, pl = row - t * p.npos;
+        const int pos = prob_local * p.npos + pl;
+        if (t >= p.T || pos >= p.HW) return -1;
+        return static_cast<long long>(t) * p.HW + pos;
+    }
+    // key column c of key tile `kt` visible from query row r of query tile `qt`
+    __device__ static bool visible(const BwdParams &p, int kind, int prob_local, int qt, int r, int kt, int c) {
+        if (kind == BWD_GEOM_FRAME) return kt * 128 + c < p.m;
+        if (kind == BWD_GEOM_TILED) {
+            const int rr = c / p.tile_w;
+            return rr < p.rows_per_tile && kt * p.rows_per_tile + rr < p.tile_h;
+        }
+        (void)qt;
+        (void)kt;
+        if (c % p.npos != r % p.npos) return false;
+        if (c / p.npos >= p.T) return false;
+        return prob_local * p.npos + c % p.npos < p.HW;
+    }
+};
+
+// TMA load of one 128-row tile of a problem.  frame map (d, m, T, heads, B),
+// box (64, 128, 1, 1, 1); stage-2 map (d, HW, T, heads, B), box (64, npos, T, 1, 1).
+template <int NP>
+__device__ __forceinline__ int bwd_load(const BwdParams &p, int kind, const CUtensorMap *map, uint32_t dst,
+                                        uint32_t bar, int bh, int prob_local, int tile) {
+    const int b = bh / p.heads, hd = bh - b * p.heads;
+    if (kind == BWD_GEOM_TILED) {
+        // map (d, tile_w, tiles_w, tile_h, tiles_h * B*heads*T), box (64, tile_w, 1, rows_per_tile, 1)
+        const int tpf = p.tiles_h * p.tiles_w;
+        const int t = prob_local / tpf, tif = prob_local - t * tpf;
+        const int ti = tif / p.tiles_w, tj = tif - ti * p.tiles_w;
+        const int frame = bh * p.T + t;
+#pragma unroll
+        for (int pn = 0; pn < NP; ++pn)
+            tma_load_5d(dst + pn * 16384, map, bar, pn * 64, 0, tj, tile * p.rows_per_tile, frame * p.tiles_h + ti);
+        return p.rows_per_tile * p.tile_w;
+    }
+    if (kind == BWD_GEOM_FRAME) {
+#pragma unroll
+        for (int pn = 0; pn < NP; ++pn) tma_load_5d(dst + pn * 16384, map, bar, pn * 64, tile * 128, prob_local, hd, b);
+        return 128;  // rows past the frame end are zero-filled
+    }
+#pragma unroll
+    for (int pn = 0; pn < NP; ++pn) tma_load_5d(dst + pn * 16384, map, bar, pn * 64, prob_local * p.npos, 0, hd, b);
+    return p.npos * p.T;
+}
+
+template <int NP>
+__device__ __forceinline__ void bwd_zero_rows(uint32_t tile, int from, int to) {
+    for (int r = from; r < to; ++r)
+#pragma unroll
+        for (int pn = 0; pn < NP; ++pn)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) st_shared_v4(tile + pn * 16384 + r * 128 + c * 16, 0, 0, 0, 0);
+}
+
+// S-form MMA: D[128 x 128] = A[128 x d] B[128 x d]^T, both K-major SW128 tiles.
+template <int D, bool F16>
+__device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
+    constexpr uint32_t KM_HI = sdesc_sw128_hi(1024);
+    constexpr uint32_t IDESC = F16 ? idesc_f16_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+    const uint32_t a = sdesc_sw128_lo(a_addr, 16), b = sdesc_sw128_lo(b_addr, 16);
+    mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, IDESC);
+#pragma unroll
+    for (int k = 1; k < D / 16; ++k) {
+        const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+        mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, IDESC);
+    }
+}
+
+// PV-form MMA: D[128 x d] (+)= A[128 x 128] (16-bit pairs in TMEM at a_tmem)
+// * B[128 x d] (SW128 tile read MN-major: K = tile rows, N = d).
+template <int D, bool F16>
+__device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, bool accumulate) {
+    constexpr uint32_t MN_HI = sdesc_sw128_hi(1024);
+    constexpr uint32_t IDESC = F16 ? idesc_f16_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
+    const uint32_t b = sdesc_sw128_lo(b_addr, 16384);
+    mma_ts_lh(d_tmem, a_tmem, b, MN_HI, IDESC, accumulate ? 1u : 0u);
+#pragma unroll
+    for (int k = 1; k < 8; ++k) mma_ts_lh(d_tmem, a_tmem + k * 8, b + k * 128, MN_HI, IDESC, 1u);
+}
+
+template <bool F16>
+__device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
+    if constexpr (F16)
+        return pack_f16x2(lo, hi);
+    else
+        return pack_bf16x2(lo, hi);
+}
+
+// ------------------------------------------------------------------ dq kernel
+// grid: one CTA per (bh, problem, query tile).  Maps: q, k, vals, dy (same geometry).
+template <int D, bool F16, int KIND>
+__global__ void __launch_bounds__(256, 1)
+monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+               const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
+               const BwdParams p) {
+    using L = BwdLayout<D>;
+    constexpr int NP = L::NP;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *base_ptr = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = base + L::OFF_BAR;
+    const uint32_t ld_full = bar0, mma_done = bar0 + 8, ew_done = bar0 + 16, mm2_done = bar0 + 24, fin = bar0 + 32;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
+    WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
+
+    // problem decode
+    const int nq_tiles = KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile;
+    const int per_bh = (KIND == BWD_GEOM_STAGE2 ? p.s2_chunks : p.nblk_bh) * nq_tiles;
+    const int bh = blockIdx.x / per_bh;
+    const int rem = blockIdx.x - bh * per_bh;
+    const int prob = rem / nq_tiles, qt = rem - prob * nq_tiles;
+    const int nk_tiles = nq_tiles;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0u;
+        mbar_init(ld_full, 1);
+        mbar_init(mma_done, 1);
+        mbar_init(ew_done, 128);
+        mbar_init(mm2_done, 1);
+        mbar_init(fin, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = base + L::OFF_A, tdy = base + L::OFF_B, tk = base + L::OFF_C, tv = base + L::OFF_E;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------ control thread
+        uint32_t ld_par = 0u, ew_par = 0u, m2_par = 0u;
+        bool ok = true;
+        // pass 1: S = Q K_j^T per key tile (the elementwise threads keep max and sum);
+        // Q arrives with K_0 in one phase of ld_full
+        for (int j = 0; j < nk_tiles && ok; ++j) {
+            if (j > 0) {  // the elementwise threads have read the previous S
+                ok = mbar_wait(ew_done, ew_par, ctl);
+                ew_par ^= 1u;
+                if (!ok) break;
+            }
+            const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
+            mbar_arrive_expect_tx(ld_full, (j == 0 ? 2 : 1) * NP * rows * 128);
+            if (j == 0) bwd_load<NP>(p, KIND, &mq, tq, ld_full, bh, prob, qt);
+            bwd_load<NP>(p, KIND, &mk, tk, ld_full, bh, prob, j);
+            ok = mbar_wait(ld_full, ld_par, ctl);
+            ld_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            bwd_mma_ss<D, F16>(tmem + L::COL_S, tq, tk);
+            mma_commit(mma_done);
+        }
+        // pass 2: dY, then per key tile S, dP = dY Vals_j^T, (elementwise dS), dQ += dS K_j
+        if (ok) {
+            ok = mbar_wait(ew_done, ew_par, ctl);  // last pass-1 S consumed
+            ew_par ^= 1u;
+        }
+        if (ok) {
+            const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
+            mbar_arrive_expect_tx(ld_full, NP * rows * 128);
+            bwd_load<NP>(p, KIND, &mdy, tdy, ld_full, bh, prob, qt);
+            ok = mbar_wait(ld_full, ld_par, ctl);
+            ld_par ^= 1u;
+        }
+        for (int j = 0; j < nk_tiles && ok; ++j) {
+            if (j > 0) {  // the previous dQ MMA has read K_j and dS
+                ok = mbar_wait(mm2_done, m2_par, ctl);
+                m2_par ^= 1u;
+                if (!ok) break;
+            }
+            const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
+            if (rows < 128) {  // K_j rows the dQ MMA reads but TMA does not write
+                bwd_zero_rows<NP>(tk, rows, 128);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive_expect_tx(ld_full, 2 * NP * rows * 128);
+            bwd_load<NP>(p, KIND, &mk, tk, ld_full, bh, prob, j);
+            bwd_load<NP>(p, KIND, &mvals, tv, ld_full, bh, prob, j);
+            ok = mbar_wait(ld_full, ld_par, ctl);
+            ld_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            bwd_mma_ss<D, F16>(tmem + L::COL_S, tq, tk);
+            bwd_mma_ss<D, F16>(tmem + L::COL_DP, tdy, tv);
+            mma_commit(mma_done);
+            ok = mbar_wait(ew_done, ew_par, ctl);  // dS stored (16-bit pairs at COL_DP)
+            ew_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_DP, tk, j > 0);
+            mma_commit(mm2_done);
+        }
+        if (ok) {
+            ok = mbar_wait(mm2_done, m2_par, ctl);
+            m2_par ^= 1u;
+        }
+        if (ok) mma_commit(fin);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------ elementwise threads
+        const int row = threadIdx.x - 128;  // TMEM lane
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const long long tok = BwdGeom::token(p, KIND, prob, qt, row);
+        const long long rowg = tok >= 0 ? static_cast<long long>(bh) * p.N + tok : -1;
+        uint32_t md_par = 0u;
+        bool ok = true;
+        float m_run = -INFINITY, l_run = 0.f;  // of the scaled logits, base 2
+        for (int j = 0; j < nk_tiles && ok; ++j) {
+            ok = mbar_wait_warp(mma_done, md_par, ctl);
+            md_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + L::COL_S + 32 * c, r);
+                tmem_wait_ld();
+                float mx = -INFINITY;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const bool vis = BwdGeom::visible(p, KIND, prob, qt, row, j, 32 * c + e);
+                    const float x = vis ? __uint_as_float(r[e]) * p.scale_log2 : -INFINITY;
+                    r[e] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
+                const float mn = fmaxf(m_run, mx);
+                if (mn != -INFINITY) {  // nothing visible so far: keep (-inf, 0)
+                    float sum = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) sum += fast_exp2(__uint_as_float(r[e]) - mn);
+                    l_run = (m_run == -INFINITY ? 0.f : l_run * fast_exp2(m_run - mn)) + sum;
+                    m_run = mn;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(ew_done);
+        }
+        const float lse = (m_run == -INFINITY) ? 0.f : m_run + __log2f(l_run);
+        if (ok && rowg >= 0) p.lse[rowg] = lse;
+        const float dd = rowg >= 0 ? p.D[rowg] : 0.f;
+        for (int j = 0; j < nk_tiles && ok; ++j) {
+            ok = mbar_wait_warp(mma_done, md_par, ctl);
+            md_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            // dS = P * (dP - D), P = 2^(s*c - lse); stored as 16-bit pairs over the
+            // dP columns already read (chunk c writes [16c, 16c+16) after reading [32c, 32c+32))
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t rs[32], rp[32];
+                tmem_ld32(lane_base + L::COL_S + 32 * c, rs);
+                tmem_ld32(lane_base + L::COL_DP + 32 * c, rp);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float ds[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int col = 32 * c + 2 * e + h2;
+                        const bool vis = rowg >= 0 && BwdGeom::visible(p, KIND, prob, qt, row, j, col);
+                        // hidden pairs are exact zeros (their S and dP may be stale bits)
+                        ds[h2] = vis ? fast_exp2(__uint_as_float(rs[2 * e + h2]) * p.scale_log2 - lse) *
+                                           (__uint_as_float(rp[2 * e + h2]) - dd)
+                                     : 0.f;
+                    }
+                    pk[e] = bwd_pack<F16>(ds[0], ds[1]);
+                }
+                tmem_st16(lane_base + L::COL_DP + 16 * c, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ew_done);
+        }
+        if (ok) ok = mbar_wait_warp(fin, 0u, ctl);
+        if (ok) {
+            tc_fence_after();
+            float *dst = rowg >= 0 ? p.dq + rowg * D : nullptr;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, r);
+                tmem_wait_ld();
+                if (dst) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float v = __uint_as_float(r[e]) * p.scale;
+                        dst[32 * c + e] = p.add_dq ? dst[32 * c + e] + v : v;
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+    __syncthreads();
+    if (*abort_flag) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < (1ll << 24)) {
+        }
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ------------------------------------------------------------------ dk/dv kernel
+// grid: one CTA per (bh, problem, key tile).  Maps: k, vals (A operands), q, dy.
+template <int D, bool F16, int KIND>
+__global__ void __launch_bounds__(256, 1)
+monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                 const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
+                 const BwdParams p) {
+    using L = BwdLayout<D>;
+    constexpr int NP = L::NP;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *base_ptr = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar0 = base + L::OFF_BAR;
+    const uint32_t ld_full = bar0, mma_done = bar0 + 8, ew_done = bar0 + 16, mm2_done = bar0 + 24, fin = bar0 + 32;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
+    WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
+
+    const int nk_tiles = KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile;
+    const int per_bh = (KIND == BWD_GEOM_STAGE2 ? p.s2_chunks : p.nblk_bh) * nk_tiles;
+    const int bh = blockIdx.x / per_bh;
+    const int rem = blockIdx.x - bh * per_bh;
+    const int prob = rem / nk_tiles, kt = rem - prob * nk_tiles;
+    const int nq_tiles = nk_tiles;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0u;
+        mbar_init(ld_full, 1);
+        mbar_init(mma_done, 1);
+        mbar_init(ew_done, 128);
+        mbar_init(mm2_done, 1);
+        mbar_init(fin, 1);
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tk = base + L::OFF_A, tv = base + L::OFF_B, tq = base + L::OFF_C, tdy = base + L::OFF_E;
+
+    if (warp == 0 && lane == 0) {
+        uint32_t ld_par = 0u, ew_par = 0u, m2_par = 0u;
+        bool ok = true;
+        const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
+        mbar_arrive_expect_tx(ld_full, 2 * NP * rows * 128);
+        bwd_load<NP>(p, KIND, &mk, tk, ld_full, bh, prob, kt);
+        bwd_load<NP>(p, KIND, &mvals, tv, ld_full, bh, prob, kt);
+        ok = mbar_wait(ld_full, ld_par, ctl);
+        ld_par ^= 1u;
+        for (int i = 0; i < nq_tiles && ok; ++i) {
+            if (i > 0) {  // the previous dV/dK MMAs have read Q_i, dY_i, P^T and dS^T
+                ok = mbar_wait(mm2_done, m2_par, ctl);
+                m2_par ^= 1u;
+                if (!ok) break;
+            }
+            if (rows < 128) {  // Q and dY rows the dK/dV MMAs read but TMA does not write
+                bwd_zero_rows<NP>(tq, rows, 128);
+                bwd_zero_rows<NP>(tdy, rows, 128);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive_expect_tx(ld_full, 2 * NP * rows * 128);
+            bwd_load<NP>(p, KIND, &mq, tq, ld_full, bh, prob, i);
+            bwd_load<NP>(p, KIND, &mdy, tdy, ld_full, bh, prob, i);
+            ok = mbar_wait(ld_full, ld_par, ctl);
+            ld_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            bwd_mma_ss<D, F16>(tmem + L::COL_S, tk, tq);    // S^T = K Q^T
+            bwd_mma_ss<D, F16>(tmem + L::COL_DP, tv, tdy);  // dP^T = Vals dY^T
+            mma_commit(mma_done);
+            ok = mbar_wait(ew_done, ew_par, ctl);  // P^T at COL_S, dS^T at COL_DP (16-bit pairs)
+            ew_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+            bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_S, tdy, i > 0);   // dV += P^T dY
+            bwd_mma_ts<D, F16>(tmem + L::COL_ACC1, tmem + L::COL_DP, tq, i > 0);   // dK += dS^T Q
+            mma_commit(mm2_done);
+        }
+        if (ok) {
+            ok = mbar_wait(mm2_done, m2_par, ctl);
+            m2_par ^= 1u;
+        }
+        if (ok) mma_commit(fin);
+    } else if (warp >= 4) {
+        const int row = threadIdx.x - 128;  // key row of this tile
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const long long tok = BwdGeom::token(p, KIND, prob, kt, row);
+        const long long rowg = tok >= 0 ? static_cast<long long>(bh) * p.N + tok : -1;
+        uint32_t md_par = 0u;
+        bool ok = true;
+        for (int i = 0; i < nq_tiles && ok; ++i) {
+            ok = mbar_wait_warp(mma_done, md_par, ctl);
+            md_par ^= 1u;
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t rs[32], rp[32];
+                tmem_ld32(lane_base + L::COL_S + 32 * c, rs);
+                tmem_ld32(lane_base + L::COL_DP + 32 * c, rp);
+                tmem_wait_ld();
+                uint32_t pp[16], pd[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float pv[2], dsv[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int q = 32 * c + 2 * e + h2;  // query column of tile i
+                        // column q is query row q of tile i; visible when the pair is in one block
+                        const long long qtok = BwdGeom::token(p, KIND, prob, i, q);
+                        const bool vis = rowg >= 0 && qtok >= 0 && BwdGeom::visible(p, KIND, prob, i, q, kt, row);
+                        const long long qg = static_cast<long long>(bh) * p.N + (qtok >= 0 ? qtok : 0);
+                        const float lse = vis ? __ldg(p.lse + qg) : 0.f;
+                        const float dd = vis ? __ldg(p.D + qg) : 0.f;
+                        pv[h2] = vis ? fast_exp2(__uint_as_float(rs[2 * e + h2]) * p.scale_log2 - lse) : 0.f;
+                        dsv[h2] = vis ? pv[h2] * (__uint_as_float(rp[2 * e + h2]) - dd) : 0.f;
+                    }
+                    pp[e] = bwd_pack<F16>(pv[0], pv[1]);
+                    pd[e] = bwd_pack<F16>(dsv[0], dsv[1]);
+                }
+                tmem_st16(lane_base + L::COL_S + 16 * c, pp);
+                tmem_st16(lane_base + L::COL_DP + 16 * c, pd);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(ew_done);
+        }
+        if (ok) ok = mbar_wait_warp(fin, 0u, ctl);
+        if (ok) {
+            // every lane of the warp takes part in the TMEM loads (they are
+            // warp-collective); only rows holding a real key store
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t rv[32], rk[32];
+                tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, rv);
+                tmem_ld32(lane_base + L::COL_ACC1 + 32 * c, rk);
+                tmem_wait_ld();
+                if (rowg >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const long long o = rowg * D + 32 * c + e;
+                        const float dvv = __uint_as_float(rv[e]);
+                        const float dkv = __uint_as_float(rk[e]) * p.scale;
+                        if (p.dv) p.dv[o] = dvv;
+                        p.dk[o] = p.add_dk ? p.dk[o] + dkv : dkv;
+                    }
+                    if (p.dv16) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            w[e] = bwd_pack<F16>(__uint_as_float(rv[2 * e]), __uint_as_float(rv[2 * e + 1]));
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.dv16) + rowg * D + 32 * c);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+    __syncthreads();
+    if (*abort_flag) {
+        const long long t0 = clock64();
+        while (clock64() - t0 < (1ll << 24)) {
+        }
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace monarch

@@ -687,7 +687,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 int kvalid, ext;
                 key_extent(p, un, j, kvalid, ext);
                 const bool masked = (un.kind == UNIT_STAGE2) || (kvalid < 128);
-                if (!mbar_wait(s_full(li), sf_par, ctl)) { ok = false; break; }
+                if (!mbar_wait_warp(s_full(li), sf_par, ctl)) { ok = false; break; }
                 sf_par ^= 1u;
                 tc_fence_after();
                 float s[64];
@@ -786,7 +786,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const int ob = static_cast<int>(fdiv(static_cast<uint32_t>(bh), p.fd_heads)), oh = bh - ob * p.heads;
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + ob * p.sB + oh * p.sH +
                                                    (tok < 0 ? 0 : tok) * p.sN + h * (D / 2));
-            if (!mbar_wait(o_full(li), of_par, ctl)) { ok = false; break; }
+            if (!mbar_wait_warp(o_full(li), of_par, ctl)) { ok = false; break; }
             of_par ^= 1u;
             tc_fence_after();
             // read this half's O columns, then release O at once: the next

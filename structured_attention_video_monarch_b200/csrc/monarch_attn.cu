@@ -10,13 +10,17 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <list>
 #include <mutex>
 #include <type_traits>
+#include <unordered_map>
 #include <utility>
 #include <vector>
 
 #include "../../include/monarch_attn.h"
+#include "attn_bwd_tc.cuh"
 #include "attn_chunk.cuh"
+#include "attn_chunk_mma.cuh"
 #include "attn_f32.cuh"
 #include "attn_tc.cuh"
 
@@ -32,19 +36,10 @@ struct DeviceInfo {
     bool init = false;
     int sms = 0;
     bool tc_attr[4] = {false, false, false, false};  // [fp16][d == 128]
+    int tc_resident[4] = {0, 0, 0, 0};                // CTAs of monarch_tc_kernel per SM
     bool f32_attr[2] = {false, false};
 };
 
-// Per (device, stream) buffer of per-batch-head stage-1 completion counters:
-// calls queued on one stream run in order, so each buffer is used by one call
-// at a time; calls on different streams get different buffers.
-struct CounterBuf {
-    int dev;
-    cudaStream_t stream;
-    unsigned *ptr;
-    size_t cap;  // elements
-};
-std::vector<CounterBuf> g_counters;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 
@@ -81,90 +76,167 @@ int device_info(DeviceInfo **out) {
     return MONARCH_OK;
 }
 
-// Counter buffer of at least n elements for (current device, stream),
-// allocated on first use; when a call needs more, the stream is drained and
-// the buffer replaced.
-// Per (device, stream) scratch for the (f*h, w) split's stage-1 output,
-// allocated on first use and replaced (after draining the stream) when a call
-// needs more.
-struct ScratchBuf {
-    int dev;
-    cudaStream_t stream;
-    void *ptr;
-    size_t cap;
-};
-std::vector<ScratchBuf> g_scratch;
+// ------------------------------------------------------------ device buffers
+//
+// The bf16 / fp16 path needs one 32-bit completion counter per batch-head for
+// each call in flight, and the (f*h, w) split a Y1 scratch of N*d elements per
+// batch-head.  Both are taken from per-device pools that the library
+// allocates on first use and never frees while it is loaded, so their size is
+// bounded and a pointer baked into a captured CUDA graph stays valid:
+//   counters: kCounterSlots slots of `cap` words (cap >= 4096, doubled when a
+//     call has more batch-heads; the old pool is retired, not freed).  A
+//     stream keeps its slot while it is among the kCounterSlots most recently
+//     used; a stream that takes over a slot first waits (cudaStreamWaitEvent)
+//     for the event its previous user recorded after its last launch, so no
+//     host synchronisation is needed.  A stream being captured pins its slot.
+//   Y1 scratch: one buffer per device, grown geometrically (old buffers
+//     retired); calls on different streams are ordered through its event.
+// All of this runs under g_buf_mu, held across each launch so that the event
+// recorded after a launch is the one the next user of the buffer waits for.
+constexpr int kCounterSlots = 64;
+constexpr size_t kCounterMinWords = 4096;
 
-int scratch_for(cudaStream_t stream, size_t bytes, void **out) {
+struct CounterSlot {
+    cudaStream_t stream = nullptr;
+    unsigned long long last = 0;  // LRU tick
+    cudaEvent_t done = nullptr;   // recorded after the slot's last launch
+    bool used = false;
+    bool recorded = false;
+    bool pinned = false;          // taken by a stream under capture
+};
+
+struct DevicePools {
+    unsigned *counters = nullptr;
+    size_t cap = 0;  // words per slot
+    CounterSlot slot[kCounterSlots];
+    unsigned long long tick = 0;
+    void *y1 = nullptr;
+    size_t y1_cap = 0;
+    cudaStream_t y1_stream = nullptr;
+    cudaEvent_t y1_done = nullptr;
+    bool y1_recorded = false;
+    std::vector<void *> retired;  // outgrown buffers (kept: captured graphs may name them)
+};
+
+DevicePools g_pools[kMaxDevices];
+std::recursive_mutex g_buf_mu;
+
+bool capturing(cudaStream_t stream) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    return cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive;
+}
+
+// A counter slot of at least n words for (current device, stream), with
+// `stream` ordered after the slot's previous user.  Caller holds g_buf_mu and
+// calls counters_done() after its launch.
+int counters_acquire(cudaStream_t stream, size_t n, unsigned **out, int *slot_out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MONARCH_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_mu);
-    ScratchBuf *sb = nullptr;
-    for (auto &c : g_scratch)
-        if (c.dev == dev && c.stream == stream) sb = &c;
-    if (!sb) {
-        g_scratch.push_back(ScratchBuf{dev, stream, nullptr, 0});
-        sb = &g_scratch.back();
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    DevicePools &dp = g_pools[dev];
+    if (dp.cap < n) {
+        size_t cap = dp.cap ? dp.cap : kCounterMinWords;
+        while (cap < n) cap *= 2;
+        unsigned *ptr = nullptr;
+        if (cudaMalloc(reinterpret_cast<void **>(&ptr), cap * kCounterSlots * sizeof(unsigned)) != cudaSuccess)
+            return MONARCH_ERR_CUDA;
+        if (dp.counters) dp.retired.push_back(dp.counters);
+        dp.counters = ptr;
+        dp.cap = cap;
     }
-    if (sb->cap < bytes) {
-        if (sb->ptr) {
-            if (cudaStreamSynchronize(stream) != cudaSuccess) return MONARCH_ERR_CUDA;
-            cudaFree(sb->ptr);
-            sb->ptr = nullptr;
-            sb->cap = 0;
-        }
-        if (cudaMalloc(&sb->ptr, bytes) != cudaSuccess) return MONARCH_ERR_CUDA;
-        sb->cap = bytes;
+    const bool cap_mode = capturing(stream);
+    int pick = -1, lru = -1;
+    for (int i = 0; i < kCounterSlots; ++i) {
+        const CounterSlot &c = dp.slot[i];
+        if (c.used && c.stream == stream) { pick = i; break; }
+        if (!c.used) { if (pick < 0) pick = i; continue; }
+        if (!c.pinned && (lru < 0 || c.last < dp.slot[lru].last)) lru = i;
     }
-    *out = sb->ptr;
+    if (pick < 0 || (dp.slot[pick].used && dp.slot[pick].stream != stream)) {
+        if (pick < 0) pick = lru;
+        if (pick < 0) return MONARCH_ERR_UNSUPPORTED;  // every slot pinned by captures
+    }
+    CounterSlot &c = dp.slot[pick];
+    if (!c.done && cudaEventCreateWithFlags(&c.done, cudaEventDisableTiming) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    if (c.used && c.stream != stream && c.recorded) {
+        // a stream under capture cannot wait on work outside the capture
+        if (cap_mode) return MONARCH_ERR_UNSUPPORTED;
+        if (cudaStreamWaitEvent(stream, c.done, 0) != cudaSuccess) return MONARCH_ERR_CUDA;
+    }
+    if (!c.used || c.stream != stream) c.recorded = false;
+    c.used = true;
+    c.stream = stream;
+    c.last = ++dp.tick;
+    if (cap_mode) c.pinned = true;
+    *out = dp.counters + static_cast<size_t>(pick) * dp.cap;
+    *slot_out = pick;
     return MONARCH_OK;
 }
 
-int counters_for(cudaStream_t stream, size_t n, unsigned **out) {
+int counters_done(cudaStream_t stream, int slot) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MONARCH_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_mu);
-    CounterBuf *cb = nullptr;
-    for (auto &c : g_counters)
-        if (c.dev == dev && c.stream == stream) cb = &c;
-    if (!cb) {
-        g_counters.push_back(CounterBuf{dev, stream, nullptr, 0});
-        cb = &g_counters.back();
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    CounterSlot &c = g_pools[dev].slot[slot];
+    if (c.pinned) return MONARCH_OK;  // captured: never handed to another stream
+    if (cudaEventRecord(c.done, stream) != cudaSuccess) return MONARCH_ERR_CUDA;
+    c.recorded = true;
+    return MONARCH_OK;
+}
+
+// The device's Y1 scratch, at least `bytes` long, with `stream` ordered after
+// its previous user.  Caller holds g_buf_mu and calls scratch_done() after
+// its launches.
+int scratch_acquire(cudaStream_t stream, size_t bytes, void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    DevicePools &dp = g_pools[dev];
+    if (dp.y1_cap < bytes) {
+        size_t cap = dp.y1_cap ? dp.y1_cap : (size_t(1) << 20);
+        while (cap < bytes) cap *= 2;
+        void *ptr = nullptr;
+        if (cudaMalloc(&ptr, cap) != cudaSuccess) return MONARCH_ERR_CUDA;
+        if (dp.y1) dp.retired.push_back(dp.y1);
+        dp.y1 = ptr;
+        dp.y1_cap = cap;
+        dp.y1_recorded = false;  // fresh memory: no earlier user
     }
-    if (cb->cap < n) {
-        const size_t cap = n < 1024 ? 1024 : n;
-        if (cb->ptr) {
-            if (cudaStreamSynchronize(stream) != cudaSuccess) return MONARCH_ERR_CUDA;
-            cudaFree(cb->ptr);
-            cb->ptr = nullptr;
-            cb->cap = 0;
-        }
-        if (cudaMalloc(reinterpret_cast<void **>(&cb->ptr), cap * sizeof(unsigned)) != cudaSuccess)
-            return MONARCH_ERR_CUDA;
-        cb->cap = cap;
+    if (!dp.y1_done && cudaEventCreateWithFlags(&dp.y1_done, cudaEventDisableTiming) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    if (dp.y1_recorded && dp.y1_stream != stream) {
+        if (capturing(stream)) return MONARCH_ERR_UNSUPPORTED;
+        if (cudaStreamWaitEvent(stream, dp.y1_done, 0) != cudaSuccess) return MONARCH_ERR_CUDA;
     }
-    *out = cb->ptr;
+    dp.y1_stream = stream;
+    *out = dp.y1;
+    return MONARCH_OK;
+}
+
+int scratch_done(cudaStream_t stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    DevicePools &dp = g_pools[dev];
+    if (capturing(stream)) {
+        dp.y1_recorded = false;
+        return MONARCH_OK;
+    }
+    if (cudaEventRecord(dp.y1_done, stream) != cudaSuccess) return MONARCH_ERR_CUDA;
+    dp.y1_recorded = true;
     return MONARCH_OK;
 }
 
 // Completion counters for monarch_attn_fwd_noalloc: a file-scope device array
-// (4096 words, 16 KB) in place of the per-stream cudaMalloc buffer above, its
-// address looked up once per device.  One array per device means calls of
-// that entry point on one device must not overlap in time.
+// (4096 words, 16 KB) in place of the pooled cudaMalloc buffers above.  Its
+// device address is looked up on every call (with the caller's device
+// current): the lookup allocates nothing and stays right after a device reset
+// gives the module a new context.  One array per device means calls of that
+// entry point on one device must not overlap in time.
 static __device__ __align__(256) unsigned g_noalloc_counters[MONARCH_NOALLOC_MAX_BH];
-unsigned *g_noalloc_ptr[kMaxDevices] = {};
 
 int noalloc_counters(unsigned **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_counters) != cudaSuccess || ptr == nullptr)
-            return MONARCH_ERR_CUDA;
-        g_noalloc_ptr[dev] = static_cast<unsigned *>(ptr);
-    }
-    *out = g_noalloc_ptr[dev];
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_counters) != cudaSuccess || ptr == nullptr)
+        return MONARCH_ERR_CUDA;
+    *out = static_cast<unsigned *>(ptr);
     return MONARCH_OK;
 }
 
@@ -245,17 +317,68 @@ int validate(const void *q, const void *k, const void *v, void *out, Shape &s) {
 
 // <tc-launch> (the tensor-core kernel's launch code; profile summaries hash
 // this region with the kernel's own sources)
+// Host-side cache of encoded tensor maps, keyed by everything the encoding
+// reads (address, type, rank, dims, strides, box), least recently used first
+// out.  A map holds no reference to the memory, so a key that matches is the
+// same map even if the buffer was freed and reallocated at that address.
+struct MapKey {
+    uint64_t ptr;
+    uint32_t dtype, rank;
+    cuuint64_t dims[5];
+    cuuint64_t strides[4];
+    cuuint32_t box[5];
+    bool operator==(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey &k) const {
+        const unsigned char *b = reinterpret_cast<const unsigned char *>(&k);
+        uint64_t h = 1469598103934665603ull;  // FNV-1a
+        for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ b[i]) * 1099511628211ull;
+        return static_cast<size_t>(h);
+    }
+};
+constexpr size_t kMapCacheEntries = 1024;
+std::list<std::pair<MapKey, CUtensorMap>> g_map_lru;  // front = most recent
+std::unordered_map<MapKey, std::list<std::pair<MapKey, CUtensorMap>>::iterator, MapKeyHash> g_map_index;
+std::mutex g_map_mu;
+
 // 16-bit (bf16 or fp16) tensor map with 128-byte swizzle; dims/strides
 // innermost first, strides in bytes for dims 1..rank-1.
 int make_map(CUtensorMap *map, const void *ptr, int rank, const cuuint64_t *dims,
              const cuuint64_t *strides, const cuuint32_t *box, int dtype) {
+    MapKey key;
+    std::memset(&key, 0, sizeof(key));  // padding takes part in the hash
+    key.ptr = reinterpret_cast<uint64_t>(ptr);
+    key.dtype = static_cast<uint32_t>(dtype);
+    key.rank = static_cast<uint32_t>(rank);
+    for (int i = 0; i < rank; ++i) key.dims[i] = dims[i], key.box[i] = box[i];
+    for (int i = 0; i + 1 < rank; ++i) key.strides[i] = strides[i];
+    {
+        std::lock_guard<std::mutex> lk(g_map_mu);
+        auto it = g_map_index.find(key);
+        if (it != g_map_index.end()) {
+            g_map_lru.splice(g_map_lru.begin(), g_map_lru, it->second);
+            *map = it->second->second;
+            return MONARCH_OK;
+        }
+    }
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     const CUtensorMapDataType ty =
         dtype == MONARCH_DTYPE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUresult r = g_encode(map, ty, rank, const_cast<void *>(ptr), dims,
                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? MONARCH_OK : MONARCH_ERR_CUDA;
+    if (r != CUDA_SUCCESS) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    if (g_map_index.find(key) == g_map_index.end()) {
+        g_map_lru.emplace_front(key, *map);
+        g_map_index[key] = g_map_lru.begin();
+        if (g_map_lru.size() > kMapCacheEntries) {
+            g_map_index.erase(g_map_lru.back().first);
+            g_map_lru.pop_back();
+        }
+    }
+    return MONARCH_OK;
 }
 
 // Stage-1 view of a 16-bit tensor with element strides (sB, sH, sN).
@@ -321,11 +444,19 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     if ((st = get_encode())) return st;
     using L = TcLayout<D>;
     const int di_idx = (F16 ? 2 : 0) + (D == 128 ? 1 : 0);
-    if (!di->tc_attr[di_idx]) {
-        if (cudaFuncSetAttribute(monarch_tc_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::ALLOC) != cudaSuccess)
-            return MONARCH_ERR_CUDA;
-        di->tc_attr[di_idx] = true;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!di->tc_attr[di_idx]) {
+            int occ = 0;
+            if (cudaFuncSetAttribute(monarch_tc_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     L::ALLOC) != cudaSuccess ||
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, monarch_tc_kernel<D, F16>, 640, L::ALLOC) !=
+                    cudaSuccess)
+                return MONARCH_ERR_CUDA;
+            if (occ < 1) return MONARCH_ERR_UNSUPPORTED;
+            di->tc_resident[di_idx] = occ;
+            di->tc_attr[di_idx] = true;
+        }
     }
     TcParams p{};
     p.B = s.B; p.heads = s.heads; p.T = s.T; p.H = s.H; p.W = s.W; p.HW = s.H * s.W;
@@ -408,17 +539,38 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     // One persistent launch runs both stages: stage-1 units write Y1 = B1 V
     // into out; stage-2 units overwrite it in place with P^T B2 P Y1 once the
     // stage-1 lanes of their batch-head have published (per-batch-head
-    // counters, zeroed for every call).
+    // counters, zeroed for every call).  Stage-2 units wait for other CTAs,
+    // so the launch is cooperative: the driver makes every CTA of the grid
+    // resident at once, or refuses the launch (MONARCH_ERR_LAUNCH), rather
+    // than leaving resident CTAs waiting for ones that cannot start.
+    std::unique_lock<std::recursive_mutex> lk(g_buf_mu, std::defer_lock);
     unsigned *counters = fixed_counters;
-    if (!counters && (st = counters_for(stream, static_cast<size_t>(bh), &counters))) return st;
+    int slot = -1;
+    if (!counters) {
+        lk.lock();
+        if ((st = counters_acquire(stream, static_cast<size_t>(bh), &counters, &slot))) return st;
+    }
     p.s1_done = counters;
     if (cudaMemsetAsync(counters, 0, static_cast<size_t>(bh) * sizeof(unsigned), stream) != cudaSuccess)
         return MONARCH_ERR_CUDA;
+    const int resident = di->sms * di->tc_resident[di_idx];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(p.units < resident ? p.units : resident));
+    cfg.blockDim = dim3(640);
+    cfg.dynamicSmemBytes = L::ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     lev.start(stream);
-    const int grid = p.units < di->sms ? p.units : di->sms;
-    monarch_tc_kernel<D, F16><<<grid, 640, L::ALLOC, stream>>>(mq1, mk1, mv1, mq2, mk2, my2, p);
-    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    if (cudaLaunchKernelEx(&cfg, monarch_tc_kernel<D, F16>, mq1, mk1, mv1, mq2, mk2, my2, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return MONARCH_ERR_LAUNCH;
+    }
     lev.record(++lev.launches, stream);
+    if (slot >= 0) return counters_done(stream, slot);
     return MONARCH_OK;
 }
 // </tc-launch>
@@ -451,11 +603,14 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
     if (g1 >= (1ll << 31) || g2 >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
     const int smem2 = 2 * s.T * D * 4;
     const int di_idx = D == 128 ? 1 : 0;
-    if (!di->f32_attr[di_idx]) {
-        if (cudaFuncSetAttribute(monarch_f32_stage2<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 2 * 128 * D * 4) != cudaSuccess)
-            return MONARCH_ERR_CUDA;
-        di->f32_attr[di_idx] = true;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!di->f32_attr[di_idx]) {
+            if (cudaFuncSetAttribute(monarch_f32_stage2<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     2 * 128 * D * 4) != cudaSuccess)
+                return MONARCH_ERR_CUDA;
+            di->f32_attr[di_idx] = true;
+        }
     }
     const float *fq = static_cast<const float *>(q);
     const float *fk = static_cast<const float *>(k);
@@ -482,8 +637,9 @@ int launch_f32(const void *q, const void *k, const void *v, void *out, const Sha
 template <int D, typename E>
 int launch_row(const void *q, const void *k, const void *v, void *out, const Shape &s, cudaStream_t stream,
                LaunchEvents &lev) {
+    std::lock_guard<std::recursive_mutex> lk(g_buf_mu);
     void *y1 = nullptr;
-    int st = scratch_for(stream, static_cast<size_t>(s.elems) * sizeof(E), &y1);
+    int st = scratch_acquire(stream, static_cast<size_t>(s.elems) * sizeof(E), &y1);
     if (st) return st;
     Shape rows = s;
     rows.T = s.T * s.H; rows.H = 1; rows.fact = MONARCH_FACT_FRAME; rows.tile_h = rows.tile_w = 0;
@@ -493,11 +649,204 @@ int launch_row(const void *q, const void *k, const void *v, void *out, const Sha
     if constexpr (tc) {
         constexpr bool f16 = std::is_same<E, __half>::value;
         if ((st = launch_tc<D, f16>(q, k, v, y1, rows, stream, lev, nullptr, true))) return st;
-        return launch_tc<D, f16>(q, k, y1, out, cols, stream, lev, nullptr, true);
+        st = launch_tc<D, f16>(q, k, y1, out, cols, stream, lev, nullptr, true);
     } else {
         if ((st = launch_f32<D>(q, k, v, y1, rows, stream, lev, true))) return st;
-        return launch_f32<D>(q, k, y1, out, cols, stream, lev, true);
+        st = launch_f32<D>(q, k, y1, out, cols, stream, lev, true);
     }
+    if (st) return st;
+    return scratch_done(stream);
+}
+
+
+// ---------------------------------------------------------------- gradients
+// bf16 / fp16 gradients on tensor cores (attn_bwd_tc.cuh), orchestrated here
+// beside the forward's launch code, whose kernels recompute Y1 and O.
+
+// D[row] = sum_c a[row][c] * b[row][c] over 16-bit rows: one warp per row.
+template <int D, typename E>
+__global__ void bwd_rowdot(const E *a, const E *b, float *out, long long rows) {
+    const long long r = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int lane = threadIdx.x & 31;
+    float s = 0.f;
+#pragma unroll
+    for (int c = lane; c < D; c += 32) {
+        float x, y;
+        if constexpr (std::is_same<E, __half>::value) {
+            x = __half2float(a[r * D + c]);
+            y = __half2float(b[r * D + c]);
+        } else {
+            x = __bfloat162float(a[r * D + c]);
+            y = __bfloat162float(b[r * D + c]);
+        }
+        s = fmaf(x, y, s);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) out[r] = s;
+}
+
+template <typename E>
+__global__ void bwd_cast(const float *in, E *out, long long n) {
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        if constexpr (std::is_same<E, __half>::value)
+            out[i] = __float2half_rn(in[i]);
+        else
+            out[i] = __float2bfloat16_rn(in[i]);
+    }
+}
+
+// Workspace (bytes): Y1, O, dY1 (16-bit, N*d each), LSE and D (fp32, N each),
+// dq, dk, dv accumulators (fp32, N*d each); per batch-head.
+size_t bwd_tc_workspace(long long bh, long long N, int d, int es) {
+    return static_cast<size_t>(bh * N) * (3 * d * es + 2 * 4 + 3 * d * 4);
+}
+
+// Geometry of one stage from a (possibly virtual) frame or tiled shape, and the
+// forward's map parameters for the same shape.
+void bwd_geometry(const Shape &s, int D, BwdParams &p, TcParams &tp) {
+    p.B = s.B; p.heads = s.heads; p.T = s.T; p.H = s.H; p.W = s.W; p.HW = s.H * s.W; p.N = s.N;
+    if (s.fact == MONARCH_FACT_TILED) {
+        p.tile_h = s.tile_h; p.tile_w = s.tile_w; p.tiles_h = s.H / s.tile_h; p.tiles_w = s.W / s.tile_w;
+        const int r = 128 / s.tile_w;
+        p.rows_per_tile = r < s.tile_h ? r : s.tile_h;
+        p.m = s.tile_h * s.tile_w;
+        p.nblk_bh = s.T * p.tiles_h * p.tiles_w;
+        p.ntile = (s.tile_h + p.rows_per_tile - 1) / p.rows_per_tile;
+    } else {
+        p.m = p.HW; p.nblk_bh = s.T; p.ntile = (p.m + 127) / 128;
+    }
+    p.npos = s.T <= 128 ? 128 / s.T : 1;
+    p.s2_chunks = (p.HW + p.npos - 1) / p.npos;
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    tp = TcParams{};
+    tp.m = p.m; tp.HW = p.HW; tp.npos = p.npos;
+    tp.tiles_h = p.tiles_h; tp.tiles_w = p.tiles_w; tp.rows_per_tile = p.rows_per_tile;
+}
+
+// The dq then the dk/dv kernel of one stage.  Maps: q, k, values, upstream
+// gradient, all in the geometry KIND.
+template <int D, bool F16, int KIND>
+int bwd_run_stage(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mvals, const CUtensorMap &mdy,
+                  const BwdParams &p, long long bh, cudaStream_t stream) {
+    using LB = BwdLayout<D>;
+    static bool attr_done[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!attr_done[dev]) {
+            if (cudaFuncSetAttribute(monarch_bwd_dq<D, F16, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     LB::ALLOC) != cudaSuccess ||
+                cudaFuncSetAttribute(monarch_bwd_dkdv<D, F16, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     LB::ALLOC) != cudaSuccess)
+                return MONARCH_ERR_CUDA;
+            attr_done[dev] = true;
+        }
+    }
+    const long long per_bh = (KIND == BWD_GEOM_STAGE2 ? p.s2_chunks : p.nblk_bh) *
+                             static_cast<long long>(KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile);
+    if (bh * per_bh >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+    const unsigned grid = static_cast<unsigned>(bh * per_bh);
+    monarch_bwd_dq<D, F16, KIND><<<grid, 256, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    monarch_bwd_dkdv<D, F16, KIND><<<grid, 256, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
+    return cudaGetLastError() == cudaSuccess ? MONARCH_OK : MONARCH_ERR_LAUNCH;
+}
+
+template <int D, bool F16>
+int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk, void *dv,
+                  void *ws, const Shape &s, cudaStream_t stream, LaunchEvents &lev) {
+    using E = typename std::conditional<F16, __half, __nv_bfloat16>::type;
+    DeviceInfo *di = nullptr;
+    int st = device_info(&di);
+    if (st) return st;
+    if ((st = get_encode())) return st;
+    const long long bh = static_cast<long long>(s.B) * s.heads, N = s.N, nd = bh * N * D;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    E *y1 = reinterpret_cast<E *>(w);
+    E *o = y1 + nd;
+    E *dy1 = o + nd;
+    float *lse = reinterpret_cast<float *>(dy1 + nd);
+    float *dd = lse + bh * N;
+    float *dq32 = dd + bh * N;
+    float *dk32 = dq32 + nd;
+    float *dv32 = dk32 + nd;
+    const bool row = s.fact == MONARCH_FACT_ROW;
+    // the two stages' shapes: the (f*h, w) split runs both as stage-1
+    // geometries of virtual shapes (rows: one-row frames; columns: one tall
+    // frame cut into one-column tiles)
+    Shape s1 = s, s2 = s;
+    if (row) {
+        s1.T = s.T * s.H; s1.H = 1; s1.fact = MONARCH_FACT_FRAME; s1.tile_h = s1.tile_w = 0;
+        s2.T = 1; s2.H = s.T * s.H; s2.fact = MONARCH_FACT_TILED; s2.tile_h = s.T * s.H; s2.tile_w = 1;
+    }
+    // recompute Y1 (stage 1 alone) and O (both stages; for the (f*h, w)
+    // split the columns pass over Y1)
+    if ((st = launch_tc<D, F16>(q, k, v, y1, s1, stream, lev, nullptr, true))) return st;
+    if (row) {
+        if ((st = launch_tc<D, F16>(q, k, y1, o, s2, stream, lev, nullptr, true))) return st;
+    } else if ((st = launch_tc<D, F16>(q, k, v, o, s, stream, lev))) {
+        return st;
+    }
+    unsigned *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_device_status) != cudaSuccess)
+        return MONARCH_ERR_CUDA;
+    const long long rows = bh * N;
+    const unsigned rd_grid = static_cast<unsigned>((rows + 7) / 8);
+    // stage 2: values Y1, upstream dO, output O; its value gradient is dY1 (16-bit)
+    {
+        BwdParams p{};
+        TcParams tp{};
+        bwd_geometry(s2, D, p, tp);
+        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 0; p.dk = dk32; p.add_dk = 0; p.dv = nullptr; p.dv16 = dy1;
+        p.timeout_cycles = env_timeout_cycles();
+        p.status = status;
+        bwd_rowdot<D, E><<<rd_grid, 256, 0, stream>>>(static_cast<const E *>(dout), o, dd, rows);
+        if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+        CUtensorMap mq, mk, my, mdo;
+        if (row) {
+            if ((st = stage1_map(&mq, q, s2, tp)) || (st = stage1_map(&mk, k, s2, tp)) ||
+                (st = stage1_map(&my, y1, s2, tp)) || (st = stage1_map(&mdo, dout, s2, tp)))
+                return st;
+            st = bwd_run_stage<D, F16, BWD_GEOM_TILED>(mq, mk, my, mdo, p, bh, stream);
+        } else {
+            if ((st = stage2_map(&mq, q, s2, tp)) || (st = stage2_map(&mk, k, s2, tp)) ||
+                (st = stage2_map(&my, y1, s2, tp)) || (st = stage2_map(&mdo, dout, s2, tp)))
+                return st;
+            st = bwd_run_stage<D, F16, BWD_GEOM_STAGE2>(mq, mk, my, mdo, p, bh, stream);
+        }
+        if (st) return st;
+        lev.record(++lev.launches, stream);
+    }
+    // stage 1: values V, upstream dY1, output Y1
+    {
+        BwdParams p{};
+        TcParams tp{};
+        bwd_geometry(s1, D, p, tp);
+        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 1; p.dk = dk32; p.add_dk = 1; p.dv = dv32; p.dv16 = nullptr;
+        p.timeout_cycles = env_timeout_cycles();
+        p.status = status;
+        bwd_rowdot<D, E><<<rd_grid, 256, 0, stream>>>(dy1, y1, dd, rows);
+        if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+        CUtensorMap mq, mk, mv, mdy;
+        if ((st = stage1_map(&mq, q, s1, tp)) || (st = stage1_map(&mk, k, s1, tp)) ||
+            (st = stage1_map(&mv, v, s1, tp)) || (st = stage1_map(&mdy, dy1, s1, tp)))
+            return st;
+        st = s1.fact == MONARCH_FACT_TILED ? bwd_run_stage<D, F16, BWD_GEOM_TILED>(mq, mk, mv, mdy, p, bh, stream)
+                                           : bwd_run_stage<D, F16, BWD_GEOM_FRAME>(mq, mk, mv, mdy, p, bh, stream);
+        if (st) return st;
+        lev.record(++lev.launches, stream);
+    }
+    bwd_cast<E><<<4 * di->sms, 256, 0, stream>>>(dq32, static_cast<E *>(dq), nd);
+    bwd_cast<E><<<4 * di->sms, 256, 0, stream>>>(dk32, static_cast<E *>(dk), nd);
+    bwd_cast<E><<<4 * di->sms, 256, 0, stream>>>(dv32, static_cast<E *>(dv), nd);
+    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+    lev.record(++lev.launches, stream);
+    return MONARCH_OK;
 }
 
 // <chunk-launch> (hashed with attn_chunk.cuh by the profile summaries)
@@ -515,6 +864,27 @@ int launch_chunk_stage2(const void *q, const void *k, const void *k_cache, const
     p.groups = static_cast<long long>(s.B) * s.heads * p.HW;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     if (p.groups / ChunkCfg<D, E>::WARPS >= (1ll << 31) - 1) return MONARCH_ERR_UNSUPPORTED;
+    if constexpr (!std::is_same<E, float>::value) {
+        // 16-bit inputs: warp-level MMAs for the logits and the weighted sum of Y1
+        // (attn_chunk_mma.cuh); fp32 keeps the CUDA-core kernel
+        using M = ChunkMmaCfg<D, E>;
+        ChunkMmaParams mp{p.HW, p.T_old, p.T_new, p.n_old, p.n_new, p.groups, p.scale_log2,
+                          p.T_new < M::QM ? p.T_new : M::QM,
+                          p.T_old + p.T_new < M::KC ? p.T_old + p.T_new : M::KC};
+        const int smem = M::smem_bytes(mp.qrows, mp.krows);
+        if (smem > 227 * 1024) return MONARCH_ERR_UNSUPPORTED;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(monarch_chunk_stage2_mma<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                cudaSuccess)
+            return MONARCH_ERR_CUDA;
+        const long long blocks = (p.groups + M::WARPS - 1) / M::WARPS;
+        monarch_chunk_stage2_mma<D, E><<<static_cast<unsigned>(blocks), 32 * M::WARPS, smem, stream>>>(
+            static_cast<const E *>(q), static_cast<const E *>(k), static_cast<const E *>(k_cache),
+            static_cast<const E *>(y1_cache), static_cast<const E *>(y1_new), static_cast<E *>(out), mp);
+        if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
+        lev.record(++lev.launches, stream);
+        return MONARCH_OK;
+    }
     if (chunk_stage2_launch<D, E>(static_cast<const E *>(q), static_cast<const E *>(k),
                                   static_cast<const E *>(k_cache), static_cast<const E *>(y1_cache),
                                   static_cast<const E *>(y1_new), static_cast<E *>(out), p, stream) != cudaSuccess)
@@ -555,6 +925,31 @@ int read_status(cudaStream_t stream, int reset) {
 }
 
 }  // namespace
+
+// The 16-bit gradients (monarch_attn_bwd in monarch_bwd.cu calls these).
+size_t bwd_tc_workspace_bytes(long long bh, long long N, int d, int es) { return bwd_tc_workspace(bh, N, d, es); }
+
+int bwd_tc_run(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk, void *dv, void *ws,
+               int B, int heads, int T, int H, int W, int d, int fact, int tile_h, int tile_w, int dtype,
+               cudaStream_t stream, void **events, int nevents, int *nlaunch) {
+    Shape s{B, heads, T, H, W, d, fact, tile_h, tile_w, dtype, 0, 0};
+    int st = validate(q, k, v, dq, s);
+    if (st) return st;
+    LaunchEvents lev;
+    lev.ev = events;
+    lev.n = events ? nevents : 0;
+    if (dtype == MONARCH_DTYPE_F16)
+        st = d == 128 ? launch_bwd_tc<128, true>(q, k, v, dout, dq, dk, dv, ws, s, stream, lev)
+                      : launch_bwd_tc<64, true>(q, k, v, dout, dq, dk, dv, ws, s, stream, lev);
+    else
+        st = d == 128 ? launch_bwd_tc<128, false>(q, k, v, dout, dq, dk, dv, ws, s, stream, lev)
+                      : launch_bwd_tc<64, false>(q, k, v, dout, dq, dk, dv, ws, s, stream, lev);
+    if (nlaunch) *nlaunch = lev.launches;
+    if (st) return st;
+    if (env_debug()) return read_status(stream, 0);
+    return MONARCH_OK;
+}
+
 }  // namespace monarch
 
 using namespace monarch;

@@ -12,6 +12,14 @@
 
 using namespace monarch;
 
+namespace monarch {
+// The 16-bit path lives beside the forward's launch code (monarch_attn.cu).
+size_t bwd_tc_workspace_bytes(long long bh, long long N, int d, int es);
+int bwd_tc_run(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk, void *dv, void *ws,
+               int B, int heads, int T, int H, int W, int d, int fact, int tile_h, int tile_w, int dtype,
+               cudaStream_t stream, void **events, int nevents, int *nlaunch);
+}  // namespace monarch
+
 namespace {
 
 // [a, a + na) and [b, b + nb) share a byte
@@ -76,24 +84,51 @@ int launch_bwd(const float *q, const float *k, const float *v, const float *dout
 extern "C" {
 
 size_t monarch_attn_bwd_workspace_size(int B, int heads, int T, int H, int W, int d, int dtype) {
-    if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1 || (d != 64 && d != 128) || dtype != MONARCH_DTYPE_F32)
-        return 0;
+    if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1 || (d != 64 && d != 128)) return 0;
+    if (dtype == MONARCH_DTYPE_BF16 || dtype == MONARCH_DTYPE_F16)
+        return bwd_tc_workspace_bytes(static_cast<long long>(B) * heads, static_cast<long long>(T) * H * W, d, 2);
+    if (dtype != MONARCH_DTYPE_F32) return 0;
     return 2 * static_cast<size_t>(B) * heads * T * H * W * d * sizeof(float);
 }
 
-int monarch_attn_bwd(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
-                     void *dv, void *workspace, size_t workspace_bytes, int B, int heads, int T, int H,
-                     int W, int d, int factorisation, int tile_h, int tile_w, int dtype, void *stream) {
+static int bwd_impl(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk, void *dv,
+                    void *workspace, size_t workspace_bytes, int B, int heads, int T, int H, int W, int d,
+                    int factorisation, int tile_h, int tile_w, int dtype, void *stream, void **events, int nevents,
+                    int *nlaunch) {
+    if (nlaunch) *nlaunch = 0;
     if (!q || !k || !v || !dout || !dq || !dk || !dv || !workspace) return MONARCH_ERR_INVALID_ARG;
     if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1) return MONARCH_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return MONARCH_ERR_INVALID_ARG;
-    if (factorisation != MONARCH_FACT_FRAME && factorisation != MONARCH_FACT_TILED) return MONARCH_ERR_INVALID_ARG;
+    if (dtype != MONARCH_DTYPE_F32 && dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F16)
+        return MONARCH_ERR_INVALID_ARG;
+    const bool half = dtype == MONARCH_DTYPE_BF16 || dtype == MONARCH_DTYPE_F16;
+    // the (f*h, w) split has gradients on the tensor-core path only
+    if (factorisation != MONARCH_FACT_FRAME && factorisation != MONARCH_FACT_TILED &&
+        !(half && factorisation == MONARCH_FACT_ROW))
+        return MONARCH_ERR_INVALID_ARG;
     if (factorisation == MONARCH_FACT_TILED &&
         (tile_h < 1 || tile_w < 1 || H % tile_h != 0 || W % tile_w != 0))
         return MONARCH_ERR_INVALID_ARG;
-    if (dtype != MONARCH_DTYPE_F32 && dtype != MONARCH_DTYPE_BF16 && dtype != MONARCH_DTYPE_F16)
-        return MONARCH_ERR_INVALID_ARG;
-    if (dtype != MONARCH_DTYPE_F32) return MONARCH_ERR_UNSUPPORTED;  // the tensor-core backward is not built
+    if (half) {
+        // tensor cores: outputs and workspace may not overlap the inputs or each other
+        const size_t need = monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, dtype);
+        if (need == 0 || workspace_bytes < need) return MONARCH_ERR_INVALID_ARG;
+        const size_t bytes = static_cast<size_t>(B) * heads * T * H * W * d * 2;
+        for (const void *p : {q, k, v, dout, static_cast<const void *>(dq), static_cast<const void *>(dk),
+                              static_cast<const void *>(dv), static_cast<const void *>(workspace)})
+            if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return MONARCH_ERR_INVALID_ARG;
+        const void *outs[4] = {dq, dk, dv, workspace};
+        const size_t out_bytes[4] = {bytes, bytes, bytes, need};
+        const void *ins[4] = {q, k, v, dout};
+        for (int a = 0; a < 4; ++a) {
+            for (int b = 0; b < 4; ++b)
+                if (overlap(outs[a], out_bytes[a], ins[b], bytes)) return MONARCH_ERR_INVALID_ARG;
+            for (int b = a + 1; b < 4; ++b)
+                if (overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) return MONARCH_ERR_INVALID_ARG;
+        }
+        return bwd_tc_run(q, k, v, dout, dq, dk, dv, workspace, B, heads, T, H, W, d, factorisation, tile_h, tile_w,
+                          dtype, static_cast<cudaStream_t>(stream), events, nevents, nlaunch);
+    }
     if (T > 128) return MONARCH_ERR_UNSUPPORTED;
     const long long N = static_cast<long long>(T) * H * W;
     if (N > (1ll << 31) || static_cast<long long>(B) * heads > (1ll << 30)) return MONARCH_ERR_UNSUPPORTED;
@@ -119,10 +154,30 @@ int monarch_attn_bwd(const void *q, const void *k, const void *v, const void *do
                 *fv = static_cast<const float *>(v), *fdo = static_cast<const float *>(dout);
     float *fdq = static_cast<float *>(dq), *fdk = static_cast<float *>(dk), *fdv = static_cast<float *>(dv);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    return d == 128 ? launch_bwd<128>(fq, fk, fv, fdo, fdq, fdk, fdv, y1, dy1, B, heads, T, H, W, factorisation,
-                                      tile_h, tile_w, cs)
-                    : launch_bwd<64>(fq, fk, fv, fdo, fdq, fdk, fdv, y1, dy1, B, heads, T, H, W, factorisation,
-                                     tile_h, tile_w, cs);
+    if (events && nevents > 0 && events[0]) cudaEventRecord(static_cast<cudaEvent_t>(events[0]), cs);
+    const int st = d == 128 ? launch_bwd<128>(fq, fk, fv, fdo, fdq, fdk, fdv, y1, dy1, B, heads, T, H, W,
+                                              factorisation, tile_h, tile_w, cs)
+                            : launch_bwd<64>(fq, fk, fv, fdo, fdq, fdk, fdv, y1, dy1, B, heads, T, H, W,
+                                             factorisation, tile_h, tile_w, cs);
+    if (st) return st;
+    if (events && nevents > 1 && events[1]) cudaEventRecord(static_cast<cudaEvent_t>(events[1]), cs);
+    if (nlaunch) *nlaunch = 1;
+    return MONARCH_OK;
+}
+
+int monarch_attn_bwd(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                     void *dv, void *workspace, size_t workspace_bytes, int B, int heads, int T, int H,
+                     int W, int d, int factorisation, int tile_h, int tile_w, int dtype, void *stream) {
+    return bwd_impl(q, k, v, dout, dq, dk, dv, workspace, workspace_bytes, B, heads, T, H, W, d, factorisation,
+                    tile_h, tile_w, dtype, stream, nullptr, 0, nullptr);
+}
+
+int monarch_attn_bwd_profiled(const void *q, const void *k, const void *v, const void *dout, void *dq, void *dk,
+                              void *dv, void *workspace, size_t workspace_bytes, int B, int heads, int T, int H,
+                              int W, int d, int factorisation, int tile_h, int tile_w, int dtype, void *stream,
+                              void **events, int nevents, int *nlaunch) {
+    return bwd_impl(q, k, v, dout, dq, dk, dv, workspace, workspace_bytes, B, heads, T, H, W, d, factorisation,
+                    tile_h, tile_w, dtype, stream, events, nevents, nlaunch);
 }
 
 }  // extern "C"

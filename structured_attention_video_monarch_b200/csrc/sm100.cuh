@@ -122,6 +122,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     return mbar_wait_slow(bar, parity, ctl);
 }
 
+// mbar_wait for warps that go on to warp-collective instructions
+// (tcgen05.ld / tcgen05.st, .sync.aligned): the 32 lanes agree on the result,
+// so either all of them go on or all of them give up.  A lane that went on
+// alone into a collective instruction would wait for the others forever.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtl &ctl) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl));
+}
+
 // Waits until *counter >= target (acquire at GPU scope), sleeping between
 // polls; gives up like mbar_wait.
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const unsigned *p) {

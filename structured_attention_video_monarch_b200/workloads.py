@@ -36,6 +36,11 @@ index, fp32 draws in the order Q, K, V, then extras, then cast):
                   N(0,1) * d^-1/4 (moderate logits for the exact path); dO the
                   same, drawn by generate_upstream from a generator seeded
                   2000 + index.
+  8 bwd_chunk_bf16 gradients on the chunk shape in bf16 (tensor cores):
+                  Q, K, V iid N(0,1), as chunk_bf16; dO iid N(0,1), drawn by
+                  generate_upstream from a generator seeded 2000 + index.
+  9 bwd_fullclip_bf16 gradients on the full-clip grid in bf16: Q, K, V and
+                  dO iid N(0,1).
 """
 from __future__ import annotations
 
@@ -122,6 +127,8 @@ WORKLOADS = [
     Workload(5, "chunk_ar_bf16", 1, 12, 128, 3, 30, 52, "bf16", T_ctx=18),
     Workload(6, "fullclip_row_bf16", 1, 12, 128, 21, 30, 52, "bf16", FACT_ROW),
     Workload(7, "bwd_chunk_f32", 1, 12, 128, 3, 30, 52, "f32", grad=True),
+    Workload(8, "bwd_chunk_bf16", 1, 12, 128, 3, 30, 52, "bf16", grad=True),
+    Workload(9, "bwd_fullclip_bf16", 1, 12, 128, 21, 30, 52, "bf16", grad=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -163,7 +170,7 @@ def generate(wl: Workload, seed: int | None = None, B: int | None = None,
         R = torch.randn((8, wl.d), generator=g, dtype=torch.float32)
         pos = (0.5 * positional_features(wl.T, wl.H, wl.W).float() @ R)  # [N, d]
         q.add_(pos); k.add_(pos)
-    elif wl.grad:
+    elif wl.grad and wl.dtype == "f32":
         s = wl.d ** -0.25
         q.mul_(s); k.mul_(s); v.mul_(s)
     elif wl.extra == "outliers":
@@ -208,5 +215,7 @@ def generate_upstream(wl: Workload, seed: int | None = None, heads: int | None =
     heads = wl.heads if heads is None else heads
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
-    do = torch.randn((wl.B, heads, wl.N, wl.d), generator=g, dtype=torch.float32) * wl.d ** -0.25
+    do = torch.randn((wl.B, heads, wl.N, wl.d), generator=g, dtype=torch.float32)
+    if wl.dtype == "f32":
+        do.mul_(wl.d ** -0.25)
     return do.to(wl.torch_dtype())

@@ -127,7 +127,10 @@ def test_noalloc_refuses_the_row_split_without_cuda(lib):
 def test_bwd_workspace_size_and_validation_without_cuda(lib):
     size = lib.monarch_attn_bwd_workspace_size
     assert size(1, 2, 3, 4, 5, 64, 0) == 2 * 1 * 2 * 3 * 4 * 5 * 64 * 4
-    assert size(1, 2, 3, 4, 5, 64, 1) == 0   # bf16 backward not built
+    # bf16 / fp16: 16-bit Y1, O, dY1, fp32 LSE and row sums, fp32 dq/dk/dv accumulators
+    assert size(1, 2, 3, 4, 5, 64, 1) == 2 * 60 * (3 * 64 * 2 + 2 * 4 + 3 * 64 * 4)
+    assert size(1, 2, 3, 4, 5, 64, 2) == size(1, 2, 3, 4, 5, 64, 1)
+    assert size(1, 2, 3, 4, 5, 64, 3) == 0   # unknown dtype
     assert size(1, 2, 3, 4, 5, 96, 0) == 0   # unsupported head width
     big = 1 << 40
     ptrs = [16 + i * big for i in range(8)]
@@ -140,7 +143,14 @@ def test_bwd_workspace_size_and_validation_without_cuda(lib):
         return lib.monarch_attn_bwd(*p, a["ws"], a["B"], a["heads"], a["T"], a["H"], a["W"], a["d"],
                                     a["fact"], a["th"], a["tw"], a["dtype"], None)
 
-    assert call(dtype=1) == 2                     # bf16: not built
+    assert call(dtype=1) == 1                     # bf16 needs its larger workspace
+    ws16 = size(1, 1, 2, 4, 4, 128, 1)
+    assert call(dtype=1, ws=ws16 - 16) == 1
+    assert call(dtype=3) == 1                     # unknown dtype
+    assert call(dtype=0, fact=2) == 1             # fp32 has no (f*h, w) gradients
+    big16 = [16 + i * big for i in range(7)] + [16 + 7 * big]
+    assert call(dtype=1, T=129, H=1, W=1, ws=size(1, 1, 129, 1, 1, 128, 1), p=big16) == 2  # T > 128
+    assert call(dtype=1, p=ptrs[:4] + [ptrs[1]] + ptrs[5:], ws=ws16) == 1  # dq aliases k
     assert call(ws=ws - 16) == 1                  # workspace too small
     assert call(p=[0] + ptrs[1:]) == 1            # null pointer
     assert call(p=ptrs[:4] + [ptrs[0]] + ptrs[5:]) == 1  # dq aliases q
