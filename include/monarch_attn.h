@@ -27,8 +27,9 @@
  * Both come from per-device pools that the first call needing them allocates
  * with cudaMalloc and that stay allocated while the library is loaded (never
  * freed, so a pointer captured into a CUDA graph stays valid):
- *   - counters: 64 slots of max(4096, B*heads) words (1 MB for up to 4096
- *     batch-heads).  A larger call allocates a pool of twice the slot size and
+ *   - counters: 64 slots of max(4160, B*heads + 1) words (about 1 MB for up
+ *     to 4096 batch-heads): one word per batch-head and the counter from
+ *     which the persistent kernel's CTAs claim units.  A larger call allocates a pool of twice the slot size and
  *     retires the old one, so the total stays below twice the largest pool.
  *     A stream keeps its slot while it is among the 64 most recently used;
  *     a stream taking over a slot is ordered after the slot's previous user
@@ -206,7 +207,8 @@ int monarch_attn_fwd_profiled(const void *q, const void *k, const void *v, void 
                               void *stream, void **events, int nevents, int *nlaunch);
 
 /* Largest B*heads monarch_attn_fwd_noalloc accepts (size of its static
- * counter array: one 32-bit word per batch-head, 16 KB per device). */
+ * counter array: one 32-bit word per batch-head plus the unit-claim counter,
+ * about 16 KB per device). */
 #define MONARCH_NOALLOC_MAX_BH 4096
 
 /*

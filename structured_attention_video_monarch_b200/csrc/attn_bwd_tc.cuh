@@ -61,14 +61,19 @@ template <int D>
 struct BwdLayout {
     static constexpr int NP = D / 64;
     static constexpr int TILE = NP * 16384;            // 128 rows x D bf16, SW128 panels
-    static constexpr int OFF_A = 0;                    // dq: Q      dkdv: K
-    static constexpr int OFF_B = OFF_A + TILE;         // dq: dY     dkdv: Vals
-    static constexpr int OFF_C = OFF_B + TILE;         // dq: K_j    dkdv: Q_i
-    static constexpr int OFF_E = OFF_C + TILE;         // dq: Vals_j dkdv: dY_i
-    static constexpr int OFF_BAR = OFF_E + TILE;
-    static constexpr int NBAR = 6;                     // ld_full, mma_done, ew_done, mm2_done, fin, spare
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
-    static constexpr int BYTES = OFF_MISC + 16;
+    // The operands that stay are single tiles; the streamed ones are double
+    // buffered, so tile t + 1 loads while tile t is computed.
+    static constexpr int OFF_A = 0;                    // dq: Q          dkdv: K
+    static constexpr int OFF_B = OFF_A + TILE;         // dq: dY         dkdv: Vals
+    static constexpr int OFF_C = OFF_B + TILE;         // dq: K_j [2]    dkdv: Q_i [2]
+    static constexpr int OFF_E = OFF_C + 2 * TILE;     // dq: Vals_j [2] dkdv: dY_i [2]
+    static constexpr int OFF_BAR = OFF_E + 2 * TILE;
+    // ld_full[2] (one per buffer), mma_done, ew_done, mm2_done, fin, ls_ready
+    static constexpr int NBAR = 7;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8 + 8;  // tmem base, abort flag (16-byte aligned)
+    // dk/dv kernel: LSE and rowsum terms of the current query tile's rows, [2 tiles][128]
+    static constexpr int OFF_LS = OFF_MISC + 16;
+    static constexpr int BYTES = OFF_LS + 2 * 2 * 128 * 4;
     static constexpr int SLACK = 1024;
     // Every CTA allocates all 512 TMEM columns, so a second CTA on the same SM
     // could only block in tcgen05.alloc until the first one exits.  Asking for
@@ -106,18 +111,32 @@ struct BwdGeom {
         if (t >= p.T || pos >= p.HW) return -1;
         return static_cast<long long>(t) * p.HW + pos;
     }
-    // key column c of key tile `kt` visible from query row r of query tile `qt`
-    __device__ static bool visible(const BwdParams &p, int kind, int prob_local, int qt, int r, int kt, int c) {
-        if (kind == BWD_GEOM_FRAME) return kt * 128 + c < p.m;
-        if (kind == BWD_GEOM_TILED) {
-            const int rr = c / p.tile_w;
-            return rr < p.rows_per_tile && kt * p.rows_per_tile + rr < p.tile_h;
+    // Validity bits of columns [32*chunk, 32*chunk + 32) of tile `kt` seen
+    // from row `row` of the other operand's tile: frame and tiled geometries,
+    // the columns holding real tokens of the block (a prefix); stage 2, the
+    // columns of the row's own position slot in real frames (the relation is
+    // symmetric, so it serves query rows and key rows alike).
+    __device__ static uint32_t col_mask(const BwdParams &p, int kind, int kt, int row, int chunk) {
+        const int c0 = 32 * chunk;
+        if (kind == BWD_GEOM_STAGE2) {
+            const int lim = p.npos * p.T;
+            int c = row % p.npos;
+            if (c < c0) c += ((c0 - c + p.npos - 1) / p.npos) * p.npos;
+            uint32_t m = 0u;
+            for (; c < c0 + 32 && c < lim; c += p.npos) m |= 1u << (c - c0);
+            return m;
         }
-        (void)qt;
-        (void)kt;
-        if (c % p.npos != r % p.npos) return false;
-        if (c / p.npos >= p.T) return false;
-        return prob_local * p.npos + c % p.npos < p.HW;
+        int n;
+        if (kind == BWD_GEOM_FRAME) {
+            n = p.m - kt * 128;
+        } else {
+            int r = p.tile_h - kt * p.rows_per_tile;
+            if (r > p.rows_per_tile) r = p.rows_per_tile;
+            n = r * p.tile_w;
+        }
+        if (n > 128) n = 128;
+        n -= c0;
+        return n >= 32 ? 0xFFFFFFFFu : (n <= 0 ? 0u : ((1u << n) - 1u));
     }
 };
 
@@ -206,7 +225,9 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     uint8_t *base_ptr = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = base + L::OFF_BAR;
-    const uint32_t ld_full = bar0, mma_done = bar0 + 8, ew_done = bar0 + 16, mm2_done = bar0 + 24, fin = bar0 + 32;
+    // ld_full(b): the tiles of buffer b landed; then mma_done, ew_done, mm2_done, fin
+    auto ld_full = [&](int b) { return bar0 + 8u * static_cast<uint32_t>(b); };
+    const uint32_t mma_done = bar0 + 16, ew_done = bar0 + 24, mm2_done = bar0 + 32, fin = bar0 + 40;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
     WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
@@ -221,7 +242,8 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 
     if (threadIdx.x == 0) {
         *abort_flag = 0u;
-        mbar_init(ld_full, 1);
+        mbar_init(ld_full(0), 1);
+        mbar_init(ld_full(1), 1);
         mbar_init(mma_done, 1);
         mbar_init(ew_done, 128);
         mbar_init(mm2_done, 1);
@@ -240,65 +262,61 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------ control thread
-        uint32_t ld_par = 0u, ew_par = 0u, m2_par = 0u;
+        // Tiles g = 0 .. 2*nk - 1: pass 1 (g < nk) computes S = Q K_g^T for
+        // the row LSE; pass 2 (key tile j = g - nk) computes S and dP = dY Vals_j^T,
+        // waits for the elementwise dS, then dQ += dS K_j.  Tile g's K (and
+        // Vals) land in buffer g & 1, loaded while tile g - 1 is computed; Q
+        // arrives with tile 0, dY with tile nk.
+        const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
+        const int ng = 2 * nk_tiles;
+        uint32_t ew_par = 0u, m2_par = 0u;
         bool ok = true;
-        // pass 1: S = Q K_j^T per key tile (the elementwise threads keep max and sum);
-        // Q arrives with K_0 in one phase of ld_full
-        for (int j = 0; j < nk_tiles && ok; ++j) {
-            if (j > 0) {  // the elementwise threads have read the previous S
-                ok = mbar_wait(ew_done, ew_par, ctl);
-                ew_par ^= 1u;
-                if (!ok) break;
-            }
-            const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
-            mbar_arrive_expect_tx(ld_full, (j == 0 ? 2 : 1) * NP * rows * 128);
-            if (j == 0) bwd_load<NP>(p, KIND, &mq, tq, ld_full, bh, prob, qt);
-            bwd_load<NP>(p, KIND, &mk, tk, ld_full, bh, prob, j);
-            ok = mbar_wait(ld_full, ld_par, ctl);
-            ld_par ^= 1u;
-            if (!ok) break;
-            tc_fence_after();
-            bwd_mma_ss<D, F16>(tmem + L::COL_S, tq, tk);
-            mma_commit(mma_done);
-        }
-        // pass 2: dY, then per key tile S, dP = dY Vals_j^T, (elementwise dS), dQ += dS K_j
-        if (ok) {
-            ok = mbar_wait(ew_done, ew_par, ctl);  // last pass-1 S consumed
-            ew_par ^= 1u;
-        }
-        if (ok) {
-            const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
-            mbar_arrive_expect_tx(ld_full, NP * rows * 128);
-            bwd_load<NP>(p, KIND, &mdy, tdy, ld_full, bh, prob, qt);
-            ok = mbar_wait(ld_full, ld_par, ctl);
-            ld_par ^= 1u;
-        }
-        for (int j = 0; j < nk_tiles && ok; ++j) {
-            if (j > 0) {  // the previous dQ MMA has read K_j and dS
-                ok = mbar_wait(mm2_done, m2_par, ctl);
-                m2_par ^= 1u;
-                if (!ok) break;
-            }
-            const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
-            if (rows < 128) {  // K_j rows the dQ MMA reads but TMA does not write
-                bwd_zero_rows<NP>(tk, rows, 128);
+        auto issue_load = [&](int g) {
+            const int b = g & 1;
+            const bool pass2 = g >= nk_tiles;
+            const int jt = pass2 ? g - nk_tiles : g;
+            const uint32_t kb = tk + b * L::TILE, vb = tv + b * L::TILE;
+            if (pass2 && rows < 128) {  // K rows the dQ MMA reads but TMA does not write
+                bwd_zero_rows<NP>(kb, rows, 128);
                 fence_proxy_async_smem();
             }
-            mbar_arrive_expect_tx(ld_full, 2 * NP * rows * 128);
-            bwd_load<NP>(p, KIND, &mk, tk, ld_full, bh, prob, j);
-            bwd_load<NP>(p, KIND, &mvals, tv, ld_full, bh, prob, j);
-            ok = mbar_wait(ld_full, ld_par, ctl);
-            ld_par ^= 1u;
+            const int ntiles = 1 + (g == 0) + (pass2 ? 1 : 0) + (g == nk_tiles);
+            mbar_arrive_expect_tx(ld_full(b), ntiles * NP * rows * 128);
+            if (g == 0) bwd_load<NP>(p, KIND, &mq, tq, ld_full(b), bh, prob, qt);
+            if (g == nk_tiles) bwd_load<NP>(p, KIND, &mdy, tdy, ld_full(b), bh, prob, qt);
+            bwd_load<NP>(p, KIND, &mk, kb, ld_full(b), bh, prob, jt);
+            if (pass2) bwd_load<NP>(p, KIND, &mvals, vb, ld_full(b), bh, prob, jt);
+        };
+        issue_load(0);
+        for (int g = 0; g < ng && ok; ++g) {
+            const int b = g & 1;
+            if (g > 0) {
+                if (g - 1 < nk_tiles) {  // pass-1 tile g-1: its S was read (its MMA is complete)
+                    ok = mbar_wait(ew_done, ew_par, ctl);
+                    ew_par ^= 1u;
+                } else {  // pass-2 tile g-1: its dQ MMA (the last reader of its buffers and of dS) is complete
+                    ok = mbar_wait(mm2_done, m2_par, ctl);
+                    m2_par ^= 1u;
+                }
+                if (!ok) break;
+            }
+            if (g + 1 < ng) issue_load(g + 1);  // into the buffer tile g-1 used
+            ok = mbar_wait(ld_full(b), static_cast<uint32_t>(g >> 1) & 1u, ctl);
             if (!ok) break;
             tc_fence_after();
-            bwd_mma_ss<D, F16>(tmem + L::COL_S, tq, tk);
-            bwd_mma_ss<D, F16>(tmem + L::COL_DP, tdy, tv);
+            const uint32_t kb = tk + b * L::TILE, vb = tv + b * L::TILE;
+            bwd_mma_ss<D, F16>(tmem + L::COL_S, tq, kb);
+            if (g < nk_tiles) {
+                mma_commit(mma_done);
+                continue;
+            }
+            bwd_mma_ss<D, F16>(tmem + L::COL_DP, tdy, vb);
             mma_commit(mma_done);
             ok = mbar_wait(ew_done, ew_par, ctl);  // dS stored (16-bit pairs at COL_DP)
             ew_par ^= 1u;
             if (!ok) break;
             tc_fence_after();
-            bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_DP, tk, j > 0);
+            bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_DP, kb, g > nk_tiles);
             mma_commit(mm2_done);
         }
         if (ok) {
@@ -324,11 +342,12 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             for (int c = 0; c < 4; ++c) {
                 uint32_t r[32];
                 tmem_ld32(lane_base + L::COL_S + 32 * c, r);
+                const uint32_t vm = BwdGeom::col_mask(p, KIND, j, row, c);
                 tmem_wait_ld();
                 float mx = -INFINITY;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const bool vis = BwdGeom::visible(p, KIND, prob, qt, row, j, 32 * c + e);
+                    const bool vis = (vm >> e) & 1u;
                     const float x = vis ? __uint_as_float(r[e]) * p.scale_log2 : -INFINITY;
                     r[e] = __float_as_uint(x);
                     mx = fmaxf(mx, x);
@@ -360,6 +379,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 uint32_t rs[32], rp[32];
                 tmem_ld32(lane_base + L::COL_S + 32 * c, rs);
                 tmem_ld32(lane_base + L::COL_DP + 32 * c, rp);
+                const uint32_t vm = rowg >= 0 ? BwdGeom::col_mask(p, KIND, j, row, c) : 0u;
                 tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
@@ -367,8 +387,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                     float ds[2];
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
-                        const int col = 32 * c + 2 * e + h2;
-                        const bool vis = rowg >= 0 && BwdGeom::visible(p, KIND, prob, qt, row, j, col);
+                        const bool vis = (vm >> (2 * e + h2)) & 1u;
                         // hidden pairs are exact zeros (their S and dP may be stale bits)
                         ds[h2] = vis ? fast_exp2(__uint_as_float(rs[2 * e + h2]) * p.scale_log2 - lse) *
                                            (__uint_as_float(rp[2 * e + h2]) - dd)
@@ -430,7 +449,10 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     uint8_t *base_ptr = smem_raw + (base - raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = base + L::OFF_BAR;
-    const uint32_t ld_full = bar0, mma_done = bar0 + 8, ew_done = bar0 + 16, mm2_done = bar0 + 24, fin = bar0 + 32;
+    // ld_full(b): the tiles of buffer b landed; then mma_done, ew_done, mm2_done, fin
+    auto ld_full = [&](int b) { return bar0 + 8u * static_cast<uint32_t>(b); };
+    const uint32_t mma_done = bar0 + 16, ew_done = bar0 + 24, mm2_done = bar0 + 32, fin = bar0 + 40;
+    const uint32_t ls_ready = bar0 + 48;  // the 128 elementwise threads posted a query tile's LSE and D
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
     WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
@@ -444,11 +466,13 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
     if (threadIdx.x == 0) {
         *abort_flag = 0u;
-        mbar_init(ld_full, 1);
+        mbar_init(ld_full(0), 1);
+        mbar_init(ld_full(1), 1);
         mbar_init(mma_done, 1);
         mbar_init(ew_done, 128);
         mbar_init(mm2_done, 1);
         mbar_init(fin, 1);
+        mbar_init(ls_ready, 128);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -462,41 +486,49 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     const uint32_t tk = base + L::OFF_A, tv = base + L::OFF_B, tq = base + L::OFF_C, tdy = base + L::OFF_E;
 
     if (warp == 0 && lane == 0) {
-        uint32_t ld_par = 0u, ew_par = 0u, m2_par = 0u;
+        // Query tile i's Q and dY land in buffer i & 1, loaded while tile
+        // i - 1 is computed; K and Vals arrive with tile 0.
+        uint32_t ew_par = 0u, m2_par = 0u;
         bool ok = true;
         const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
-        mbar_arrive_expect_tx(ld_full, 2 * NP * rows * 128);
-        bwd_load<NP>(p, KIND, &mk, tk, ld_full, bh, prob, kt);
-        bwd_load<NP>(p, KIND, &mvals, tv, ld_full, bh, prob, kt);
-        ok = mbar_wait(ld_full, ld_par, ctl);
-        ld_par ^= 1u;
+        auto issue_load = [&](int i) {
+            const int b = i & 1;
+            const uint32_t qb = tq + b * L::TILE, yb = tdy + b * L::TILE;
+            if (rows < 128) {  // Q and dY rows the dK/dV MMAs read but TMA does not write
+                bwd_zero_rows<NP>(qb, rows, 128);
+                bwd_zero_rows<NP>(yb, rows, 128);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive_expect_tx(ld_full(b), (i == 0 ? 4 : 2) * NP * rows * 128);
+            if (i == 0) {
+                bwd_load<NP>(p, KIND, &mk, tk, ld_full(b), bh, prob, kt);
+                bwd_load<NP>(p, KIND, &mvals, tv, ld_full(b), bh, prob, kt);
+            }
+            bwd_load<NP>(p, KIND, &mq, qb, ld_full(b), bh, prob, i);
+            bwd_load<NP>(p, KIND, &mdy, yb, ld_full(b), bh, prob, i);
+        };
+        issue_load(0);
         for (int i = 0; i < nq_tiles && ok; ++i) {
-            if (i > 0) {  // the previous dV/dK MMAs have read Q_i, dY_i, P^T and dS^T
+            const int b = i & 1;
+            if (i > 0) {  // the dV/dK MMAs of tile i-1 (the last readers of its buffers, P^T and dS^T) are complete
                 ok = mbar_wait(mm2_done, m2_par, ctl);
                 m2_par ^= 1u;
                 if (!ok) break;
             }
-            if (rows < 128) {  // Q and dY rows the dK/dV MMAs read but TMA does not write
-                bwd_zero_rows<NP>(tq, rows, 128);
-                bwd_zero_rows<NP>(tdy, rows, 128);
-                fence_proxy_async_smem();
-            }
-            mbar_arrive_expect_tx(ld_full, 2 * NP * rows * 128);
-            bwd_load<NP>(p, KIND, &mq, tq, ld_full, bh, prob, i);
-            bwd_load<NP>(p, KIND, &mdy, tdy, ld_full, bh, prob, i);
-            ok = mbar_wait(ld_full, ld_par, ctl);
-            ld_par ^= 1u;
+            if (i + 1 < nq_tiles) issue_load(i + 1);  // into the buffer tile i-1 used
+            ok = mbar_wait(ld_full(b), static_cast<uint32_t>(i >> 1) & 1u, ctl);
             if (!ok) break;
             tc_fence_after();
-            bwd_mma_ss<D, F16>(tmem + L::COL_S, tk, tq);    // S^T = K Q^T
-            bwd_mma_ss<D, F16>(tmem + L::COL_DP, tv, tdy);  // dP^T = Vals dY^T
+            const uint32_t qb = tq + b * L::TILE, yb = tdy + b * L::TILE;
+            bwd_mma_ss<D, F16>(tmem + L::COL_S, tk, qb);    // S^T = K Q^T
+            bwd_mma_ss<D, F16>(tmem + L::COL_DP, tv, yb);   // dP^T = Vals dY^T
             mma_commit(mma_done);
             ok = mbar_wait(ew_done, ew_par, ctl);  // P^T at COL_S, dS^T at COL_DP (16-bit pairs)
             ew_par ^= 1u;
             if (!ok) break;
             tc_fence_after();
-            bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_S, tdy, i > 0);   // dV += P^T dY
-            bwd_mma_ts<D, F16>(tmem + L::COL_ACC1, tmem + L::COL_DP, tq, i > 0);   // dK += dS^T Q
+            bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_S, yb, i > 0);   // dV += P^T dY
+            bwd_mma_ts<D, F16>(tmem + L::COL_ACC1, tmem + L::COL_DP, qb, i > 0);  // dK += dS^T Q
             mma_commit(mm2_done);
         }
         if (ok) {
@@ -509,9 +541,26 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const long long tok = BwdGeom::token(p, KIND, prob, kt, row);
         const long long rowg = tok >= 0 ? static_cast<long long>(bh) * p.N + tok : -1;
+        // LSE and rowsum term of each query row of the current query tile, by
+        // column: each thread posts those of its own row index; a query row
+        // that holds no token gets LSE = +inf, so its weights are exactly 0
+        float *ls_buf = reinterpret_cast<float *>(base_ptr + L::OFF_LS);
         uint32_t md_par = 0u;
         bool ok = true;
         for (int i = 0; i < nq_tiles && ok; ++i) {
+            float *lse_s = ls_buf + (i & 1) * 256, *d_s = lse_s + 128;
+            {
+                const long long qtok = BwdGeom::token(p, KIND, prob, i, row);
+                const long long qg = static_cast<long long>(bh) * p.N + qtok;
+                lse_s[row] = qtok >= 0 ? __ldg(p.lse + qg) : INFINITY;
+                d_s[row] = qtok >= 0 ? __ldg(p.D + qg) : 0.f;
+            }
+            // wait until all 128 threads posted tile i's values (a bounded
+            // wait, like every other); the other buffer was last read in tile
+            // i - 1, which every thread finished before arriving here
+            mbar_arrive(ls_ready);
+            ok = mbar_wait_warp(ls_ready, static_cast<uint32_t>(i) & 1u, ctl);
+            if (!ok) break;
             ok = mbar_wait_warp(mma_done, md_par, ctl);
             md_par ^= 1u;
             if (!ok) break;
@@ -521,6 +570,8 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 uint32_t rs[32], rp[32];
                 tmem_ld32(lane_base + L::COL_S + 32 * c, rs);
                 tmem_ld32(lane_base + L::COL_DP + 32 * c, rp);
+                // stage 2: the query columns of this key's position slot
+                const uint32_t vm = KIND == BWD_GEOM_STAGE2 ? BwdGeom::col_mask(p, KIND, i, row, c) : 0xFFFFFFFFu;
                 tmem_wait_ld();
                 uint32_t pp[16], pd[16];
 #pragma unroll
@@ -529,14 +580,9 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int q = 32 * c + 2 * e + h2;  // query column of tile i
-                        // column q is query row q of tile i; visible when the pair is in one block
-                        const long long qtok = BwdGeom::token(p, KIND, prob, i, q);
-                        const bool vis = rowg >= 0 && qtok >= 0 && BwdGeom::visible(p, KIND, prob, i, q, kt, row);
-                        const long long qg = static_cast<long long>(bh) * p.N + (qtok >= 0 ? qtok : 0);
-                        const float lse = vis ? __ldg(p.lse + qg) : 0.f;
-                        const float dd = vis ? __ldg(p.D + qg) : 0.f;
-                        pv[h2] = vis ? fast_exp2(__uint_as_float(rs[2 * e + h2]) * p.scale_log2 - lse) : 0.f;
-                        dsv[h2] = vis ? pv[h2] * (__uint_as_float(rp[2 * e + h2]) - dd) : 0.f;
+                        const float x = fast_exp2(__uint_as_float(rs[2 * e + h2]) * p.scale_log2 - lse_s[q]);
+                        pv[h2] = ((vm >> (2 * e + h2)) & 1u) ? x : 0.f;
+                        dsv[h2] = pv[h2] * (__uint_as_float(rp[2 * e + h2]) - d_s[q]);
                     }
                     pp[e] = bwd_pack<F16>(pv[0], pv[1]);
                     pd[e] = bwd_pack<F16>(dsv[0], dsv[1]);

@@ -74,6 +74,7 @@ struct TcParams {
     FastDiv fd_u1, fd_u12, fd_u2;   // u1_bh, u1_bh + s2_pairs, s2_pairs
     FastDiv fd_upg, fd_nblk_bh, fd_tpf, fd_tiles_w, fd_tile_w, fd_npos;
     unsigned *s1_done;              // per batch-head: stage-1 lanes whose Y1 rows are stored
+    unsigned *work;                 // next unit to claim (zero at launch); CTAs claim units in order
     unsigned s1_target;             // stage-1 lanes per batch-head
     float scale_log2;               // d^-1/2 * log2(e)
     long long timeout_cycles;
@@ -267,13 +268,20 @@ struct TcLayout {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_KV = OFF_Q + 2 * TILE;
     static constexpr int OFF_BAR = OFF_KV + NS * TILE;
+    // Claimed unit indices, passed from the TMA producer (which claims them)
+    // to the other roles through a ring of NUQ slots.
+    static constexpr int NUQ = 8;
+    // roles reading each slot: the two MMA issuers, the Y1 publisher and the
+    // 16 softmax warps
+    static constexpr int UQ_READERS = 19;
     // barriers: q_full[2] q_empty[2] kv_full[NS] kv_empty[NS] s_full[2] p_full[2]
-    //           o_full[2] o_free[2] y_done[2] y_free[2] pv_done[2]
-    static constexpr int NBAR = 18 + 2 * NS;
-    // exchange of per-row values (partial maxima, partial sums) between the two
-    // column halves of a lane: [2 lanes][2 halves][128 rows] fp32
+    //           o_full[2] o_free[2] y_done[2] y_free[2] pv_done[2] uq_full[NUQ] uq_empty[NUQ]
+    static constexpr int NBAR = 18 + 2 * NS + 2 * NUQ;
+    // exchange of per-row values (row maxima, row sums) between the two column
+    // halves of a lane: [2 lanes][128 rows] fp32
     static constexpr int OFF_X = OFF_BAR + NBAR * 8;
-    static constexpr int OFF_MISC = OFF_X + 2 * 2 * 128 * 4;  // tmem base, abort flag
+    static constexpr int OFF_UQ = OFF_X + 2 * 128 * 4;
+    static constexpr int OFF_MISC = OFF_UQ + NUQ * 4;  // tmem base, abort flag
     static constexpr int BYTES = OFF_MISC + 16;
     // The dynamic shared-memory base is at least 256-byte aligned; up to 768
     // bytes of slack realign it to the 1024 bytes the 128-byte swizzle needs.
@@ -394,6 +402,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     auto y_done = [&](int i) { return bar0 + 8u * (12 + 2 * NS + i); };
     auto y_free = [&](int i) { return bar0 + 8u * (14 + 2 * NS + i); };
     auto pv_done = [&](int i) { return bar0 + 8u * (16 + 2 * NS + i); };
+    auto uq_full = [&](int k) { return bar0 + 8u * (18 + 2 * NS + k); };
+    auto uq_empty = [&](int k) { return bar0 + 8u * (18 + 2 * NS + L::NUQ + k); };
+    volatile int *uq = reinterpret_cast<volatile int *>(base_ptr + L::OFF_UQ);
     float *x_buf = reinterpret_cast<float *>(base_ptr + L::OFF_X);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
@@ -402,6 +413,22 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
     const int lane = threadIdx.x & 31;
     const int wg = warp >> 2;
     WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
+
+    // The k-th unit this CTA runs: the producer claims units from the global
+    // counter in order and posts them in the ring; every other role takes
+    // them from it in the same order (a single thread, or the 32 lanes of a
+    // softmax warp, of which lane 0 frees the slot).  u = -1: no more units.
+    // Returns false when the wait gave up.
+    auto take_unit = [&](int k, int &u, bool whole_warp) -> bool {
+        const int slot = k % L::NUQ;
+        const uint32_t par = static_cast<uint32_t>(k / L::NUQ) & 1u;
+        const bool got = whole_warp ? mbar_wait_warp(uq_full(slot), par, ctl) : mbar_wait(uq_full(slot), par, ctl);
+        if (!got) return false;
+        u = uq[slot];
+        if (whole_warp) __syncwarp();
+        if (!whole_warp || (threadIdx.x & 31) == 0) mbar_arrive(uq_empty(slot));
+        return true;
+    };
 
     if (threadIdx.x == 0) {
         *abort_flag = 0u;
@@ -419,6 +446,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full(s), 1);
             mbar_init(kv_empty(s), 1);
+        }
+        for (int k = 0; k < L::NUQ; ++k) {
+            mbar_init(uq_full(k), 1);
+            mbar_init(uq_empty(k), L::UQ_READERS);
         }
         fence_barrier_init();
     }
@@ -445,7 +476,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             // softmax warps so the fence latency is not on their path.
             uint32_t yd_par = 0u;  // bit i: parity to wait for on y_done(i)
             bool ok = true;
-            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            for (int k = 0; ok; ++k) {
+                int u;
+                if (!take_unit(k, u, false)) break;
+                if (u < 0) break;
                 const Unit un = decode_unit(p, u);
                 if (un.kind != UNIT_STAGE1) continue;
                 for (int i = 0; i < un.nq && ok; ++i) {
@@ -464,11 +498,22 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             // tile(s) then the V tile(s): one K and one V for a shared unit,
             // K_A, K_B, V_A, V_B for a separate one.  The MMA issuer consumes
             // the ring in exactly this order.
+            // Units are claimed one ahead (the atomic's latency overlaps the
+            // current unit's loads) and posted in the ring before their loads.
             uint32_t qe_par = 3u;  // bit i: parity to wait for on q_empty(i)
             int slot = 0;
             uint32_t kv_round = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            unsigned next = atomicAdd(p.work, 1u);
+            for (int k = 0; ok; ++k) {
+                const int u = next < static_cast<unsigned>(p.units) ? static_cast<int>(next) : -1;
+                const int qs = k % L::NUQ;
+                ok = mbar_wait(uq_empty(qs), (static_cast<uint32_t>(k / L::NUQ) & 1u) ^ 1u, ctl);
+                if (!ok) break;
+                uq[qs] = u;
+                mbar_arrive(uq_full(qs));
+                if (u < 0) break;
+                next = atomicAdd(p.work, 1u);
                 const Unit un = decode_unit(p, u);
 #pragma unroll 1
                 for (int i = 0; i < un.nq && ok; ++i) {
@@ -557,7 +602,10 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const uint32_t v_lo0 = sdesc_sw128_lo(base + L::OFF_KV, 16384);  // D panels 16 KB apart
             constexpr uint32_t TILE16 = L::TILE >> 4;
             constexpr uint32_t IDESC_O = F16 ? idesc_f16_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
-            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+            for (int k = 0; ok; ++k) {
+                int u;
+                if (!take_unit(k, u, false)) break;
+                if (u < 0) break;
                 const Unit un = decode_unit(p, u);
                 if (s_role) {
 #pragma unroll 1
@@ -659,19 +707,31 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
         const float sl2 = p.scale_log2;
         uint32_t sf_par = 0u, of_par = 0u, yf_par = 1u;
         bool ok = true;
-        // value of this row in the other column half of the lane.  Only the
-        // two warps holding the same 32 rows (one per half) take part: named
-        // barrier `pair_bar` (64 threads) makes sure the other half has read
-        // the previous value before it is overwritten, then publishes the new one.
-        float *xb = x_buf + li * 2 * 128;
+        // Combines a per-row value of the two column halves of the lane (the
+        // maximum, or the sum), both halves getting the same result.  Only the
+        // two warps holding the same 32 rows (one per half) take part, through
+        // named barrier `pair_bar` (64 threads): half 0 posts its value, half
+        // 1 combines and posts the result, half 0 reads it.  Half 0 writes the
+        // next value only after reading the result, which half 1 posted before
+        // the second barrier, so one slot per row suffices.
+        float *xb = x_buf + li * 128;
         const uint32_t pair_bar = 1u + static_cast<uint32_t>(li * 4 + (warp & 3));
-        auto exchange = [&](float v) -> float {
+        auto combine = [&](float v, bool is_max) -> float {
+            if (h == 0) xb[row] = v;
             named_barrier_sync(pair_bar, 64);
-            xb[h * 128 + row] = v;
+            if (h == 1) {
+                const float o = xb[row];
+                v = is_max ? fmaxf(o, v) : o + v;
+                xb[row] = v;
+            }
             named_barrier_sync(pair_bar, 64);
-            return xb[(1 - h) * 128 + row];
+            if (h == 0) v = xb[row];
+            return v;
         };
-        for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            int u;
+            if (!take_unit(k, u, true)) break;
+            if (u < 0) break;
             const Unit un = decode_unit(p, u);
             if (li >= un.nq) continue;
             float m_run = -INFINITY;  // running max of raw logits (whole row)
@@ -729,9 +789,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                 bool rescale = false;
                 float alpha = 1.f;
                 if (j == 0) {
-                    m_run = fmaxf(mx, exchange(mx));
+                    m_run = combine(mx, true);
                 } else if (named_barrier_or(pair_bar, 64, (mx - m_run) * sl2 > 8.f)) {
-                    mx = fmaxf(mx, exchange(mx));
+                    mx = combine(mx, true);
                     if ((mx - m_run) * sl2 > 8.f) {
                         alpha = fast_exp2((m_run - mx) * sl2);
                         m_run = mx;
@@ -779,7 +839,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             if (!ok) break;
             // ---------------------------------------------------- epilogue
             // row sum over both halves, then O / l for this half's columns
-            const float l = l_half + exchange(l_half);
+            const float l = combine(l_half, false);
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             int bh;
             const long long tok = lane_row_token(p, un.kind, un.ln[li], row, bh);

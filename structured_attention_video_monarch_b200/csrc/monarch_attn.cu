@@ -83,8 +83,9 @@ int device_info(DeviceInfo **out) {
 // batch-head.  Both are taken from per-device pools that the library
 // allocates on first use and never frees while it is loaded, so their size is
 // bounded and a pointer baked into a captured CUDA graph stays valid:
-//   counters: kCounterSlots slots of `cap` words (cap >= 4096, doubled when a
-//     call has more batch-heads; the old pool is retired, not freed).  A
+//   counters: kCounterSlots slots of `cap` words (cap >= 4160: one word per
+//     batch-head plus the unit-claim counter; doubled when a call has more
+//     batch-heads; the old pool is retired, not freed).  A
 //     stream keeps its slot while it is among the kCounterSlots most recently
 //     used; a stream that takes over a slot first waits (cudaStreamWaitEvent)
 //     for the event its previous user recorded after its last launch, so no
@@ -94,7 +95,7 @@ int device_info(DeviceInfo **out) {
 // All of this runs under g_buf_mu, held across each launch so that the event
 // recorded after a launch is the one the next user of the buffer waits for.
 constexpr int kCounterSlots = 64;
-constexpr size_t kCounterMinWords = 4096;
+constexpr size_t kCounterMinWords = 4160;  // 4096 batch-heads + the claim counter, rounded to 256 bytes
 
 struct CounterSlot {
     cudaStream_t stream = nullptr;
@@ -225,12 +226,13 @@ int scratch_done(cudaStream_t stream) {
 }
 
 // Completion counters for monarch_attn_fwd_noalloc: a file-scope device array
-// (4096 words, 16 KB) in place of the pooled cudaMalloc buffers above.  Its
+// (4096 + 1 words, about 16 KB: one per batch-head and the unit-claim
+// counter) in place of the pooled cudaMalloc buffers above.  Its
 // device address is looked up on every call (with the caller's device
 // current): the lookup allocates nothing and stays right after a device reset
 // gives the module a new context.  One array per device means calls of that
 // entry point on one device must not overlap in time.
-static __device__ __align__(256) unsigned g_noalloc_counters[MONARCH_NOALLOC_MAX_BH];
+static __device__ __align__(256) unsigned g_noalloc_counters[MONARCH_NOALLOC_MAX_BH + 1];
 
 int noalloc_counters(unsigned **out) {
     void *ptr = nullptr;
@@ -548,10 +550,13 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     int slot = -1;
     if (!counters) {
         lk.lock();
-        if ((st = counters_acquire(stream, static_cast<size_t>(bh), &counters, &slot))) return st;
+        if ((st = counters_acquire(stream, static_cast<size_t>(bh) + 1, &counters, &slot))) return st;
     }
+    // counters[0, bh): stage-1 lanes published per batch-head; counters[bh]:
+    // the next unit to claim (CTAs take units in order as they free up)
     p.s1_done = counters;
-    if (cudaMemsetAsync(counters, 0, static_cast<size_t>(bh) * sizeof(unsigned), stream) != cudaSuccess)
+    p.work = counters + bh;
+    if (cudaMemsetAsync(counters, 0, (static_cast<size_t>(bh) + 1) * sizeof(unsigned), stream) != cudaSuccess)
         return MONARCH_ERR_CUDA;
     const int resident = di->sms * di->tc_resident[di_idx];
     cudaLaunchConfig_t cfg = {};

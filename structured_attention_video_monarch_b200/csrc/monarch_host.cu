@@ -18,22 +18,22 @@
 
 namespace {
 
-// Upload and download streams, created once per device and kept (creating
-// them costs about as much as a chunk's copy).  Calls from several host
-// threads on one device share them, which orders their copies but keeps
-// each call correct: every call waits only on its own events.
-struct CopyStreams {
+// Upload and download streams and the call's events, created once per device
+// and kept (creating them costs about as much as a chunk's copy).  A call
+// holds its device's lock from its first copy to its final synchronisation,
+// so calls from several host threads on one device run one after another and
+// never share an event while it is in use.
+struct CopyState {
     cudaStream_t up = nullptr, down = nullptr;
+    std::vector<cudaEvent_t> ev;  // grown as calls need more, never destroyed
+    std::mutex mu;
 };
 constexpr int kMaxDevices = 64;
-CopyStreams g_copy[kMaxDevices];
-std::mutex g_copy_mu;
+CopyState g_copy[kMaxDevices];
 
-int copy_streams(CopyStreams *out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MONARCH_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_copy_mu);
-    CopyStreams &c = g_copy[dev];
+// The device's copy state with at least `nev` events; the caller holds cs->mu.
+int copy_state(int dev, size_t nev, CopyState **out) {
+    CopyState &c = g_copy[dev];
     if (!c.up && cudaStreamCreateWithFlags(&c.up, cudaStreamNonBlocking) != cudaSuccess) {
         c.up = nullptr;
         return MONARCH_ERR_CUDA;
@@ -42,17 +42,14 @@ int copy_streams(CopyStreams *out) {
         c.down = nullptr;
         return MONARCH_ERR_CUDA;
     }
-    *out = c;
+    while (c.ev.size() < nev) {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MONARCH_ERR_CUDA;
+        c.ev.push_back(e);
+    }
+    *out = &c;
     return MONARCH_OK;
 }
-
-struct Events {
-    std::vector<cudaEvent_t> ev;
-    ~Events() {
-        for (cudaEvent_t e : ev)
-            if (e) cudaEventDestroy(e);
-    }
-};
 
 }  // namespace
 
@@ -78,17 +75,16 @@ extern "C" int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k,
         if (x < o + total && o < x + total) return MONARCH_ERR_INVALID_ARG;
     }
     cudaStream_t compute = static_cast<cudaStream_t>(stream);
-    CopyStreams s;
-    if (copy_streams(&s) != MONARCH_OK) return MONARCH_ERR_CUDA;
-    Events e;
-    e.ev.assign(static_cast<size_t>(2 * n), nullptr);
-    for (cudaEvent_t &x : e.ev)
-        if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return MONARCH_ERR_CUDA;
+    int devi = 0;
+    if (cudaGetDevice(&devi) != cudaSuccess || devi < 0 || devi >= kMaxDevices) return MONARCH_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_copy[devi].mu);
+    CopyState *cs = nullptr;
+    if (copy_state(devi, static_cast<size_t>(2 * n + 1), &cs) != MONARCH_OK) return MONARCH_ERR_CUDA;
+    CopyState &s = *cs;
+    const std::vector<cudaEvent_t> &ev = s.ev;
     // the computation must not start before earlier work on the caller's stream
     // is done with the device buffers: uploads wait for it
-    cudaEvent_t start = nullptr;
-    if (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess) return MONARCH_ERR_CUDA;
-    e.ev.push_back(start);
+    cudaEvent_t start = ev[2 * n];
     if (cudaEventRecord(start, compute) != cudaSuccess || cudaStreamWaitEvent(s.up, start, 0) != cudaSuccess)
         return MONARCH_ERR_CUDA;
     int st = MONARCH_OK;
@@ -97,7 +93,7 @@ extern "C" int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k,
         const size_t off = static_cast<size_t>(b0) * per_bh, bytes = static_cast<size_t>(b1 - b0) * per_bh;
         auto dev = [&](void *p) { return static_cast<void *>(static_cast<uint8_t *>(p) + off); };
         auto host = [&](const void *p) { return static_cast<const void *>(static_cast<const uint8_t *>(p) + off); };
-        cudaEvent_t in = e.ev[2 * c], out = e.ev[2 * c + 1];
+        cudaEvent_t in = ev[2 * c], out = ev[2 * c + 1];
         if (cudaMemcpyAsync(dev(d_q), host(h_q), bytes, cudaMemcpyHostToDevice, s.up) != cudaSuccess ||
             cudaMemcpyAsync(dev(d_k), host(h_k), bytes, cudaMemcpyHostToDevice, s.up) != cudaSuccess ||
             cudaMemcpyAsync(dev(d_v), host(h_v), bytes, cudaMemcpyHostToDevice, s.up) != cudaSuccess ||
@@ -114,7 +110,7 @@ extern "C" int monarch_attn_fwd_host_pipelined(const void *h_q, const void *h_k,
                             s.down) != cudaSuccess)
             st = MONARCH_ERR_CUDA;
     }
-    // the events are released only after all queued work is done
+    // the events are reused by the next call only after all queued work is done
     const cudaError_t e1 = cudaStreamSynchronize(s.up), e2 = cudaStreamSynchronize(compute),
                       e3 = cudaStreamSynchronize(s.down);
     if (st == MONARCH_OK && (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess)) st = MONARCH_ERR_CUDA;
