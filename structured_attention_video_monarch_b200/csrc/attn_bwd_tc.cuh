@@ -23,10 +23,10 @@
 // and an MN-major B operand (K = rows, N = d).  Every output row has one
 // owning CTA: no atomics.
 //
-// Roles (256 threads): warp 0 lane 0 controls loads and MMAs; warp 1
-// allocates TMEM; warps 4-7 (TMEM lanes 0-127, thread = row) do the
-// elementwise work.  Single-buffered: load, MMA, elementwise, MMA per tile.
-// Every wait is a bounded mbarrier wait.
+// Roles (384 threads): warp 0 lane 0 controls loads and MMAs; warp 1
+// allocates TMEM; warps 4-11 do the elementwise work, two threads per row
+// (thread = TMEM lane and column half).  The streamed tiles are double
+// buffered.  Every wait is a bounded mbarrier wait.
 #pragma once
 
 #include "sm100.cuh"
@@ -68,12 +68,15 @@ struct BwdLayout {
     static constexpr int OFF_C = OFF_B + TILE;         // dq: K_j [2]    dkdv: Q_i [2]
     static constexpr int OFF_E = OFF_C + 2 * TILE;     // dq: Vals_j [2] dkdv: dY_i [2]
     static constexpr int OFF_BAR = OFF_E + 2 * TILE;
-    // ld_full[2] (one per buffer), mma_done, ew_done, mm2_done, fin, ls_ready
-    static constexpr int NBAR = 7;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8 + 8;  // tmem base, abort flag (16-byte aligned)
-    // dk/dv kernel: LSE and rowsum terms of the current query tile's rows, [2 tiles][128]
+    // ld_full[2] (one per buffer), mma_done, ew_done, mm2_done, fin, ls_ready, x_ready
+    static constexpr int NBAR = 8;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+    // dk/dv kernel: LSE and rowsum terms of the current query tile's rows, [2 tiles][2][128];
+    // dq kernel: each column half's running (max, sum) of every row, [2 halves][128][2]
     static constexpr int OFF_LS = OFF_MISC + 16;
     static constexpr int BYTES = OFF_LS + 2 * 2 * 128 * 4;
+    // 8 elementwise warps: thread = (row, column half)
+    static constexpr int THREADS = 384;
     static constexpr int SLACK = 1024;
     // Every CTA allocates all 512 TMEM columns, so a second CTA on the same SM
     // could only block in tcgen05.alloc until the first one exits.  Asking for
@@ -82,6 +85,11 @@ struct BwdLayout {
     static constexpr int ALLOC = BYTES + SLACK > ONE_PER_SM ? BYTES + SLACK : ONE_PER_SM;
     static_assert(ALLOC <= 232448, "too much shared memory");
     static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_ACC0 = 256, COL_ACC1 = 256 + D;
+    // 16-bit pairs written over a 128-column S or dP region: column half h
+    // (keys 64h .. 64h+63) packs into columns [64h, 64h + 32) of the region,
+    // inside the columns it read itself, so the two halves never touch each
+    // other's data; the TMEM-operand MMA reads K steps 4-7 from there
+    static constexpr uint32_t pack_col(int h, int c) { return 64u * h + 16u * (c - 2 * h); }
 };
 
 // Problem geometry: which tokens a 128-row tile holds and which (row, col)
@@ -198,8 +206,9 @@ __device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uin
     constexpr uint32_t IDESC = F16 ? idesc_f16_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
     const uint32_t b = sdesc_sw128_lo(b_addr, 16384);
     mma_ts_lh(d_tmem, a_tmem, b, MN_HI, IDESC, accumulate ? 1u : 0u);
+    // keys 0-63 are packed in columns [0, 32) of the A region, keys 64-127 in [64, 96)
 #pragma unroll
-    for (int k = 1; k < 8; ++k) mma_ts_lh(d_tmem, a_tmem + k * 8, b + k * 128, MN_HI, IDESC, 1u);
+    for (int k = 1; k < 8; ++k) mma_ts_lh(d_tmem, a_tmem + k * 8 + (k >= 4 ? 32 : 0), b + k * 128, MN_HI, IDESC, 1u);
 }
 
 template <bool F16>
@@ -213,7 +222,7 @@ __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
 // ------------------------------------------------------------------ dq kernel
 // grid: one CTA per (bh, problem, query tile).  Maps: q, k, vals, dy (same geometry).
 template <int D, bool F16, int KIND>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
                const BwdParams p) {
@@ -228,6 +237,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     // ld_full(b): the tiles of buffer b landed; then mma_done, ew_done, mm2_done, fin
     auto ld_full = [&](int b) { return bar0 + 8u * static_cast<uint32_t>(b); };
     const uint32_t mma_done = bar0 + 16, ew_done = bar0 + 24, mm2_done = bar0 + 32, fin = bar0 + 40;
+    const uint32_t x_ready = bar0 + 56;  // both column halves posted their running (max, sum)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
     WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
@@ -245,9 +255,10 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         mbar_init(ld_full(0), 1);
         mbar_init(ld_full(1), 1);
         mbar_init(mma_done, 1);
-        mbar_init(ew_done, 128);
+        mbar_init(ew_done, 256);
         mbar_init(mm2_done, 1);
         mbar_init(fin, 1);
+        mbar_init(x_ready, 256);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -326,20 +337,22 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         if (ok) mma_commit(fin);
     } else if (warp >= 4) {
         // ------------------------------------------------------ elementwise threads
-        const int row = threadIdx.x - 128;  // TMEM lane
+        // thread = (row, column half h): S / dP columns [64h, 64h + 64), 32-column chunks 2h, 2h + 1
+        const int ew = threadIdx.x - 128;
+        const int row = ew & 127, h = ew >> 7;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const long long tok = BwdGeom::token(p, KIND, prob, qt, row);
         const long long rowg = tok >= 0 ? static_cast<long long>(bh) * p.N + tok : -1;
         uint32_t md_par = 0u;
         bool ok = true;
-        float m_run = -INFINITY, l_run = 0.f;  // of the scaled logits, base 2
+        float m_run = -INFINITY, l_run = 0.f;  // this half's running max and sum, base 2
         for (int j = 0; j < nk_tiles && ok; ++j) {
             ok = mbar_wait_warp(mma_done, md_par, ctl);
             md_par ^= 1u;
             if (!ok) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * h; c < 2 * h + 2; ++c) {
                 uint32_t r[32];
                 tmem_ld32(lane_base + L::COL_S + 32 * c, r);
                 const uint32_t vm = BwdGeom::col_mask(p, KIND, j, row, c);
@@ -364,18 +377,37 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(ew_done);
         }
-        const float lse = (m_run == -INFINITY) ? 0.f : m_run + __log2f(l_run);
-        if (ok && rowg >= 0) p.lse[rowg] = lse;
+        // the row's LSE from both halves' (max, sum), combined in the same
+        // order by both, so both get the same bits
+        float lse = 0.f;
+        if (ok) {
+            float *xs = reinterpret_cast<float *>(base_ptr + L::OFF_LS);
+            xs[(h * 128 + row) * 2] = m_run;
+            xs[(h * 128 + row) * 2 + 1] = l_run;
+            mbar_arrive(x_ready);
+            ok = mbar_wait_warp(x_ready, 0u, ctl);
+            if (ok) {
+                const float m0 = xs[row * 2], l0 = xs[row * 2 + 1];
+                const float m1 = xs[(128 + row) * 2], l1 = xs[(128 + row) * 2 + 1];
+                const float m = fmaxf(m0, m1);
+                if (m != -INFINITY) {
+                    const float l = (m0 == -INFINITY ? 0.f : l0 * fast_exp2(m0 - m)) +
+                                    (m1 == -INFINITY ? 0.f : l1 * fast_exp2(m1 - m));
+                    lse = m + __log2f(l);
+                }
+            }
+        }
+        if (ok && h == 0 && rowg >= 0) p.lse[rowg] = lse;
         const float dd = rowg >= 0 ? p.D[rowg] : 0.f;
         for (int j = 0; j < nk_tiles && ok; ++j) {
             ok = mbar_wait_warp(mma_done, md_par, ctl);
             md_par ^= 1u;
             if (!ok) break;
             tc_fence_after();
-            // dS = P * (dP - D), P = 2^(s*c - lse); stored as 16-bit pairs over the
-            // dP columns already read (chunk c writes [16c, 16c+16) after reading [32c, 32c+32))
+            // dS = P * (dP - D), P = 2^(s*c - lse); stored as 16-bit pairs over
+            // dP columns this thread has already read (L::pack_col)
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * h; c < 2 * h + 2; ++c) {
                 uint32_t rs[32], rp[32];
                 tmem_ld32(lane_base + L::COL_S + 32 * c, rs);
                 tmem_ld32(lane_base + L::COL_DP + 32 * c, rp);
@@ -395,7 +427,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                     }
                     pk[e] = bwd_pack<F16>(ds[0], ds[1]);
                 }
-                tmem_st16(lane_base + L::COL_DP + 16 * c, pk);
+                tmem_st16(lane_base + L::COL_DP + L::pack_col(h, c), pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -406,7 +438,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             tc_fence_after();
             float *dst = rowg >= 0 ? p.dq + rowg * D : nullptr;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
                 uint32_t r[32];
                 tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, r);
                 tmem_wait_ld();
@@ -437,7 +469,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 // ------------------------------------------------------------------ dk/dv kernel
 // grid: one CTA per (bh, problem, key tile).  Maps: k, vals (A operands), q, dy.
 template <int D, bool F16, int KIND>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                  const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
                  const BwdParams p) {
@@ -452,7 +484,7 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     // ld_full(b): the tiles of buffer b landed; then mma_done, ew_done, mm2_done, fin
     auto ld_full = [&](int b) { return bar0 + 8u * static_cast<uint32_t>(b); };
     const uint32_t mma_done = bar0 + 16, ew_done = bar0 + 24, mm2_done = bar0 + 32, fin = bar0 + 40;
-    const uint32_t ls_ready = bar0 + 48;  // the 128 elementwise threads posted a query tile's LSE and D
+    const uint32_t ls_ready = bar0 + 48;  // the 256 elementwise threads posted a query tile's LSE and D
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base_ptr + L::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(base_ptr + L::OFF_MISC + 4);
     WaitCtl ctl{abort_flag, p.status, p.timeout_cycles};
@@ -469,10 +501,10 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         mbar_init(ld_full(0), 1);
         mbar_init(ld_full(1), 1);
         mbar_init(mma_done, 1);
-        mbar_init(ew_done, 128);
+        mbar_init(ew_done, 256);
         mbar_init(mm2_done, 1);
         mbar_init(fin, 1);
-        mbar_init(ls_ready, 128);
+        mbar_init(ls_ready, 256);
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -537,13 +569,16 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         }
         if (ok) mma_commit(fin);
     } else if (warp >= 4) {
-        const int row = threadIdx.x - 128;  // key row of this tile
+        // thread = (key row, column half h): query columns [64h, 64h + 64)
+        const int ew = threadIdx.x - 128;
+        const int row = ew & 127, h = ew >> 7;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const long long tok = BwdGeom::token(p, KIND, prob, kt, row);
         const long long rowg = tok >= 0 ? static_cast<long long>(bh) * p.N + tok : -1;
         // LSE and rowsum term of each query row of the current query tile, by
-        // column: each thread posts those of its own row index; a query row
-        // that holds no token gets LSE = +inf, so its weights are exactly 0
+        // column: the two threads of row index r post those of query row r (half
+        // 0 the LSE, half 1 the rowsum term); a query row that holds no token
+        // gets LSE = +inf, so its weights are exactly 0
         float *ls_buf = reinterpret_cast<float *>(base_ptr + L::OFF_LS);
         uint32_t md_par = 0u;
         bool ok = true;
@@ -552,10 +587,12 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             {
                 const long long qtok = BwdGeom::token(p, KIND, prob, i, row);
                 const long long qg = static_cast<long long>(bh) * p.N + qtok;
-                lse_s[row] = qtok >= 0 ? __ldg(p.lse + qg) : INFINITY;
-                d_s[row] = qtok >= 0 ? __ldg(p.D + qg) : 0.f;
+                if (h == 0)
+                    lse_s[row] = qtok >= 0 ? __ldg(p.lse + qg) : INFINITY;
+                else
+                    d_s[row] = qtok >= 0 ? __ldg(p.D + qg) : 0.f;
             }
-            // wait until all 128 threads posted tile i's values (a bounded
+            // wait until all 256 threads posted tile i's values (a bounded
             // wait, like every other); the other buffer was last read in tile
             // i - 1, which every thread finished before arriving here
             mbar_arrive(ls_ready);
@@ -566,7 +603,7 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             if (!ok) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * h; c < 2 * h + 2; ++c) {
                 uint32_t rs[32], rp[32];
                 tmem_ld32(lane_base + L::COL_S + 32 * c, rs);
                 tmem_ld32(lane_base + L::COL_DP + 32 * c, rp);
@@ -587,8 +624,8 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                     pp[e] = bwd_pack<F16>(pv[0], pv[1]);
                     pd[e] = bwd_pack<F16>(dsv[0], dsv[1]);
                 }
-                tmem_st16(lane_base + L::COL_S + 16 * c, pp);
-                tmem_st16(lane_base + L::COL_DP + 16 * c, pd);
+                tmem_st16(lane_base + L::COL_S + L::pack_col(h, c), pp);
+                tmem_st16(lane_base + L::COL_DP + L::pack_col(h, c), pd);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -600,7 +637,7 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             // warp-collective); only rows holding a real key store
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
                 uint32_t rv[32], rk[32];
                 tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, rv);
                 tmem_ld32(lane_base + L::COL_ACC1 + 32 * c, rk);

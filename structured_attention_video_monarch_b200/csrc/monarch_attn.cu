@@ -756,9 +756,9 @@ int bwd_run_stage(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMa
                              static_cast<long long>(KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile);
     if (bh * per_bh >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
     const unsigned grid = static_cast<unsigned>(bh * per_bh);
-    monarch_bwd_dq<D, F16, KIND><<<grid, 256, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
+    monarch_bwd_dq<D, F16, KIND><<<grid, LB::THREADS, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
-    monarch_bwd_dkdv<D, F16, KIND><<<grid, 256, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
+    monarch_bwd_dkdv<D, F16, KIND><<<grid, LB::THREADS, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
     return cudaGetLastError() == cudaSuccess ? MONARCH_OK : MONARCH_ERR_LAUNCH;
 }
 
