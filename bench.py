@@ -343,7 +343,10 @@ def run_reference_heads(args, wl, budget):
 # or "file#region" for the text between "// <region>" and "// </region>".
 KERNEL_SOURCES = {
     "monarch_tc_kernel": ("attn_tc.cuh", "sm100.cuh", "monarch_attn.cu#tc-launch"),
-    "monarch_chunk_stage2": ("attn_chunk.cuh", "monarch_attn.cu#chunk-launch"),
+    "monarch_chunk_stage2": ("attn_chunk_mma.cuh", "attn_chunk.cuh", "monarch_attn.cu#chunk-launch"),
+    # the tensor-core backward's per-stage phases (row sums, dQ kernel, dK/dV kernel)
+    "monarch_bwd_tc_stage1": ("attn_bwd_tc.cuh", "sm100.cuh", "monarch_attn.cu#bwd-launch"),
+    "monarch_bwd_tc_stage2": ("attn_bwd_tc.cuh", "sm100.cuh", "monarch_attn.cu#bwd-launch"),
 }
 
 
@@ -366,22 +369,27 @@ def kernel_sources_sha256(kernel: str = "monarch_tc_kernel") -> str:
     return h.hexdigest()
 
 
-def traffic_source(workload: str, kernel: str = "monarch_tc_kernel") -> str:
+def profile_name(workload: str, kernel: str, part: str | None = None) -> str:
+    """Committed ncu summary of a kernel on a workload (one launch or pass of it)."""
+    return f"{kernel}_{workload}{'_' + part if part else ''}.md"
+
+
+def traffic_source(workload: str, kernel: str = "monarch_tc_kernel", part: str | None = None) -> str:
     """Where roofline.traffic comes from, or why it is null."""
-    rel = os.path.join("profiles", f"{kernel}_{workload}.md")
+    rel = os.path.join("profiles", profile_name(workload, kernel, part))
     if not os.path.exists(os.path.join(ROOT, rel)):
         return "none: no ncu summary for this kernel and workload"
-    if captured_traffic(workload, kernel) is None:
+    if captured_traffic(workload, kernel, part) is None:
         return (f"none: {rel} was taken on earlier sources (its kernel_sources_sha256 does not match "
                 "the current ones), so its DRAM counters are not reported")
     return f"{rel} (dram__bytes_read.sum + dram__bytes_write.sum of one launch)"
 
 
-def captured_traffic(workload: str, kernel: str = "monarch_tc_kernel"):
+def captured_traffic(workload: str, kernel: str = "monarch_tc_kernel", part: str | None = None):
     """DRAM bytes per launch of `kernel` from the committed ncu summary of this
     workload, or None when there is none or the kernel's sources changed since
     it was taken."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    path = os.path.join(ROOT, "profiles", profile_name(workload, kernel, part))
     if not os.path.exists(path):
         return None
     fields = {}
@@ -549,7 +557,7 @@ def run_ours(args):
     # x 1.965 GHz (nothing measured applies to CUDA-core FFMA work)
     alu_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
 
-    def rate(kernel, label, launch_idx, flops, io_bytes, alu=False):
+    def rate(kernel, label, launch_idx, flops, io_bytes, alu=False, part=None):
         per = sorted(ev[i][launch_idx].elapsed_time(ev[i][launch_idx + 1]) for i in range(args.steps))
         k_avg = statistics.mean(per) / 1e3
 
@@ -559,8 +567,8 @@ def run_ours(args):
         k_tflops = flops / k_avg / 1e12
         k_gbs = io_bytes / k_avg / 1e9
         tensor_bound = flops / io_bytes >= ridge
-        traffic = captured_traffic(wl.name, kernel)
-        t_src = traffic_source(wl.name, kernel)
+        traffic = captured_traffic(wl.name, kernel, part)
+        t_src = traffic_source(wl.name, kernel, part)
         if args.traffic is not None and launch_idx == 0 and not chunk:
             traffic, t_src = args.traffic, "--traffic argument"
         if alu:
@@ -617,13 +625,10 @@ def run_ours(args):
     elif row:
         es, bhd = 2, wl.B * wl.heads * wl.d
         r1 = rate("monarch_tc_kernel", f"monarch_tc_kernel<{wl.d}> (rows pass: blocks of W={wl.W} tokens)", 0,
-                  4.0 * wl.N * wl.W * bhd, 4 * wl.N * bhd * es)
+                  4.0 * wl.N * wl.W * bhd, 4 * wl.N * bhd * es, part="rows")
         r2 = rate("monarch_tc_kernel",
                   f"monarch_tc_kernel<{wl.d}> (columns pass: groups of T*H={wl.T * wl.H} tokens)", 1,
-                  4.0 * wl.N * wl.T * wl.H * bhd, 4 * wl.N * bhd * es)
-        # one kernel, two launches: a single ncu summary cannot give both traffics
-        r1["traffic"] = r2["traffic"] = None
-        r1["traffic_source"] = r2["traffic_source"] = "none: no per-pass ncu summary for this split"
+                  4.0 * wl.N * wl.T * wl.H * bhd, 4 * wl.N * bhd * es, part="columns")
         roofline, other = (r1, r2) if r1["launch_ms"] >= r2["launch_ms"] else (r2, r1)
         roofline = dict(roofline, other_kernel=other)
     elif chunk:

@@ -23,7 +23,8 @@
 // and an MN-major B operand (K = rows, N = d).  Every output row has one
 // owning CTA: no atomics.
 //
-// Roles (384 threads): warp 0 lane 0 controls loads and MMAs; warp 1
+// Roles (384 threads): warp 0 controls loads and MMAs (lane 0 issues the
+// TMA loads, an elected lane the MMAs, all lanes wait); warp 1
 // allocates TMEM; warps 4-11 do the elementwise work, two threads per row
 // (thread = TMEM lane and column half).  The streamed tiles are double
 // buffered.  Every wait is a bounded mbarrier wait.
@@ -175,40 +176,42 @@ __device__ __forceinline__ int bwd_load(const BwdParams &p, int kind, const CUte
     return p.npos * p.T;
 }
 
+// Zero rows [from, to) of every panel of a tile; the 32 lanes of the calling
+// warp share the 16-byte pieces.
 template <int NP>
-__device__ __forceinline__ void bwd_zero_rows(uint32_t tile, int from, int to) {
-    for (int r = from; r < to; ++r)
-#pragma unroll
-        for (int pn = 0; pn < NP; ++pn)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) st_shared_v4(tile + pn * 16384 + r * 128 + c * 16, 0, 0, 0, 0);
+__device__ __forceinline__ void bwd_zero_rows(uint32_t tile, int from, int to, int lane) {
+    for (int x = lane; x < (to - from) * NP * 8; x += 32) {
+        const int r = from + x / (NP * 8), pn = (x / 8) % NP, c = x % 8;
+        st_shared_v4(tile + pn * 16384 + r * 128 + c * 16, 0, 0, 0, 0);
+    }
 }
 
-// S-form MMA: D[128 x 128] = A[128 x d] B[128 x d]^T, both K-major SW128 tiles.
+// S-form MMA: D[128 x 128] = A[128 x d] B[128 x d]^T, both K-major SW128 tiles;
+// called by a whole converged warp (one elected lane issues).
 template <int D, bool F16>
 __device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
     constexpr uint32_t KM_HI = sdesc_sw128_hi(1024);
     constexpr uint32_t IDESC = F16 ? idesc_f16_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
     const uint32_t a = sdesc_sw128_lo(a_addr, 16), b = sdesc_sw128_lo(b_addr, 16);
-    mma_ss_lh<0>(d_tmem, a, KM_HI, b, KM_HI, IDESC);
+    mma_ss_lh_elect<0>(d_tmem, a, KM_HI, b, KM_HI, IDESC);
 #pragma unroll
     for (int k = 1; k < D / 16; ++k) {
         const uint32_t off = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-        mma_ss_lh<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, IDESC);
+        mma_ss_lh_elect<1>(d_tmem, a + off, KM_HI, b + off, KM_HI, IDESC);
     }
 }
 
-// PV-form MMA: D[128 x d] (+)= A[128 x 128] (16-bit pairs in TMEM at a_tmem)
+// PV-form MMA (called by a whole converged warp): D[128 x d] (+)= A[128 x 128] (16-bit pairs in TMEM at a_tmem)
 // * B[128 x d] (SW128 tile read MN-major: K = tile rows, N = d).
 template <int D, bool F16>
 __device__ __forceinline__ void bwd_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_addr, bool accumulate) {
     constexpr uint32_t MN_HI = sdesc_sw128_hi(1024);
     constexpr uint32_t IDESC = F16 ? idesc_f16_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
     const uint32_t b = sdesc_sw128_lo(b_addr, 16384);
-    mma_ts_lh(d_tmem, a_tmem, b, MN_HI, IDESC, accumulate ? 1u : 0u);
+    mma_ts_lh_elect(d_tmem, a_tmem, b, MN_HI, IDESC, accumulate ? 1u : 0u);
     // keys 0-63 are packed in columns [0, 32) of the A region, keys 64-127 in [64, 96)
 #pragma unroll
-    for (int k = 1; k < 8; ++k) mma_ts_lh(d_tmem, a_tmem + k * 8 + (k >= 4 ? 32 : 0), b + k * 128, MN_HI, IDESC, 1u);
+    for (int k = 1; k < 8; ++k) mma_ts_lh_elect(d_tmem, a_tmem + k * 8 + (k >= 4 ? 32 : 0), b + k * 128, MN_HI, IDESC, 1u);
 }
 
 template <bool F16>
@@ -271,7 +274,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     const uint32_t tmem = *tmem_slot;
     const uint32_t tq = base + L::OFF_A, tdy = base + L::OFF_B, tk = base + L::OFF_C, tv = base + L::OFF_E;
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
         // ------------------------------------------------------ control thread
         // Tiles g = 0 .. 2*nk - 1: pass 1 (g < nk) computes S = Q K_g^T for
         // the row LSE; pass 2 (key tile j = g - nk) computes S and dP = dY Vals_j^T,
@@ -288,53 +291,56 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             const int jt = pass2 ? g - nk_tiles : g;
             const uint32_t kb = tk + b * L::TILE, vb = tv + b * L::TILE;
             if (pass2 && rows < 128) {  // K rows the dQ MMA reads but TMA does not write
-                bwd_zero_rows<NP>(kb, rows, 128);
+                bwd_zero_rows<NP>(kb, rows, 128, lane);
                 fence_proxy_async_smem();
             }
             const int ntiles = 1 + (g == 0) + (pass2 ? 1 : 0) + (g == nk_tiles);
-            mbar_arrive_expect_tx(ld_full(b), ntiles * NP * rows * 128);
-            if (g == 0) bwd_load<NP>(p, KIND, &mq, tq, ld_full(b), bh, prob, qt);
-            if (g == nk_tiles) bwd_load<NP>(p, KIND, &mdy, tdy, ld_full(b), bh, prob, qt);
-            bwd_load<NP>(p, KIND, &mk, kb, ld_full(b), bh, prob, jt);
-            if (pass2) bwd_load<NP>(p, KIND, &mvals, vb, ld_full(b), bh, prob, jt);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(ld_full(b), ntiles * NP * rows * 128);
+                if (g == 0) bwd_load<NP>(p, KIND, &mq, tq, ld_full(b), bh, prob, qt);
+                if (g == nk_tiles) bwd_load<NP>(p, KIND, &mdy, tdy, ld_full(b), bh, prob, qt);
+                bwd_load<NP>(p, KIND, &mk, kb, ld_full(b), bh, prob, jt);
+                if (pass2) bwd_load<NP>(p, KIND, &mvals, vb, ld_full(b), bh, prob, jt);
+            }
+            __syncwarp();
         };
         issue_load(0);
         for (int g = 0; g < ng && ok; ++g) {
             const int b = g & 1;
             if (g > 0) {
                 if (g - 1 < nk_tiles) {  // pass-1 tile g-1: its S was read (its MMA is complete)
-                    ok = mbar_wait(ew_done, ew_par, ctl);
+                    ok = mbar_wait_warp(ew_done, ew_par, ctl);
                     ew_par ^= 1u;
                 } else {  // pass-2 tile g-1: its dQ MMA (the last reader of its buffers and of dS) is complete
-                    ok = mbar_wait(mm2_done, m2_par, ctl);
+                    ok = mbar_wait_warp(mm2_done, m2_par, ctl);
                     m2_par ^= 1u;
                 }
                 if (!ok) break;
             }
             if (g + 1 < ng) issue_load(g + 1);  // into the buffer tile g-1 used
-            ok = mbar_wait(ld_full(b), static_cast<uint32_t>(g >> 1) & 1u, ctl);
+            ok = mbar_wait_warp(ld_full(b), static_cast<uint32_t>(g >> 1) & 1u, ctl);
             if (!ok) break;
             tc_fence_after();
             const uint32_t kb = tk + b * L::TILE, vb = tv + b * L::TILE;
             bwd_mma_ss<D, F16>(tmem + L::COL_S, tq, kb);
             if (g < nk_tiles) {
-                mma_commit(mma_done);
+                mma_commit_elect(mma_done);
                 continue;
             }
             bwd_mma_ss<D, F16>(tmem + L::COL_DP, tdy, vb);
-            mma_commit(mma_done);
-            ok = mbar_wait(ew_done, ew_par, ctl);  // dS stored (16-bit pairs at COL_DP)
+            mma_commit_elect(mma_done);
+            ok = mbar_wait_warp(ew_done, ew_par, ctl);  // dS stored (16-bit pairs at COL_DP)
             ew_par ^= 1u;
             if (!ok) break;
             tc_fence_after();
             bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_DP, kb, g > nk_tiles);
-            mma_commit(mm2_done);
+            mma_commit_elect(mm2_done);
         }
         if (ok) {
-            ok = mbar_wait(mm2_done, m2_par, ctl);
+            ok = mbar_wait_warp(mm2_done, m2_par, ctl);
             m2_par ^= 1u;
         }
-        if (ok) mma_commit(fin);
+        if (ok) mma_commit_elect(fin);
     } else if (warp >= 4) {
         // ------------------------------------------------------ elementwise threads
         // thread = (row, column half h): S / dP columns [64h, 64h + 64), 32-column chunks 2h, 2h + 1
@@ -343,6 +349,8 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const long long tok = BwdGeom::token(p, KIND, prob, qt, row);
         const long long rowg = tok >= 0 ? static_cast<long long>(bh) * p.N + tok : -1;
+        // the row's rowsum term, needed in pass 2: loaded now, used after pass 1
+        const float dd = rowg >= 0 ? p.D[rowg] : 0.f;
         uint32_t md_par = 0u;
         bool ok = true;
         float m_run = -INFINITY, l_run = 0.f;  // this half's running max and sum, base 2
@@ -398,7 +406,6 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             }
         }
         if (ok && h == 0 && rowg >= 0) p.lse[rowg] = lse;
-        const float dd = rowg >= 0 ? p.D[rowg] : 0.f;
         for (int j = 0; j < nk_tiles && ok; ++j) {
             ok = mbar_wait_warp(mma_done, md_par, ctl);
             md_par ^= 1u;
@@ -433,21 +440,23 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(ew_done);
         }
+        // this half's dQ columns of the other stage, loaded while the last dQ
+        // MMA runs (the epilogue adds to them)
+        float *dst = rowg >= 0 ? p.dq + rowg * D + h * (D / 2) : nullptr;
+        float prev[D / 2];
+#pragma unroll
+        for (int e = 0; e < D / 2; ++e) prev[e] = (dst && p.add_dq) ? dst[e] : 0.f;
         if (ok) ok = mbar_wait_warp(fin, 0u, ctl);
         if (ok) {
             tc_fence_after();
-            float *dst = rowg >= 0 ? p.dq + rowg * D : nullptr;
-#pragma unroll 1
-            for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t r[32];
-                tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, r);
+                tmem_ld32(lane_base + L::COL_ACC0 + h * (D / 2) + 32 * c, r);
                 tmem_wait_ld();
                 if (dst) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float v = __uint_as_float(r[e]) * p.scale;
-                        dst[32 * c + e] = p.add_dq ? dst[32 * c + e] + v : v;
-                    }
+                    for (int e = 0; e < 32; ++e) dst[32 * c + e] = prev[32 * c + e] + __uint_as_float(r[e]) * p.scale;
                 }
                 __syncwarp();
             }
@@ -517,7 +526,7 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     const uint32_t tk = base + L::OFF_A, tv = base + L::OFF_B, tq = base + L::OFF_C, tdy = base + L::OFF_E;
 
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
         // Query tile i's Q and dY land in buffer i & 1, loaded while tile
         // i - 1 is computed; K and Vals arrive with tile 0.
         uint32_t ew_par = 0u, m2_par = 0u;
@@ -527,47 +536,50 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             const int b = i & 1;
             const uint32_t qb = tq + b * L::TILE, yb = tdy + b * L::TILE;
             if (rows < 128) {  // Q and dY rows the dK/dV MMAs read but TMA does not write
-                bwd_zero_rows<NP>(qb, rows, 128);
-                bwd_zero_rows<NP>(yb, rows, 128);
+                bwd_zero_rows<NP>(qb, rows, 128, lane);
+                bwd_zero_rows<NP>(yb, rows, 128, lane);
                 fence_proxy_async_smem();
             }
-            mbar_arrive_expect_tx(ld_full(b), (i == 0 ? 4 : 2) * NP * rows * 128);
-            if (i == 0) {
-                bwd_load<NP>(p, KIND, &mk, tk, ld_full(b), bh, prob, kt);
-                bwd_load<NP>(p, KIND, &mvals, tv, ld_full(b), bh, prob, kt);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(ld_full(b), (i == 0 ? 4 : 2) * NP * rows * 128);
+                if (i == 0) {
+                    bwd_load<NP>(p, KIND, &mk, tk, ld_full(b), bh, prob, kt);
+                    bwd_load<NP>(p, KIND, &mvals, tv, ld_full(b), bh, prob, kt);
+                }
+                bwd_load<NP>(p, KIND, &mq, qb, ld_full(b), bh, prob, i);
+                bwd_load<NP>(p, KIND, &mdy, yb, ld_full(b), bh, prob, i);
             }
-            bwd_load<NP>(p, KIND, &mq, qb, ld_full(b), bh, prob, i);
-            bwd_load<NP>(p, KIND, &mdy, yb, ld_full(b), bh, prob, i);
+            __syncwarp();
         };
         issue_load(0);
         for (int i = 0; i < nq_tiles && ok; ++i) {
             const int b = i & 1;
             if (i > 0) {  // the dV/dK MMAs of tile i-1 (the last readers of its buffers, P^T and dS^T) are complete
-                ok = mbar_wait(mm2_done, m2_par, ctl);
+                ok = mbar_wait_warp(mm2_done, m2_par, ctl);
                 m2_par ^= 1u;
                 if (!ok) break;
             }
             if (i + 1 < nq_tiles) issue_load(i + 1);  // into the buffer tile i-1 used
-            ok = mbar_wait(ld_full(b), static_cast<uint32_t>(i >> 1) & 1u, ctl);
+            ok = mbar_wait_warp(ld_full(b), static_cast<uint32_t>(i >> 1) & 1u, ctl);
             if (!ok) break;
             tc_fence_after();
             const uint32_t qb = tq + b * L::TILE, yb = tdy + b * L::TILE;
             bwd_mma_ss<D, F16>(tmem + L::COL_S, tk, qb);    // S^T = K Q^T
             bwd_mma_ss<D, F16>(tmem + L::COL_DP, tv, yb);   // dP^T = Vals dY^T
-            mma_commit(mma_done);
-            ok = mbar_wait(ew_done, ew_par, ctl);  // P^T at COL_S, dS^T at COL_DP (16-bit pairs)
+            mma_commit_elect(mma_done);
+            ok = mbar_wait_warp(ew_done, ew_par, ctl);  // P^T at COL_S, dS^T at COL_DP (16-bit pairs)
             ew_par ^= 1u;
             if (!ok) break;
             tc_fence_after();
             bwd_mma_ts<D, F16>(tmem + L::COL_ACC0, tmem + L::COL_S, yb, i > 0);   // dV += P^T dY
             bwd_mma_ts<D, F16>(tmem + L::COL_ACC1, tmem + L::COL_DP, qb, i > 0);  // dK += dS^T Q
-            mma_commit(mm2_done);
+            mma_commit_elect(mm2_done);
         }
         if (ok) {
-            ok = mbar_wait(mm2_done, m2_par, ctl);
+            ok = mbar_wait_warp(mm2_done, m2_par, ctl);
             m2_par ^= 1u;
         }
-        if (ok) mma_commit(fin);
+        if (ok) mma_commit_elect(fin);
     } else if (warp >= 4) {
         // thread = (key row, column half h): query columns [64h, 64h + 64)
         const int ew = threadIdx.x - 128;
@@ -580,18 +592,20 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         // 0 the LSE, half 1 the rowsum term); a query row that holds no token
         // gets LSE = +inf, so its weights are exactly 0
         float *ls_buf = reinterpret_cast<float *>(base_ptr + L::OFF_LS);
+        // tile i's value is loaded during tile i - 1 (its latency overlaps that tile's work)
+        auto fetch = [&](int i) -> float {
+            const long long qtok = BwdGeom::token(p, KIND, prob, i, row);
+            const long long qg = static_cast<long long>(bh) * p.N + qtok;
+            if (h == 0) return qtok >= 0 ? __ldg(p.lse + qg) : INFINITY;
+            return qtok >= 0 ? __ldg(p.D + qg) : 0.f;
+        };
+        float next = fetch(0);
         uint32_t md_par = 0u;
         bool ok = true;
         for (int i = 0; i < nq_tiles && ok; ++i) {
             float *lse_s = ls_buf + (i & 1) * 256, *d_s = lse_s + 128;
-            {
-                const long long qtok = BwdGeom::token(p, KIND, prob, i, row);
-                const long long qg = static_cast<long long>(bh) * p.N + qtok;
-                if (h == 0)
-                    lse_s[row] = qtok >= 0 ? __ldg(p.lse + qg) : INFINITY;
-                else
-                    d_s[row] = qtok >= 0 ? __ldg(p.D + qg) : 0.f;
-            }
+            (h == 0 ? lse_s : d_s)[row] = next;
+            if (i + 1 < nq_tiles) next = fetch(i + 1);
             // wait until all 256 threads posted tile i's values (a bounded
             // wait, like every other); the other buffer was last read in tile
             // i - 1, which every thread finished before arriving here
@@ -631,13 +645,19 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
             tc_fence_before();
             mbar_arrive(ew_done);
         }
+        // this half's dK columns of the other stage, loaded while the last
+        // MMAs run (the epilogue adds to them)
+        float prev[D / 2];
+#pragma unroll
+        for (int e = 0; e < D / 2; ++e) prev[e] = (rowg >= 0 && p.add_dk) ? p.dk[rowg * D + h * (D / 2) + e] : 0.f;
         if (ok) ok = mbar_wait_warp(fin, 0u, ctl);
         if (ok) {
             // every lane of the warp takes part in the TMEM loads (they are
             // warp-collective); only rows holding a real key store
             tc_fence_after();
-#pragma unroll 1
-            for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+                const int c = h * (D / 64) + cc;
                 uint32_t rv[32], rk[32];
                 tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, rv);
                 tmem_ld32(lane_base + L::COL_ACC1 + 32 * c, rk);
@@ -649,7 +669,7 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                         const float dvv = __uint_as_float(rv[e]);
                         const float dkv = __uint_as_float(rk[e]) * p.scale;
                         if (p.dv) p.dv[o] = dvv;
-                        p.dk[o] = p.add_dk ? p.dk[o] + dkv : dkv;
+                        p.dk[o] = prev[32 * cc + e] + dkv;
                     }
                     if (p.dv16) {
                         uint32_t w[16];

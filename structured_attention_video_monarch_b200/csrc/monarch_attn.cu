@@ -664,6 +664,7 @@ int launch_row(const void *q, const void *k, const void *v, void *out, const Sha
 }
 
 
+// <bwd-launch> (hashed with attn_bwd_tc.cuh by the profile summaries)
 // ---------------------------------------------------------------- gradients
 // bf16 / fp16 gradients on tensor cores (attn_bwd_tc.cuh), orchestrated here
 // beside the forward's launch code, whose kernels recompute Y1 and O.
@@ -853,6 +854,8 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
     lev.record(++lev.launches, stream);
     return MONARCH_OK;
 }
+
+// </bwd-launch>
 
 // <chunk-launch> (hashed with attn_chunk.cuh by the profile summaries)
 // Stage 2 of an autoregressive chunk (attn_chunk.cuh).

@@ -101,3 +101,19 @@ def test_interleaved_streams_share_pools_in_order():
     torch.cuda.synchronize()
     for a, b in outs:
         assert torch.equal(a, ref) and torch.equal(b, ref2)
+
+
+def test_counter_pool_grows_for_many_batch_heads():
+    """More batch-heads than the counter pool's first slot size (4096 plus the
+    unit-claim counter): the pool is reallocated larger, earlier slots retired,
+    and the result still matches the oracle."""
+    import oracle
+    dev = torch.device("cuda:0")
+    B, heads, T, H, W, d = 2, 2500, 2, 1, 3, 64
+    q, k, v = workloads.random_inputs(B, heads, T, H, W, d, seed=21)
+    got = binding.monarch_attn_fwd(*(x.to(dev) for x in (q, k, v)), T, H, W)
+    torch.cuda.synchronize()
+    assert binding.last_device_error() == 0
+    ref = oracle.monarch_fwd(q, k, v, T, H, W)
+    err = (got.cpu().double() - torch.from_numpy(ref)).abs().max().item()
+    assert err <= 2e-2
