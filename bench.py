@@ -445,7 +445,7 @@ def run_ours(args):
         sets.append(bufs)
     stream = torch.cuda.current_stream(device)
 
-    grad16 = grad and wl.dtype != "f32"  # tensor-core gradients: five timed phases
+    grad16 = grad and wl.dtype != "f32"  # tensor-core gradients: four timed phases
 
     def call(i, events=None):
         if grad:
@@ -454,10 +454,10 @@ def run_ours(args):
                 if events is None:
                     binding.monarch_attn_bwd(q, k, v, do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w,
                                              out=(dq, dk, dv), workspace=ws)
-                    return 11  # 2 recomputations, 2 x (row sums, dQ, dK/dV), 3 casts
+                    return 8  # 2 recomputations, 2 x (row sums, dQ, dK/dV)
                 binding.monarch_attn_bwd_profiled(q, k, v, do, dq, dk, dv, ws, wl.T, wl.H, wl.W, events,
                                                   wl.fact, wl.tile_h, wl.tile_w)
-                return 11
+                return 8
             if events is not None:
                 events[0].record(stream)
             binding.monarch_attn_bwd(q, k, v, do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w,
@@ -497,7 +497,7 @@ def run_ours(args):
     torch.cuda.synchronize(device)
 
     # timed region: K calls, events around each kernel launch
-    nev = 6 if grad16 else 3
+    nev = 5 if grad16 else 3
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     for e in (x for row in ev for x in row):
         e.record(stream)  # torch creates the CUDA event on first record; the library needs the handle
@@ -605,18 +605,17 @@ def run_ours(args):
         }
 
     if grad16:
-        # phases: 0 Y1 recompute, 1 O recompute, 2 stage-2 backward, 3 stage-1 backward, 4 casts.
+        # phases: 0 Y1 recompute, 1 O recompute, 2 stage-2 backward, 3 stage-1 backward (writes the outputs).
         # The stage-1 backward (row sums, the dQ kernel and the dK/dV kernel over
         # frame blocks) carries 10*d FLOPs per (query, key) pair of the blocks.
         es, bhd = 2, wl.B * wl.heads * wl.d
-        # bytes: read Q, K, V, dY1, Y1 (16-bit); read-modify-write dQ, dK and write dV (fp32)
+        # bytes: read Q, K, V, dY1, Y1 (16-bit) and stage 2's dQ, dK parts (fp32); write dQ, dK, dV (16-bit)
         b1 = rate("monarch_bwd_tc_stage1", f"monarch_bwd_dq + monarch_bwd_dkdv<{wl.d}> (stage-1 blocks of "
-                  f"m={wl.m})", 3, 10.0 * wl.N * wl.m * bhd, (5 * es + 2 * 8 + 4) * wl.N * bhd)
+                  f"m={wl.m})", 3, 10.0 * wl.N * wl.m * bhd, (5 * es + 2 * 4 + 3 * es) * wl.N * bhd)
         b2 = rate("monarch_bwd_tc_stage2", f"monarch_bwd_dq + monarch_bwd_dkdv<{wl.d}> (stage-2 groups of "
                   f"b={wl.b})", 2, 10.0 * wl.N * wl.b * bhd, (5 * es + 2 * 4 + es) * wl.N * bhd)
         phase_ms = {}
-        for name, idx in (("recompute_y1", 0), ("recompute_o", 1), ("stage2_bwd", 2), ("stage1_bwd", 3),
-                          ("casts", 4)):
+        for name, idx in (("recompute_y1", 0), ("recompute_o", 1), ("stage2_bwd", 2), ("stage1_bwd", 3)):
             phase_ms[name] = statistics.mean(ev[i][idx].elapsed_time(ev[i][idx + 1]) for i in range(args.steps))
         roofline = dict(b1, other_kernel=b2, phases_ms=phase_ms)
     elif grad:

@@ -49,11 +49,13 @@ struct BwdParams {
     float scale;          // d^-1/2
     const float *D;       // per row: rowsum(dY * Y) of this stage, [BH][N]
     float *lse;           // per row: log2-sum-exp of the scaled logits, [BH][N] (dq writes, dkdv reads)
-    float *dq;            // fp32 [BH][N][d]; accumulate (add_dq) or write
-    float *dk;            // fp32 [BH][N][d]; accumulate (add_dk) or write
-    float *dv;            // fp32 [BH][N][d] (written), or null
-    void *dv16;           // 16-bit copy of dv [BH][N][d] (written), or null
+    float *dq;            // fp32 [BH][N][d]: written, or (add_dq) the other stage's part read
+    float *dk;            // fp32 [BH][N][d]: written, or (add_dk) the other stage's part read
+    void *dv16;           // value gradient in 16 bits [BH][N][d] (written), or null
     int add_dq, add_dk;
+    // 16-bit final gradients [BH][N][d] (input dtype): when set, the kernel
+    // adds the other stage's fp32 part and writes the result here
+    void *out_dq, *out_dk;
     long long timeout_cycles;
     unsigned *status;
 };
@@ -454,7 +456,16 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 uint32_t r[32];
                 tmem_ld32(lane_base + L::COL_ACC0 + h * (D / 2) + 32 * c, r);
                 tmem_wait_ld();
-                if (dst) {
+                if (dst && p.out_dq) {  // final dQ in 16 bits
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = bwd_pack<F16>(prev[32 * c + 2 * e] + __uint_as_float(r[2 * e]) * p.scale,
+                                             prev[32 * c + 2 * e + 1] + __uint_as_float(r[2 * e + 1]) * p.scale);
+                    uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out_dq) + rowg * D + h * (D / 2) + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                } else if (dst) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) dst[32 * c + e] = prev[32 * c + e] + __uint_as_float(r[e]) * p.scale;
                 }
@@ -662,15 +673,20 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
                 tmem_ld32(lane_base + L::COL_ACC0 + 32 * c, rv);
                 tmem_ld32(lane_base + L::COL_ACC1 + 32 * c, rk);
                 tmem_wait_ld();
-                if (rowg >= 0) {
+                if (rowg >= 0 && p.out_dk) {  // final dK in 16 bits
+                    uint32_t w[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const long long o = rowg * D + 32 * c + e;
-                        const float dvv = __uint_as_float(rv[e]);
-                        const float dkv = __uint_as_float(rk[e]) * p.scale;
-                        if (p.dv) p.dv[o] = dvv;
-                        p.dk[o] = prev[32 * cc + e] + dkv;
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = bwd_pack<F16>(prev[32 * cc + 2 * e] + __uint_as_float(rk[2 * e]) * p.scale,
+                                             prev[32 * cc + 2 * e + 1] + __uint_as_float(rk[2 * e + 1]) * p.scale);
+                    uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out_dk) + rowg * D + 32 * c);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                } else if (rowg >= 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) p.dk[rowg * D + 32 * c + e] = prev[32 * cc + e] + __uint_as_float(rk[e]) * p.scale;
+                }
+                if (rowg >= 0) {
                     if (p.dv16) {
                         uint32_t w[16];
 #pragma unroll

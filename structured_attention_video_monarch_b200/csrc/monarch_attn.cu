@@ -693,21 +693,10 @@ __global__ void bwd_rowdot(const E *a, const E *b, float *out, long long rows) {
     if (lane == 0) out[r] = s;
 }
 
-template <typename E>
-__global__ void bwd_cast(const float *in, E *out, long long n) {
-    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<long long>(gridDim.x) * blockDim.x) {
-        if constexpr (std::is_same<E, __half>::value)
-            out[i] = __float2half_rn(in[i]);
-        else
-            out[i] = __float2bfloat16_rn(in[i]);
-    }
-}
-
 // Workspace (bytes): Y1, O, dY1 (16-bit, N*d each), LSE and D (fp32, N each),
-// dq, dk, dv accumulators (fp32, N*d each); per batch-head.
+// stage 2's dq and dk parts (fp32, N*d each); per batch-head.
 size_t bwd_tc_workspace(long long bh, long long N, int d, int es) {
-    return static_cast<size_t>(bh * N) * (3 * d * es + 2 * 4 + 3 * d * 4);
+    return static_cast<size_t>(bh * N) * (3 * d * es + 2 * 4 + 2 * d * 4);
 }
 
 // Geometry of one stage from a (possibly virtual) frame or tiled shape, and the
@@ -780,7 +769,6 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
     float *dd = lse + bh * N;
     float *dq32 = dd + bh * N;
     float *dk32 = dq32 + nd;
-    float *dv32 = dk32 + nd;
     const bool row = s.fact == MONARCH_FACT_ROW;
     // the two stages' shapes: the (f*h, w) split runs both as stage-1
     // geometries of virtual shapes (rows: one-row frames; columns: one tall
@@ -808,7 +796,7 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         BwdParams p{};
         TcParams tp{};
         bwd_geometry(s2, D, p, tp);
-        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 0; p.dk = dk32; p.add_dk = 0; p.dv = nullptr; p.dv16 = dy1;
+        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 0; p.dk = dk32; p.add_dk = 0; p.dv16 = dy1;
         p.timeout_cycles = env_timeout_cycles();
         p.status = status;
         bwd_rowdot<D, E><<<rd_grid, 256, 0, stream>>>(static_cast<const E *>(dout), o, dd, rows);
@@ -833,7 +821,9 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         BwdParams p{};
         TcParams tp{};
         bwd_geometry(s1, D, p, tp);
-        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 1; p.dk = dk32; p.add_dk = 1; p.dv = dv32; p.dv16 = nullptr;
+        // adds stage 2's fp32 parts and writes the final 16-bit gradients
+        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 1; p.dk = dk32; p.add_dk = 1; p.dv16 = dv;
+        p.out_dq = dq; p.out_dk = dk;
         p.timeout_cycles = env_timeout_cycles();
         p.status = status;
         bwd_rowdot<D, E><<<rd_grid, 256, 0, stream>>>(dy1, y1, dd, rows);
@@ -847,11 +837,6 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         if (st) return st;
         lev.record(++lev.launches, stream);
     }
-    bwd_cast<E><<<4 * di->sms, 256, 0, stream>>>(dq32, static_cast<E *>(dq), nd);
-    bwd_cast<E><<<4 * di->sms, 256, 0, stream>>>(dk32, static_cast<E *>(dk), nd);
-    bwd_cast<E><<<4 * di->sms, 256, 0, stream>>>(dv32, static_cast<E *>(dv), nd);
-    if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
-    lev.record(++lev.launches, stream);
     return MONARCH_OK;
 }
 
