@@ -57,6 +57,8 @@ struct TcParams {
     int tile_h, tile_w, tiles_h, tiles_w;
     int rows_per_tile;              // tiled: tile rows per 128-row query/key tile
     int m;                          // tokens per stage-1 block
+    int sub;                        // > 0: a stage-1 block packs m / sub independent sub-blocks of
+                                    // sub consecutive tokens (a query sees keys of its own one only)
     int nblk_bh;                    // stage-1 blocks per (batch, head)
     int nblocks;                    // stage-1 blocks in all
     int nqt;                        // 128-row query (= key) tiles per stage-1 block
@@ -250,6 +252,15 @@ __device__ __forceinline__ long long lane_row_token(const TcParams &p, int kind,
 __device__ __forceinline__ uint64_t stage1_valid_bits(int n) {
     return n >= 64 ? ~0ull : (n <= 0 ? 0ull : ((1ull << n) - 1ull));
 }
+// Bit c set when column c of the 64-column half h of key tile j lies in the
+// sub-block of block-local query qi (packed blocks: keys [g*sub, g*sub+sub)
+// with g = qi / sub).
+__device__ __forceinline__ uint64_t sub_valid_bits(int g_lo, int sub, int j, int h) {
+    const int lo = g_lo - (j * 128 + 64 * h), hi = lo + sub;
+    const uint64_t below_hi = hi >= 64 ? ~0ull : (hi <= 0 ? 0ull : ((1ull << hi) - 1ull));
+    const uint64_t below_lo = lo >= 64 ? ~0ull : (lo <= 0 ? 0ull : ((1ull << lo) - 1ull));
+    return below_hi & ~below_lo;
+}
 __device__ __noinline__ uint64_t stage2_valid_bits(const TcParams &p, int h, int prow, int npos_valid) {
     uint64_t vm = 0;
     if (prow >= npos_valid) return 0;
@@ -372,7 +383,10 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t sca
     }
 }
 
-template <int D, bool F16>
+// PACK: stage-1 blocks pack sub-blocks of p.sub tokens (the packed rows pass of
+// the (f*h, w) split); a separate instantiation, so the other kernels carry
+// none of its masking.
+template <int D, bool F16, bool PACK>
 __global__ void __launch_bounds__(640, 1)
 monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant__ CUtensorMap mk1,
                   const __grid_constant__ CUtensorMap mv1, const __grid_constant__ CUtensorMap mq2,
@@ -739,6 +753,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             // stage-2 mask: the row belongs to position slot prow of its chunk
             const int prow = (un.kind == UNIT_STAGE2) ? static_cast<int>(fmod_(row, p.fd_npos)) : 0;
             int npos_valid = 0;
+            // packed stage-1 blocks: the first key of this row's sub-block
+            const int sub_lo = (PACK && un.kind == UNIT_STAGE1)
+                                   ? ((un.ln[li].tile * 128 + row) / p.sub) * p.sub : 0;
             if (un.kind == UNIT_STAGE2) {
                 const int rem = p.HW - un.ln[li].tile * p.npos;
                 npos_valid = rem < p.npos ? rem : p.npos;
@@ -746,7 +763,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             for (int j = 0; j < un.nk; ++j) {
                 int kvalid, ext;
                 key_extent(p, un, j, kvalid, ext);
-                const bool masked = (un.kind == UNIT_STAGE2) || (kvalid < 128);
+                const bool masked = (un.kind == UNIT_STAGE2) || (kvalid < 128) || PACK;
                 if (!mbar_wait_warp(s_full(li), sf_par, ctl)) { ok = false; break; }
                 sf_par ^= 1u;
                 tc_fence_after();
@@ -762,9 +779,11 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
                         for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[c][e]);
                 }
                 if (masked) {  // columns 64h + c: validity bits, then -inf where 0
-                    const uint64_t vm = un.kind == UNIT_STAGE1
-                                            ? stage1_valid_bits(kvalid - 64 * h)
-                                            : stage2_valid_bits(p, h, prow, npos_valid);
+                    uint64_t vm = un.kind == UNIT_STAGE1
+                                      ? stage1_valid_bits(kvalid - 64 * h)
+                                      : stage2_valid_bits(p, h, prow, npos_valid);
+                    if constexpr (PACK)
+                        if (un.kind == UNIT_STAGE1) vm &= sub_valid_bits(sub_lo, p.sub, j, h);
 #pragma unroll
                     for (int c = 0; c < 64; ++c)
                         if (!((vm >> c) & 1ull)) s[c] = -INFINITY;

@@ -35,8 +35,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     bool init = false;
     int sms = 0;
-    bool tc_attr[4] = {false, false, false, false};  // [fp16][d == 128]
-    int tc_resident[4] = {0, 0, 0, 0};                // CTAs of monarch_tc_kernel per SM
+    bool tc_attr[8] = {};    // [packed rows][fp16][d == 128]
+    int tc_resident[8] = {};  // CTAs of monarch_tc_kernel per SM
     bool f32_attr[2] = {false, false};
 };
 
@@ -439,20 +439,21 @@ struct LaunchEvents {
 template <int D, bool F16>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
               cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr,
-              bool stage1_only = false) {
+              bool stage1_only = false, int sub = 0) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
     if ((st = get_encode())) return st;
     using L = TcLayout<D>;
-    const int di_idx = (F16 ? 2 : 0) + (D == 128 ? 1 : 0);
+    const int di_idx = (sub > 0 ? 4 : 0) + (F16 ? 2 : 0) + (D == 128 ? 1 : 0);
+    const auto kernel = sub > 0 ? monarch_tc_kernel<D, F16, true> : monarch_tc_kernel<D, F16, false>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!di->tc_attr[di_idx]) {
             int occ = 0;
-            if (cudaFuncSetAttribute(monarch_tc_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      L::ALLOC) != cudaSuccess ||
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, monarch_tc_kernel<D, F16>, 640, L::ALLOC) !=
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, 640, L::ALLOC) !=
                     cudaSuccess)
                 return MONARCH_ERR_CUDA;
             if (occ < 1) return MONARCH_ERR_UNSUPPORTED;
@@ -464,6 +465,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.B = s.B; p.heads = s.heads; p.T = s.T; p.H = s.H; p.W = s.W; p.HW = s.H * s.W;
     p.N = s.N;
     p.fact = s.fact;
+    p.sub = sub;
     if (s.fact == MONARCH_FACT_TILED) {
         p.tile_h = s.tile_h; p.tile_w = s.tile_w;
         p.tiles_h = s.H / s.tile_h; p.tiles_w = s.W / s.tile_w;
@@ -570,7 +572,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     lev.start(stream);
-    if (cudaLaunchKernelEx(&cfg, monarch_tc_kernel<D, F16>, mq1, mk1, mv1, mq2, mk2, my2, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kernel, mq1, mk1, mv1, mq2, mk2, my2, p) != cudaSuccess) {
         (void)cudaGetLastError();
         return MONARCH_ERR_LAUNCH;
     }
@@ -648,12 +650,23 @@ int launch_row(const void *q, const void *k, const void *v, void *out, const Sha
     if (st) return st;
     Shape rows = s;
     rows.T = s.T * s.H; rows.H = 1; rows.fact = MONARCH_FACT_FRAME; rows.tile_h = rows.tile_w = 0;
+    // The tensor-core rows pass packs `pack` consecutive frame rows into one
+    // block of pack * W <= 128 tokens (a query tile), each row attending to its
+    // own keys only (sub-blocks of W): short rows then fill the 128-row MMA
+    // tiles instead of leaving most of each empty.  Y1 keeps its layout.
+    int pack = 1;
+    for (int c = 128 / s.W; c > 1; --c)
+        if ((s.T * s.H) % c == 0) { pack = c; break; }
     Shape cols = s;
     cols.T = 1; cols.H = s.T * s.H; cols.fact = MONARCH_FACT_TILED; cols.tile_h = s.T * s.H; cols.tile_w = 1;
     constexpr bool tc = !std::is_same<E, float>::value;
     if constexpr (tc) {
         constexpr bool f16 = std::is_same<E, __half>::value;
-        if ((st = launch_tc<D, f16>(q, k, v, y1, rows, stream, lev, nullptr, true))) return st;
+        Shape packed = rows;
+        packed.T = rows.T / pack; packed.H = pack;
+        if ((st = launch_tc<D, f16>(q, k, v, y1, pack > 1 ? packed : rows, stream, lev, nullptr, true,
+                                    pack > 1 ? s.W : 0)))
+            return st;
         st = launch_tc<D, f16>(q, k, y1, out, cols, stream, lev, nullptr, true);
     } else {
         if ((st = launch_f32<D>(q, k, v, y1, rows, stream, lev, true))) return st;

@@ -31,6 +31,8 @@ CASES = [
     (1, 1, 9, 30, 3, 64),     # columns of 270 tokens (three tiles); rows of 3
     (1, 2, 3, 1, 30, 128),    # H = 1: the frame split's blocks and groups
     (1, 1, 130, 1, 16, 128),  # more than 128 frames (allowed for this split)
+    (1, 1, 7, 1, 40, 128),    # 7 frame rows (prime count): rows of 40 stay unpacked
+    (1, 2, 6, 5, 52, 128),    # rows of 52 packed two to a query tile (the full clip's width)
 ]
 
 
