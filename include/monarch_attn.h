@@ -313,9 +313,10 @@ int monarch_attn_fwd_chunk_profiled(const void *q, const void *k, const void *v,
  *
  * dtype MONARCH_DTYPE_BF16 / MONARCH_DTYPE_F16 (tensor cores; every
  * factorisation, including MONARCH_FACT_ROW): the workspace holds the
- * recomputed Y1 and O and dY1 (16-bit), per-row LSE and rowsum terms (fp32)
- * and stage 2's dQ and dK parts (fp32): N*(6d + 8 + 8d) bytes per
- * batch-head.  The forward's kernel recomputes Y1 and O; then per stage a
+ * recomputed Y1 and O and dY1 (16-bit), per-row rowsum terms and each
+ * stage's per-row LSE (fp32) and stage 2's dQ and dK parts (fp32):
+ * N*(6d + 12 + 8d) bytes per batch-head.  The forward's kernel recomputes Y1
+ * and O, leaving each stage's row LSE as it goes; then per stage a
  * query-outer kernel (dQ) and a key-outer kernel (dK and dValues) run on
  * tcgen05 with fp32 accumulation and 16-bit P, dS and dY1; stage 1's kernels
  * add stage 2's parts and write dq, dk, dv.  Every gradient row has one

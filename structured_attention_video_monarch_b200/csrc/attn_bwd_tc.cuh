@@ -48,7 +48,8 @@ struct BwdParams {
     float scale_log2;     // d^-1/2 * log2(e)
     float scale;          // d^-1/2
     const float *D;       // per row: rowsum(dY * Y) of this stage, [BH][N]
-    float *lse;           // per row: log2-sum-exp of the scaled logits, [BH][N] (dq writes, dkdv reads)
+    float *lse;           // per row: log2-sum-exp of the scaled logits, [BH][N] (dkdv reads)
+    int lse_given;        // lse holds the forward's values (dq skips its LSE pass); else dq writes it
     float *dq;            // fp32 [BH][N][d]: written, or (add_dq) the other stage's part read
     float *dk;            // fp32 [BH][N][d]: written, or (add_dk) the other stage's part read
     void *dv16;           // value gradient in 16 bits [BH][N][d] (written), or null
@@ -284,11 +285,14 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         // Vals) land in buffer g & 1, loaded while tile g - 1 is computed; Q
         // arrives with tile 0, dY with tile nk.
         const int rows = KIND == BWD_GEOM_FRAME ? 128 : (KIND == BWD_GEOM_TILED ? p.rows_per_tile * p.tile_w : p.npos * p.T);
+        // With the LSE given, the sequence starts at pass 2 (g0 = nk).  Buffer
+        // and barrier phase follow the position i = g - g0 in the sequence.
+        const int g0 = p.lse_given ? nk_tiles : 0;
         const int ng = 2 * nk_tiles;
         uint32_t ew_par = 0u, m2_par = 0u;
         bool ok = true;
         auto issue_load = [&](int g) {
-            const int b = g & 1;
+            const int b = (g - g0) & 1;
             const bool pass2 = g >= nk_tiles;
             const int jt = pass2 ? g - nk_tiles : g;
             const uint32_t kb = tk + b * L::TILE, vb = tv + b * L::TILE;
@@ -296,20 +300,20 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 bwd_zero_rows<NP>(kb, rows, 128, lane);
                 fence_proxy_async_smem();
             }
-            const int ntiles = 1 + (g == 0) + (pass2 ? 1 : 0) + (g == nk_tiles);
+            const int ntiles = 1 + (g == g0) + (pass2 ? 1 : 0) + (g == nk_tiles);
             if (lane == 0) {
                 mbar_arrive_expect_tx(ld_full(b), ntiles * NP * rows * 128);
-                if (g == 0) bwd_load<NP>(p, KIND, &mq, tq, ld_full(b), bh, prob, qt);
+                if (g == g0) bwd_load<NP>(p, KIND, &mq, tq, ld_full(b), bh, prob, qt);
                 if (g == nk_tiles) bwd_load<NP>(p, KIND, &mdy, tdy, ld_full(b), bh, prob, qt);
                 bwd_load<NP>(p, KIND, &mk, kb, ld_full(b), bh, prob, jt);
                 if (pass2) bwd_load<NP>(p, KIND, &mvals, vb, ld_full(b), bh, prob, jt);
             }
             __syncwarp();
         };
-        issue_load(0);
-        for (int g = 0; g < ng && ok; ++g) {
-            const int b = g & 1;
-            if (g > 0) {
+        issue_load(g0);
+        for (int g = g0; g < ng && ok; ++g) {
+            const int b = (g - g0) & 1;
+            if (g > g0) {
                 if (g - 1 < nk_tiles) {  // pass-1 tile g-1: its S was read (its MMA is complete)
                     ok = mbar_wait_warp(ew_done, ew_par, ctl);
                     ew_par ^= 1u;
@@ -320,7 +324,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 if (!ok) break;
             }
             if (g + 1 < ng) issue_load(g + 1);  // into the buffer tile g-1 used
-            ok = mbar_wait_warp(ld_full(b), static_cast<uint32_t>(g >> 1) & 1u, ctl);
+            ok = mbar_wait_warp(ld_full(b), static_cast<uint32_t>((g - g0) >> 1) & 1u, ctl);
             if (!ok) break;
             tc_fence_after();
             const uint32_t kb = tk + b * L::TILE, vb = tv + b * L::TILE;
@@ -356,7 +360,9 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         uint32_t md_par = 0u;
         bool ok = true;
         float m_run = -INFINITY, l_run = 0.f;  // this half's running max and sum, base 2
-        for (int j = 0; j < nk_tiles && ok; ++j) {
+        // pass 1 (the row LSE), unless the forward's recomputation left it
+        const int nk_pass1 = p.lse_given ? 0 : nk_tiles;
+        for (int j = 0; j < nk_pass1 && ok; ++j) {
             ok = mbar_wait_warp(mma_done, md_par, ctl);
             md_par ^= 1u;
             if (!ok) break;
@@ -390,7 +396,9 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
         // the row's LSE from both halves' (max, sum), combined in the same
         // order by both, so both get the same bits
         float lse = 0.f;
-        if (ok) {
+        if (ok && p.lse_given) {
+            lse = rowg >= 0 ? p.lse[rowg] : 0.f;
+        } else if (ok) {
             float *xs = reinterpret_cast<float *>(base_ptr + L::OFF_LS);
             xs[(h * 128 + row) * 2] = m_run;
             xs[(h * 128 + row) * 2 + 1] = l_run;
@@ -407,7 +415,7 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
                 }
             }
         }
-        if (ok && h == 0 && rowg >= 0) p.lse[rowg] = lse;
+        if (ok && !p.lse_given && h == 0 && rowg >= 0) p.lse[rowg] = lse;
         for (int j = 0; j < nk_tiles && ok; ++j) {
             ok = mbar_wait_warp(mma_done, md_par, ctl);
             md_par ^= 1u;

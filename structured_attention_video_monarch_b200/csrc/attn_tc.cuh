@@ -85,6 +85,8 @@ struct TcParams {
     long long sB, sH, sN;           // element strides of batch, head and token (all four tensors)
     FastDiv fd_heads;               // batch-head index -> (batch, head)
     int out_v8;                     // out is 32-byte aligned: 32-byte epilogue stores
+    float *lse;                     // or null: per output row of the units of kind lse_kind, the
+    int lse_kind;                   // log2-sum-exp of its scaled logits, [BH][N] (for gradients)
 };
 
 struct Lane {
@@ -383,10 +385,12 @@ __device__ __forceinline__ void softmax_chunk(const float (&s)[64], uint64_t sca
     }
 }
 
-// PACK: stage-1 blocks pack sub-blocks of p.sub tokens (the packed rows pass of
-// the (f*h, w) split); a separate instantiation, so the other kernels carry
-// none of its masking.
-template <int D, bool F16, bool PACK>
+// Instantiations: TC_PLAIN; TC_PACK, stage-1 blocks pack sub-blocks of p.sub
+// tokens (the packed rows pass of the (f*h, w) split); TC_LSE, the row LSE of
+// the units of kind p.lse_kind is written to p.lse (the recomputations of the
+// gradients).  Separate instantiations, so the plain kernel carries neither.
+enum : int { TC_PLAIN = 0, TC_PACK = 1, TC_LSE = 2 };
+template <int D, bool F16, int MODE>
 __global__ void __launch_bounds__(640, 1)
 monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant__ CUtensorMap mk1,
                   const __grid_constant__ CUtensorMap mv1, const __grid_constant__ CUtensorMap mq2,
@@ -754,6 +758,7 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const int prow = (un.kind == UNIT_STAGE2) ? static_cast<int>(fmod_(row, p.fd_npos)) : 0;
             int npos_valid = 0;
             // packed stage-1 blocks: the first key of this row's sub-block
+            constexpr bool PACK = MODE == TC_PACK;
             const int sub_lo = (PACK && un.kind == UNIT_STAGE1)
                                    ? ((un.ln[li].tile * 128 + row) / p.sub) * p.sub : 0;
             if (un.kind == UNIT_STAGE2) {
@@ -862,6 +867,9 @@ monarch_tc_kernel(const __grid_constant__ CUtensorMap mq1, const __grid_constant
             const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
             int bh;
             const long long tok = lane_row_token(p, un.kind, un.ln[li], row, bh);
+            // log2 sum_k 2^(s_k * sl2) = m * sl2 + log2(l) for any running max m
+            if (MODE == TC_LSE && un.kind == p.lse_kind && h == 0 && tok >= 0)
+                p.lse[static_cast<long long>(bh) * p.N + tok] = m_run * sl2 + __log2f(l);
             const int ob = static_cast<int>(fdiv(static_cast<uint32_t>(bh), p.fd_heads)), oh = bh - ob * p.heads;
             uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + ob * p.sB + oh * p.sH +
                                                    (tok < 0 ? 0 : tok) * p.sN + h * (D / 2));

@@ -35,8 +35,8 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     bool init = false;
     int sms = 0;
-    bool tc_attr[8] = {};    // [packed rows][fp16][d == 128]
-    int tc_resident[8] = {};  // CTAs of monarch_tc_kernel per SM
+    bool tc_attr[12] = {};    // [mode][fp16][d == 128]
+    int tc_resident[12] = {};  // CTAs of monarch_tc_kernel per SM
     bool f32_attr[2] = {false, false};
 };
 
@@ -439,14 +439,19 @@ struct LaunchEvents {
 template <int D, bool F16>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
               cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr,
-              bool stage1_only = false, int sub = 0) {
+              bool stage1_only = false, int sub = 0, float *lse = nullptr,
+              int lse_kind = UNIT_STAGE1) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
     if ((st = get_encode())) return st;
     using L = TcLayout<D>;
-    const int di_idx = (sub > 0 ? 4 : 0) + (F16 ? 2 : 0) + (D == 128 ? 1 : 0);
-    const auto kernel = sub > 0 ? monarch_tc_kernel<D, F16, true> : monarch_tc_kernel<D, F16, false>;
+    const int mode = lse != nullptr ? TC_LSE : (sub > 0 ? TC_PACK : TC_PLAIN);
+    if (lse != nullptr && sub > 0) return MONARCH_ERR_UNSUPPORTED;
+    const int di_idx = mode * 4 + (F16 ? 2 : 0) + (D == 128 ? 1 : 0);
+    const auto kernel = mode == TC_LSE ? monarch_tc_kernel<D, F16, TC_LSE>
+                                       : (mode == TC_PACK ? monarch_tc_kernel<D, F16, TC_PACK>
+                                                          : monarch_tc_kernel<D, F16, TC_PLAIN>);
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!di->tc_attr[di_idx]) {
@@ -466,6 +471,8 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.N = s.N;
     p.fact = s.fact;
     p.sub = sub;
+    p.lse = lse;
+    p.lse_kind = lse_kind;
     if (s.fact == MONARCH_FACT_TILED) {
         p.tile_h = s.tile_h; p.tile_w = s.tile_w;
         p.tiles_h = s.H / s.tile_h; p.tiles_w = s.W / s.tile_w;
@@ -706,10 +713,11 @@ __global__ void bwd_rowdot(const E *a, const E *b, float *out, long long rows) {
     if (lane == 0) out[r] = s;
 }
 
-// Workspace (bytes): Y1, O, dY1 (16-bit, N*d each), LSE and D (fp32, N each),
-// stage 2's dq and dk parts (fp32, N*d each); per batch-head.
+// Workspace (bytes): Y1, O, dY1 (16-bit, N*d each), stage 2's LSE and the
+// row sums D (fp32, N each), stage 2's dq and dk parts (fp32, N*d each) and
+// stage 1's LSE (fp32, N); per batch-head.
 size_t bwd_tc_workspace(long long bh, long long N, int d, int es) {
-    return static_cast<size_t>(bh * N) * (3 * d * es + 2 * 4 + 2 * d * 4);
+    return static_cast<size_t>(bh * N) * (3 * d * es + 3 * 4 + 2 * d * 4);
 }
 
 // Geometry of one stage from a (possibly virtual) frame or tiled shape, and the
@@ -782,6 +790,7 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
     float *dd = lse + bh * N;
     float *dq32 = dd + bh * N;
     float *dk32 = dq32 + nd;
+    float *lse1 = dk32 + nd;
     const bool row = s.fact == MONARCH_FACT_ROW;
     // the two stages' shapes: the (f*h, w) split runs both as stage-1
     // geometries of virtual shapes (rows: one-row frames; columns: one tall
@@ -792,11 +801,12 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         s2.T = 1; s2.H = s.T * s.H; s2.fact = MONARCH_FACT_TILED; s2.tile_h = s.T * s.H; s2.tile_w = 1;
     }
     // recompute Y1 (stage 1 alone) and O (both stages; for the (f*h, w)
-    // split the columns pass over Y1)
-    if ((st = launch_tc<D, F16>(q, k, v, y1, s1, stream, lev, nullptr, true))) return st;
+    // split the columns pass over Y1); they also leave each stage's row LSE
+    // (stage 1's in lse1, stage 2's in lse), so the dQ kernels skip their LSE pass
+    if ((st = launch_tc<D, F16>(q, k, v, y1, s1, stream, lev, nullptr, true, 0, lse1, UNIT_STAGE1))) return st;
     if (row) {
-        if ((st = launch_tc<D, F16>(q, k, y1, o, s2, stream, lev, nullptr, true))) return st;
-    } else if ((st = launch_tc<D, F16>(q, k, v, o, s, stream, lev))) {
+        if ((st = launch_tc<D, F16>(q, k, y1, o, s2, stream, lev, nullptr, true, 0, lse, UNIT_STAGE1))) return st;
+    } else if ((st = launch_tc<D, F16>(q, k, v, o, s, stream, lev, nullptr, false, 0, lse, UNIT_STAGE2))) {
         return st;
     }
     unsigned *status = nullptr;
@@ -809,7 +819,8 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         BwdParams p{};
         TcParams tp{};
         bwd_geometry(s2, D, p, tp);
-        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 0; p.dk = dk32; p.add_dk = 0; p.dv16 = dy1;
+        p.lse = lse; p.lse_given = 1;
+        p.D = dd; p.dq = dq32; p.add_dq = 0; p.dk = dk32; p.add_dk = 0; p.dv16 = dy1;
         p.timeout_cycles = env_timeout_cycles();
         p.status = status;
         bwd_rowdot<D, E><<<rd_grid, 256, 0, stream>>>(static_cast<const E *>(dout), o, dd, rows);
@@ -835,7 +846,8 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         TcParams tp{};
         bwd_geometry(s1, D, p, tp);
         // adds stage 2's fp32 parts and writes the final 16-bit gradients
-        p.lse = lse; p.D = dd; p.dq = dq32; p.add_dq = 1; p.dk = dk32; p.add_dk = 1; p.dv16 = dv;
+        p.lse = lse1; p.lse_given = 1;
+        p.D = dd; p.dq = dq32; p.add_dq = 1; p.dk = dk32; p.add_dk = 1; p.dv16 = dv;
         p.out_dq = dq; p.out_dk = dk;
         p.timeout_cycles = env_timeout_cycles();
         p.status = status;

@@ -127,8 +127,8 @@ def test_noalloc_refuses_the_row_split_without_cuda(lib):
 def test_bwd_workspace_size_and_validation_without_cuda(lib):
     size = lib.monarch_attn_bwd_workspace_size
     assert size(1, 2, 3, 4, 5, 64, 0) == 2 * 1 * 2 * 3 * 4 * 5 * 64 * 4
-    # bf16 / fp16: 16-bit Y1, O, dY1, fp32 LSE and row sums, fp32 stage-2 dq/dk parts
-    assert size(1, 2, 3, 4, 5, 64, 1) == 2 * 60 * (3 * 64 * 2 + 2 * 4 + 2 * 64 * 4)
+    # bf16 / fp16: 16-bit Y1, O, dY1, fp32 row sums and both stages' LSE, fp32 stage-2 dq/dk parts
+    assert size(1, 2, 3, 4, 5, 64, 1) == 2 * 60 * (3 * 64 * 2 + 3 * 4 + 2 * 64 * 4)
     assert size(1, 2, 3, 4, 5, 64, 2) == size(1, 2, 3, 4, 5, 64, 1)
     assert size(1, 2, 3, 4, 5, 64, 3) == 0   # unknown dtype
     assert size(1, 2, 3, 4, 5, 96, 0) == 0   # unsupported head width
