@@ -454,10 +454,10 @@ def run_ours(args):
                 if events is None:
                     binding.monarch_attn_bwd(q, k, v, do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w,
                                              out=(dq, dk, dv), workspace=ws)
-                    return 8  # 2 recomputations, 2 x (row sums, dQ, dK/dV)
+                    return 6  # 2 recomputations, 2 x (row sums, dQ and dK/dV in one launch)
                 binding.monarch_attn_bwd_profiled(q, k, v, do, dq, dk, dv, ws, wl.T, wl.H, wl.W, events,
                                                   wl.fact, wl.tile_h, wl.tile_w)
-                return 8
+                return 6
             if events is not None:
                 events[0].record(stream)
             binding.monarch_attn_bwd(q, k, v, do, wl.T, wl.H, wl.W, wl.fact, wl.tile_h, wl.tile_w,
@@ -610,9 +610,9 @@ def run_ours(args):
         # frame blocks) carries 10*d FLOPs per (query, key) pair of the blocks.
         es, bhd = 2, wl.B * wl.heads * wl.d
         # bytes: read Q, K, V, dY1, Y1 (16-bit) and stage 2's dQ, dK parts (fp32); write dQ, dK, dV (16-bit)
-        b1 = rate("monarch_bwd_tc_stage1", f"monarch_bwd_dq + monarch_bwd_dkdv<{wl.d}> (stage-1 blocks of "
+        b1 = rate("monarch_bwd_tc_stage1", f"bwd_rowdot + monarch_bwd_pair<{wl.d}> (dQ and dK/dV CTAs; stage-1 blocks of "
                   f"m={wl.m})", 3, 10.0 * wl.N * wl.m * bhd, (5 * es + 2 * 4 + 3 * es) * wl.N * bhd)
-        b2 = rate("monarch_bwd_tc_stage2", f"monarch_bwd_dq + monarch_bwd_dkdv<{wl.d}> (stage-2 groups of "
+        b2 = rate("monarch_bwd_tc_stage2", f"bwd_rowdot + monarch_bwd_pair<{wl.d}> (dQ and dK/dV CTAs; stage-2 groups of "
                   f"b={wl.b})", 2, 10.0 * wl.N * wl.b * bhd, (5 * es + 2 * 4 + es) * wl.N * bhd)
         phase_ms = {}
         for name, idx in (("recompute_y1", 0), ("recompute_o", 1), ("stage2_bwd", 2), ("stage1_bwd", 3)):

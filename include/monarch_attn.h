@@ -316,9 +316,10 @@ int monarch_attn_fwd_chunk_profiled(const void *q, const void *k, const void *v,
  * recomputed Y1 and O and dY1 (16-bit), per-row rowsum terms and each
  * stage's per-row LSE (fp32) and stage 2's dQ and dK parts (fp32):
  * N*(6d + 12 + 8d) bytes per batch-head.  The forward's kernel recomputes Y1
- * and O, leaving each stage's row LSE as it goes; then per stage a
- * query-outer kernel (dQ) and a key-outer kernel (dK and dValues) run on
- * tcgen05 with fp32 accumulation and 16-bit P, dS and dY1; stage 1's kernels
+ * and O, leaving each stage's row LSE as it goes; then per stage the CTAs of
+ * a query-outer kernel (dQ) and of a key-outer kernel (dK and dValues) run,
+ * in one launch, on tcgen05 with fp32 accumulation and 16-bit P, dS and dY1;
+ * stage 1's kernels
  * add stage 2's parts and write dq, dk, dv.  Every gradient row has one
  * owning CTA, so the result is deterministic.  Limits as monarch_attn_fwd.
  *
@@ -342,8 +343,8 @@ size_t monarch_attn_bwd_workspace_size(int B, int heads, int T, int H, int W, in
  * (cudaEvent_t passed as void*, created by the caller) on `stream`:
  * events[0] before the first launch and events[i] after the i-th phase.
  * Phases, 16-bit dtypes: 1 Y1 recomputation, 2 O recomputation, 3 stage-2
- * backward (row sums, dQ kernel, dK/dV kernel), 4 stage-1 backward (the
- * same, writing dq, dk, dv); fp32: 1 the whole backward.  *nlaunch receives
+ * backward (row sums, then the dQ and dK/dV CTAs in one launch), 4 stage-1
+ * backward (the same, writing dq, dk, dv); fp32: 1 the whole backward.  *nlaunch receives
  * the number of phases recorded.  Events beyond `nevents` are not recorded.
  */
 int monarch_attn_bwd_profiled(const void *q, const void *k, const void *v, const void *dout,

@@ -54,6 +54,7 @@ struct BwdParams {
     float *dk;            // fp32 [BH][N][d]: written, or (add_dk) the other stage's part read
     void *dv16;           // value gradient in 16 bits [BH][N][d] (written), or null
     int add_dq, add_dk;
+    int pair_split;       // monarch_bwd_pair: CTAs [0, pair_split) run the dq body, the rest dk/dv
     // 16-bit final gradients [BH][N][d] (input dtype): when set, the kernel
     // adds the other stage's fp32 part and writes the result here
     void *out_dq, *out_dk;
@@ -228,10 +229,8 @@ __device__ __forceinline__ uint32_t bwd_pack(float lo, float hi) {
 // ------------------------------------------------------------------ dq kernel
 // grid: one CTA per (bh, problem, query tile).  Maps: q, k, vals, dy (same geometry).
 template <int D, bool F16, int KIND>
-__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
-monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-               const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
-               const BwdParams p) {
+__device__ __forceinline__ void bwd_dq_body(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mvals,
+                                            const CUtensorMap &mdy, const BwdParams &p, const int cta) {
     using L = BwdLayout<D>;
     constexpr int NP = L::NP;
     extern __shared__ uint8_t smem_raw[];
@@ -251,8 +250,8 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
     // problem decode
     const int nq_tiles = KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile;
     const int per_bh = (KIND == BWD_GEOM_STAGE2 ? p.s2_chunks : p.nblk_bh) * nq_tiles;
-    const int bh = blockIdx.x / per_bh;
-    const int rem = blockIdx.x - bh * per_bh;
+    const int bh = cta / per_bh;
+    const int rem = cta - bh * per_bh;
     const int prob = rem / nq_tiles, qt = rem - prob * nq_tiles;
     const int nk_tiles = nq_tiles;
 
@@ -497,10 +496,8 @@ monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ C
 // ------------------------------------------------------------------ dk/dv kernel
 // grid: one CTA per (bh, problem, key tile).  Maps: k, vals (A operands), q, dy.
 template <int D, bool F16, int KIND>
-__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
-monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                 const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
-                 const BwdParams p) {
+__device__ __forceinline__ void bwd_dkdv_body(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mvals,
+                                              const CUtensorMap &mdy, const BwdParams &p, const int cta) {
     using L = BwdLayout<D>;
     constexpr int NP = L::NP;
     extern __shared__ uint8_t smem_raw[];
@@ -519,8 +516,8 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
 
     const int nk_tiles = KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile;
     const int per_bh = (KIND == BWD_GEOM_STAGE2 ? p.s2_chunks : p.nblk_bh) * nk_tiles;
-    const int bh = blockIdx.x / per_bh;
-    const int rem = blockIdx.x - bh * per_bh;
+    const int bh = cta / per_bh;
+    const int rem = cta - bh * per_bh;
     const int prob = rem / nk_tiles, kt = rem - prob * nk_tiles;
     const int nq_tiles = nk_tiles;
 
@@ -721,6 +718,40 @@ monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// ------------------------------------------------------------------ launches
+// One CTA per (bh, problem, query tile).
+template <int D, bool F16, int KIND>
+__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
+monarch_bwd_dq(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+               const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
+               const BwdParams p) {
+    bwd_dq_body<D, F16, KIND>(mq, mk, mvals, mdy, p, static_cast<int>(blockIdx.x));
+}
+
+// One CTA per (bh, problem, key tile).
+template <int D, bool F16, int KIND>
+__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
+monarch_bwd_dkdv(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                 const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
+                 const BwdParams p) {
+    bwd_dkdv_body<D, F16, KIND>(mq, mk, mvals, mdy, p, static_cast<int>(blockIdx.x));
+}
+
+// Both kernels of a stage in one launch, for when the row LSE is given (the
+// dk/dv CTAs then need nothing the dq CTAs write): the second kernel's CTAs
+// fill the SMs the first one's last wave leaves idle.
+template <int D, bool F16, int KIND>
+__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
+monarch_bwd_pair(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                 const __grid_constant__ CUtensorMap mvals, const __grid_constant__ CUtensorMap mdy,
+                 const BwdParams p) {
+    const int cta = static_cast<int>(blockIdx.x);
+    if (cta < p.pair_split)
+        bwd_dq_body<D, F16, KIND>(mq, mk, mvals, mdy, p, cta);
+    else
+        bwd_dkdv_body<D, F16, KIND>(mq, mk, mvals, mdy, p, cta - p.pair_split);
 }
 
 }  // namespace monarch

@@ -758,6 +758,8 @@ int bwd_run_stage(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMa
             if (cudaFuncSetAttribute(monarch_bwd_dq<D, F16, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      LB::ALLOC) != cudaSuccess ||
                 cudaFuncSetAttribute(monarch_bwd_dkdv<D, F16, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     LB::ALLOC) != cudaSuccess ||
+                cudaFuncSetAttribute(monarch_bwd_pair<D, F16, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      LB::ALLOC) != cudaSuccess)
                 return MONARCH_ERR_CUDA;
             attr_done[dev] = true;
@@ -767,6 +769,13 @@ int bwd_run_stage(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMa
                              static_cast<long long>(KIND == BWD_GEOM_STAGE2 ? 1 : p.ntile);
     if (bh * per_bh >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
     const unsigned grid = static_cast<unsigned>(bh * per_bh);
+    if (p.lse_given) {  // dq and dk/dv CTAs in one launch
+        if (2ll * grid >= (1ll << 31)) return MONARCH_ERR_UNSUPPORTED;
+        BwdParams pp = p;
+        pp.pair_split = static_cast<int>(grid);
+        monarch_bwd_pair<D, F16, KIND><<<2 * grid, LB::THREADS, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, pp);
+        return cudaGetLastError() == cudaSuccess ? MONARCH_OK : MONARCH_ERR_LAUNCH;
+    }
     monarch_bwd_dq<D, F16, KIND><<<grid, LB::THREADS, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
     if (cudaGetLastError() != cudaSuccess) return MONARCH_ERR_LAUNCH;
     monarch_bwd_dkdv<D, F16, KIND><<<grid, LB::THREADS, LB::ALLOC, stream>>>(mq, mk, mvals, mdy, p);
