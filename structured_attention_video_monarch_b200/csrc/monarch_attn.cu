@@ -440,7 +440,7 @@ template <int D, bool F16>
 int launch_tc(const void *q, const void *k, const void *v, void *out, const Shape &s,
               cudaStream_t stream, LaunchEvents &lev, unsigned *fixed_counters = nullptr,
               bool stage1_only = false, int sub = 0, float *lse = nullptr,
-              int lse_kind = UNIT_STAGE1) {
+              int lse_kind = UNIT_STAGE1, bool stage2_only = false) {
     DeviceInfo *di = nullptr;
     int st = device_info(&di);
     if (st) return st;
@@ -503,15 +503,17 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     p.u1_bh = (p.nblk_bh / 2) * p.upg + (p.nblk_bh % 2) * (p.ns + p.odd);
     // stage 1 alone (Y1 into `out`): no stage-2 units
     if (stage1_only) p.s2_pairs = 0;
+    // stage 2 alone: no stage-1 units; the values (Y1) are `v`, the result goes to `out`
+    if (stage2_only) p.u1_bh = 0;
     const long long units = bh * (p.u1_bh + p.s2_pairs);
     if (units >= (1ll << 31) - 1) return MONARCH_ERR_UNSUPPORTED;
     p.units = static_cast<int>(units);
-    p.s1_target = static_cast<unsigned>(p.nblk_bh) * static_cast<unsigned>(p.nqt);
+    p.s1_target = stage2_only ? 0u : static_cast<unsigned>(p.nblk_bh) * static_cast<unsigned>(p.nqt);
     // Stage-2 units of a batch-head trail its stage-1 units by about two
     // waves of the persistent grid, so they rarely wait on their inputs.
     {
         const long long wave = di->sms;
-        long long lag = (2 * wave + p.u1_bh - 1) / p.u1_bh;
+        long long lag = p.u1_bh > 0 ? (2 * wave + p.u1_bh - 1) / p.u1_bh : 1;
         if (lag < 1) lag = 1;
         if (lag > bh || stage1_only) lag = bh;
         p.lag = static_cast<int>(lag);
@@ -543,7 +545,7 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     if (stage1_only) {  // no stage-2 units read them
         mq2 = mq1; mk2 = mk1; my2 = mv1;
     } else if ((st = stage2_map(&mq2, q, s, p)) || (st = stage2_map(&mk2, k, s, p)) ||
-               (st = stage2_map(&my2, out, s, p))) {
+               (st = stage2_map(&my2, stage2_only ? v : out, s, p))) {
         return st;
     }
 
@@ -809,13 +811,13 @@ int launch_bwd_tc(const void *q, const void *k, const void *v, const void *dout,
         s1.T = s.T * s.H; s1.H = 1; s1.fact = MONARCH_FACT_FRAME; s1.tile_h = s1.tile_w = 0;
         s2.T = 1; s2.H = s.T * s.H; s2.fact = MONARCH_FACT_TILED; s2.tile_h = s.T * s.H; s2.tile_w = 1;
     }
-    // recompute Y1 (stage 1 alone) and O (both stages; for the (f*h, w)
-    // split the columns pass over Y1); they also leave each stage's row LSE
+    // recompute Y1 (stage 1 alone) and O (stage 2 alone over that Y1; for the
+    // (f*h, w) split the columns pass over Y1); they also leave each stage's row LSE
     // (stage 1's in lse1, stage 2's in lse), so the dQ kernels skip their LSE pass
     if ((st = launch_tc<D, F16>(q, k, v, y1, s1, stream, lev, nullptr, true, 0, lse1, UNIT_STAGE1))) return st;
     if (row) {
         if ((st = launch_tc<D, F16>(q, k, y1, o, s2, stream, lev, nullptr, true, 0, lse, UNIT_STAGE1))) return st;
-    } else if ((st = launch_tc<D, F16>(q, k, v, o, s, stream, lev, nullptr, false, 0, lse, UNIT_STAGE2))) {
+    } else if ((st = launch_tc<D, F16>(q, k, y1, o, s, stream, lev, nullptr, false, 0, lse, UNIT_STAGE2, true))) {
         return st;
     }
     unsigned *status = nullptr;
