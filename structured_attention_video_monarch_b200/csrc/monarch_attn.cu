@@ -509,11 +509,13 @@ int launch_tc(const void *q, const void *k, const void *v, void *out, const Shap
     if (units >= (1ll << 31) - 1) return MONARCH_ERR_UNSUPPORTED;
     p.units = static_cast<int>(units);
     p.s1_target = stage2_only ? 0u : static_cast<unsigned>(p.nblk_bh) * static_cast<unsigned>(p.nqt);
-    // Stage-2 units of a batch-head trail its stage-1 units by about two
-    // waves of the persistent grid, so they rarely wait on their inputs.
+    // Stage-2 units of a batch-head trail its stage-1 units by about sixteen
+    // waves of the persistent grid (for the full clip: after every stage-1
+    // unit), so they never wait on their inputs and the CTAs run long stretches
+    // of one unit kind; a lag of two waves measured 3 % slower on the full clip.
     {
         const long long wave = di->sms;
-        long long lag = p.u1_bh > 0 ? (2 * wave + p.u1_bh - 1) / p.u1_bh : 1;
+        long long lag = p.u1_bh > 0 ? (16 * wave + p.u1_bh - 1) / p.u1_bh : 1;
         if (lag < 1) lag = 1;
         if (lag > bh || stage1_only) lag = bh;
         p.lag = static_cast<int>(lag);
