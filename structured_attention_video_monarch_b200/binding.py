@@ -87,8 +87,17 @@ def load_library(path: str | None = None):
     return lib
 
 
-def strerror(status: int) -> str:
+def monarch_attn_strerror(status: int) -> str:
+    """Text of a library status code."""
     return load_library().monarch_attn_strerror(int(status)).decode()
+
+
+def monarch_attn_version() -> int:
+    """Library version number."""
+    return int(load_library().monarch_attn_version())
+
+
+strerror = monarch_attn_strerror
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -164,11 +173,16 @@ def monarch_attn_fwd_strided(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
     return out
 
 
+def monarch_attn_bwd_workspace_size(B: int, heads: int, T: int, H: int, W: int, d: int, dtype: int) -> int:
+    """Workspace bytes monarch_attn_bwd needs for these sizes and dtype code (0 if unsupported)."""
+    return int(load_library().monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, int(dtype)))
+
+
 def monarch_attn_bwd_workspace(q, T: int, H: int, W: int) -> torch.Tensor:
     """A workspace for monarch_attn_bwd on tensors shaped and typed like q."""
     B, heads, N, d = q.shape
-    need = load_library().monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, _dtype_code(q))
-    return torch.empty(max(int(need), 16), dtype=torch.uint8, device=q.device)
+    need = monarch_attn_bwd_workspace_size(B, heads, T, H, W, d, _dtype_code(q))
+    return torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
 
 
 def monarch_attn_bwd(q, k, v, dout, T: int, H: int, W: int, factorisation: int = FACT_FRAME,
@@ -336,13 +350,21 @@ def monarch_attn_fwd_host_pipelined(h_q, h_k, h_v, h_out, d_q, d_k, d_v, d_out, 
         raise MonarchError(st, "monarch_attn_fwd_host_pipelined")
 
 
-def last_device_error(reset: bool = True, stream=None) -> int:
-    """Status word of the library's device-side waits (0 = none timed out)."""
+def monarch_attn_device_status(stream=None, reset: bool = True) -> int:
+    """Status word of the library's device-side waits (0 = none timed out); synchronises the stream."""
     return int(load_library().monarch_attn_device_status(_stream_ptr(stream), 1 if reset else 0))
 
 
-def selftest_timeout(limit_cycles: int, stream=None) -> int:
+def monarch_attn_selftest_timeout(limit_cycles: int, stream=None) -> int:
+    """Runs one bounded wait that nothing completes; returns the resulting status (4 = timed out)."""
     return int(load_library().monarch_attn_selftest_timeout(int(limit_cycles), _stream_ptr(stream)))
+
+
+def last_device_error(reset: bool = True, stream=None) -> int:
+    return monarch_attn_device_status(stream, reset)
+
+
+selftest_timeout = monarch_attn_selftest_timeout
 
 
 def monarch_attn_bwd_profiled(q, k, v, dout, dq, dk, dv, workspace, T, H, W, events,

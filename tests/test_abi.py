@@ -48,6 +48,18 @@ def test_strerror_and_version(lib):
         assert isinstance(s, str) and s
     assert binding.strerror(99) == "unknown status"
     assert lib.monarch_attn_version() >= 100
+    assert binding.monarch_attn_version() == lib.monarch_attn_version()
+
+
+def test_binding_has_every_declared_entry_point(lib):
+    """The Python binding wraps each C entry point under the header's own name."""
+    for name in declared_functions():
+        assert callable(getattr(binding, name, None)), f"{name} has no binding wrapper"
+
+
+def test_bwd_workspace_size_binding_matches_library(lib):
+    for args in [(2, 3, 4, 5, 6, 64, 1), (1, 1, 2, 2, 2, 128, 0), (1, 1, 2, 2, 2, 96, 1)]:
+        assert binding.monarch_attn_bwd_workspace_size(*args) == lib.monarch_attn_bwd_workspace_size(*args)
 
 
 def _call(lib, q=16, k=32, v=48, out=4096, B=1, heads=1, T=2, H=4, W=4, d=128, fact=0, th=0, tw=0,
